@@ -1,0 +1,493 @@
+"""Benchmark: one decode step over a Delta-KV cache on B200.
+
+A step is one pass of the whole hot path over one batch: append one new token
+per sequence (keyframe or closed-loop 4-bit delta, dkv_append) and one decode
+step of GQA attention over the whole compressed cache (dkv_decode_attn: the
+split kernel streaming the cache, then the log-sum-exp merge).  The headline
+workload is the Llama-3-70B-shaped single layer: batch 16, 64 query / 8 KV
+heads, head_dim 128, context 32768, kf 32, fp16 K/V, bf16 queries, synthetic
+random-walk data (the inputs are larger than L2: the compressed cache alone is
+652 MB per step).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun each rank runs its own replica of the workload on its own GPU
+(weak scaling, no collective on the data path); the time is the max over ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+if str(ROOT) not in sys.path:
+    sys.path.insert(0, str(ROOT))
+
+METRIC = "Delta-KV decode-attn HBM GB/s (% of peak) and KV-token·heads/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peak():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        try:
+            d = json.loads(p.read_text())
+            return float(d["hbm_gbs"]), "measured"
+        except Exception:
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kv_bytes(fmt: str, lens, Hkv: int, kf: int) -> int:
+    """Algorithmic bytes of K+V a decode step reads (compressed, per format)."""
+    tot = 0
+    for L in lens:
+        if fmt == "delta":
+            ng = -(-L // kf)
+            tot += Hkv * (ng * 512 + (L - ng) * 144)
+        elif fmt == "q4":
+            tot += Hkv * L * 144
+        else:
+            tot += Hkv * L * 512
+    return tot
+
+
+def encode_bytes(fmt: str, lens, Hkv: int, kf: int, in_elem: int) -> int:
+    """Encode traffic: read the K/V input once, write the compressed cache."""
+    return sum(Hkv * L * 2 * 128 * in_elem for L in lens) + kv_bytes(fmt, lens, Hkv, kf)
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (getattr(self, "out", "") or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        smax = max(r[1] for r in rows)
+        load = [r for r in rows if r[0] > 0.5 * smax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# distributed helpers (also exercised by the gloo tests on CPU)
+# ---------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on the host cores, on a bounded sample
+# ---------------------------------------------------------------------------
+def cpu_oracle_sample(w, budget_s: float = 12.0, max_seqs: int = 64):
+    """Time the oracle's decode step (reconstruction from the stored codes +
+    binary64 attention) on whole (batch, kv-head) sequences of the workload
+    until ~budget_s of CPU work; returns (GB/s, token.heads/s, description)."""
+    import numpy as np
+    import oracle
+    import synthetic as S
+    oracle.build()
+    G = w.Hq // w.Hkv
+    scale = 1.0 / math.sqrt(w.D)
+    t_total, nbytes, units, nseq = 0.0, 0, 0, 0
+    b = 0
+    while t_total < budget_s and nseq < max_seqs:
+        K, V = S.gen_kv_one(w, b, w.T)
+        q = S.gen_q(w)[b].double().numpy()
+        for h in range(w.Hkv):
+            if t_total >= budget_s or nseq >= max_seqs:
+                break
+            k = K[h].float().numpy()
+            v = V[h].float().numpy()
+            ek = oracle.delta_encode(k, w.kf)          # builds the stored fields (untimed)
+            ev = oracle.delta_encode(v, w.kf)
+            t0 = time.perf_counter()
+            kh = oracle.delta_decode(w.T, w.kf, ek.kfr, ek.scales, ek.codes)
+            vh = oracle.delta_decode(w.T, w.kf, ev.kfr, ev.scales, ev.codes)
+            oracle.attn(q[h * G:(h + 1) * G], kh, vh, scale)
+            t_total += time.perf_counter() - t0
+            nbytes += kv_bytes("delta", [w.T], 1, w.kf)
+            units += w.T
+            nseq += 1
+        b += 1
+    desc = (f"{nseq} whole (batch, kv-head) sequences of {w.name} (T={w.T}, kf={w.kf}, G={G}): "
+            f"reconstruction from stored codes + binary64 attention, {t_total:.1f} s single-threaded")
+    return nbytes / t_total / 1e9, units / t_total, desc, t_total
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    import oracle
+    import synthetic as S
+    oracle.build()
+    G = w.Hq // w.Hkv
+    K, V = S.gen_kv_one(w, 0, w.T)
+    q = S.gen_q(w)[0].double().numpy()
+    k, v = K[0].float().numpy(), V[0].float().numpy()
+    ek = oracle.delta_encode(k, w.kf)
+    ev = oracle.delta_encode(v, w.kf)
+    per = []
+    for i in range(warm + steps):
+        t0 = time.perf_counter()
+        kh = oracle.delta_decode(w.T, w.kf, ek.kfr, ek.scales, ek.codes)
+        vh = oracle.delta_decode(w.T, w.kf, ev.kfr, ev.scales, ev.codes)
+        oracle.attn(q[:G], kh, vh, 1.0 / math.sqrt(w.D))
+        if i >= warm:
+            per.append(time.perf_counter() - t0)
+    t = sum(per)
+    nbytes = kv_bytes("delta", [w.T], 1, w.kf) * steps
+    val = nbytes / t / 1e9
+    sample = (f"each step: one (batch, kv-head) sequence of {w.name} (T={w.T}, kf={w.kf}, "
+              f"{G} query heads): reconstruction from stored codes + binary64 attention")
+    line = {"metric": METRIC, "value": val, "unit": "GB/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": steps, "warmup": warm,
+            "ms_per_step": 1e3 * t / steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv,
+                       "head_dim": w.D, "context": w.T, "kf": w.kf},
+            "kv_token_heads_per_s": w.T * steps / t,
+            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args, w, rank, world, local):
+    import torch
+    import delta_quantized_kv_b200 as dkv
+    import synthetic as S
+
+    from delta_quantized_kv_b200 import build as _b
+    if rank == 0 and _b.stale():
+        _b.build()
+    barrier(world)
+    dkv.load()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    W, K = args.warmup, args.steps
+    n_app = W + K                        # appended tokens, device-timed loop
+    n_e2e = W + K                        # appended tokens, end-to-end loop
+    T0 = w.T
+    cap = T0 + n_app + n_e2e + 8
+    B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
+    scale = 1.0 / math.sqrt(D)
+
+    # ---- inputs (generated on the device, then only the cache stays) -------
+    torch.manual_seed(1234 + rank)
+    K_all = torch.empty((B, Hkv, T0 + n_app + n_e2e, D), dtype=w.kv_dtype, device=dev)
+    V_all = torch.empty_like(K_all)
+    for b in range(B):
+        K_all[b], V_all[b] = S.gen_kv_one(w, b, T0 + n_app + n_e2e, device=dev)
+    Kp, Vp = K_all[:, :, :T0].contiguous(), V_all[:, :, :T0].contiguous()
+    app_k = [K_all[:, :, T0 + i:T0 + i + 1].contiguous() for i in range(n_app + n_e2e)]
+    app_v = [V_all[:, :, T0 + i:T0 + i + 1].contiguous() for i in range(n_app + n_e2e)]
+    del K_all, V_all
+    qs = [S.gen_q(w, device=dev, step=i) for i in range(n_app + n_e2e)]
+    in_elem = torch.finfo(w.kv_dtype).bits // 8
+
+    res = {}
+    # ---- encode throughput (prefill of the whole context) --------------------
+    cache = dkv.Cache(B, Hkv, cap, args.fmt, kf=w.kf, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    enc_ms = []
+    for i in range(3):
+        ev[0].record(stream)
+        cache.encode(Kp, Vp)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        enc_ms.append(ev[0].elapsed_time(ev[1]))
+    enc_t = min(enc_ms[1:])
+    res["encode"] = {"ms": enc_t, "gbps": encode_bytes(args.fmt, [T0] * B, Hkv, w.kf, in_elem)
+                     / (enc_t * 1e-3) / 1e9}
+
+    ws = cache.workspace(Hq)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    qcode = dkv._dtype_code(w.q_dtype)
+    wsb = ws.numel() * 4
+
+    def step(i):
+        cache.append(app_k[i], app_v[i])
+        dkv.dkv_decode_attn_split(cache.c, qs[i], qcode, Hq, scale, ws, wsb, stream)
+        dkv.dkv_decode_attn_merge(cache.c, Hq, out, ws, wsb, stream)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    # per-step events: [append | split | merge]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lens = []
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        barrier(world)
+        e_start.record(stream)
+        for k in range(K):
+            i = W + k
+            e = evs[k]
+            e[0].record(stream)
+            cache.append(app_k[i], app_v[i])
+            e[1].record(stream)
+            dkv.dkv_decode_attn_split(cache.c, qs[i], qcode, Hq, scale, ws, wsb, stream)
+            e[2].record(stream)
+            dkv.dkv_decode_attn_merge(cache.c, Hq, out, ws, wsb, stream)
+            e[3].record(stream)
+            lens.append(T0 + i + 1)
+        e_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    status = cache.device_status()
+    total_ms = e_start.elapsed_time(e_end)
+    total_ms = max_over_ranks(total_ms, world, dev)
+    split_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    app_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    merge_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    bytes_steps = sum(kv_bytes(args.fmt, [L] * B, Hkv, w.kf) for L in lens)
+    units_steps = sum(L * B * Hkv for L in lens)
+    value = world * bytes_steps / (total_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    split_avg = sum(split_ms) / K
+    bytes_avg = bytes_steps / K
+
+    # ---- end to end through the public API with host buffers ------------------
+    pin_k = [t.cpu().pin_memory() for t in app_k[n_app:]]
+    pin_v = [t.cpu().pin_memory() for t in app_v[n_app:]]
+    pin_q = [t.cpu().pin_memory() for t in qs[n_app:]]
+    dk = torch.empty_like(app_k[0]); dv = torch.empty_like(app_v[0]); dq = torch.empty_like(qs[0])
+    host_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
+    h2d = pin_k[0].numel() * pin_k[0].element_size() * 2 + pin_q[0].numel() * pin_q[0].element_size()
+    d2h = host_out.numel() * 4
+
+    def e2e_step(j):
+        dk.copy_(pin_k[j], non_blocking=True)
+        dv.copy_(pin_v[j], non_blocking=True)
+        dq.copy_(pin_q[j], non_blocking=True)
+        cache.append(dk, dv)
+        cache.decode_attn(dq, scale, out=out)
+        host_out.copy_(out, non_blocking=True)
+
+    for j in range(W):
+        e2e_step(j)
+    torch.cuda.synchronize()
+    barrier(world)
+    lens2 = []
+    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0e.record(stream)
+    for k in range(K):
+        e2e_step(W + k)
+        lens2.append(T0 + n_app + W + k + 1)
+    t1e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0e.elapsed_time(t1e), world, dev)
+    e2e_val = world * sum(kv_bytes(args.fmt, [L] * B, Hkv, w.kf) for L in lens2) / (e2e_ms * 1e-3) / 1e9
+
+    # ---- comparators and MSE (rank 0 only, outside the timed region) ----------
+    extra = {}
+    if rank == 0 and args.comparators and args.fmt == "delta":
+        for fmt in ("fp16", "q4"):
+            cc = dkv.Cache(B, Hkv, T0, fmt, kf=w.kf, device=dev)
+            cc.encode(Kp, Vp)
+            wsc = cc.workspace(Hq)
+            for _ in range(3):
+                cc.decode_attn(qs[0], scale, out=out)
+            torch.cuda.synchronize()
+            a, bq = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = max(5, K)
+            a.record(stream)
+            for i in range(n):
+                dkv.dkv_decode_attn_split(cc.c, qs[i % len(qs)], qcode, Hq, scale, wsc,
+                                          wsc.numel() * 4, stream)
+            bq.record(stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(bq) / n
+            nb = kv_bytes(fmt, [T0] * B, Hkv, w.kf)
+            extra[fmt] = {"split_us": 1e3 * t, "bytes": nb, "gbps": nb / (t * 1e-3) / 1e9,
+                          "speedup_delta_vs": t / split_avg}
+            del cc
+        # reconstruction MSE on a slice (first 2 batch entries)
+        nb_ = min(2, B)
+        xs = {"K": Kp[:nb_].float(), "V": Vp[:nb_].float()}
+        mse = {}
+        for fmt in ("delta", "q4", "fp16"):
+            cc = dkv.Cache(nb_, Hkv, T0, fmt, kf=w.kf, device=dev)
+            cc.encode(Kp[:nb_].contiguous(), Vp[:nb_].contiguous())
+            xh = cc.dequantize()
+            errs = [((xh[:, :, t, :T0] - xs[n]) ** 2).mean().item() for t, n in enumerate("KV")]
+            pw = [(xs[n] ** 2).mean().item() for n in "KV"]
+            mse[fmt] = {"mse": sum(errs) / 2, "rel": sum(errs) / sum(pw)}
+            del cc, xh
+        res["mse"] = mse
+    torch.cuda.synchronize()
+
+    if rank != 0:
+        return
+    cpu = None
+    if args.cpu_baseline:
+        gbps, tps, desc, tcpu = cpu_oracle_sample(w, budget_s=args.cpu_budget)
+        cpu = {"value": gbps, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
+               "kv_token_heads_per_s": tps}
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv,
+                   "head_dim": D, "context": T0, "kf": w.kf, "format": args.fmt,
+                   "kv_dtype": str(w.kv_dtype).replace("torch.", ""),
+                   "q_dtype": str(w.q_dtype).replace("torch.", ""),
+                   "step": "dkv_append (1 token/seq) + dkv_decode_attn (split + merge)",
+                   "l2": "no flush: the compressed cache read per step exceeds the 126 MB L2",
+                   "parallelism": f"replica x{world}"},
+        "pct_of_peak": {"measured": 100.0 * value / world / peak, "nominal_8TBs": 100.0 * value / world / NOMINAL_HBM_GBS,
+                        "peak_kind": peak_kind},
+        "kv_token_heads_per_s": world * units_steps / (total_ms * 1e-3),
+        "query_token_heads_per_s": world * units_steps * (Hq // Hkv) / (total_ms * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": bytes_avg / (split_avg * 1e-3) / 1e9,
+                     "peak": peak, "unit": "GB/s",
+                     "frac": bytes_avg / (split_avg * 1e-3) / 1e9 / peak,
+                     "traffic": None, "kernel": "split_kernel (decode split)",
+                     "peak_kind": f"{peak_kind} (copy bandwidth, MEASURED_PEAKS hbm_gbs)"},
+        "kernels_us": {"append": 1e3 * sum(app_ms) / K, "split": 1e3 * split_avg,
+                       "merge": 1e3 * sum(merge_ms) / K},
+        "encode": res["encode"],
+        "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+        "device_status": status,
+        "cpu_baseline": cpu,
+    }
+    if extra:
+        line["comparators"] = extra
+    if "mse" in res:
+        line["mse"] = res["mse"]
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama3_70b_layer")
+    ap.add_argument("--kf", type=int, default=None)
+    ap.add_argument("--fmt", default="delta", choices=["delta", "q4", "fp16"])
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--context", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-comparators", dest="comparators", action="store_false")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+
+    import synthetic as S
+    w = S.WORKLOADS[args.workload]
+    if args.kf:
+        w = w.with_(kf=args.kf)
+    if args.batch:
+        w = w.with_(B=args.batch)
+    if args.context:
+        w = w.with_(T=args.context)
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if args.impl == "reference" and rank != 0:
+            return 0
+        if args.impl == "ours":
+            import torch
+            torch.cuda.set_device(local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, rank, world)
+        else:
+            run_ours(args, w, rank, world, local)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,286 @@
+"""Python binding of the Delta-KV decode library (``include/dkv.h``).
+
+Argument marshalling only: every step of the encode, append and decode path
+runs in the library's CUDA kernels (``_lib/libdkv.so``, built for sm_100a).
+PyTorch is used for device memory and streams.  If the shared library is
+missing, every call raises -- there is no CPU fallback.
+
+The functions carry the C names (``dkv_encode`` ...) and take either raw
+integers (device pointers, a stream handle) or torch tensors / streams.
+``Cache`` is a small convenience that allocates a cache with torch and keeps
+its ``dkv_cache`` descriptor.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "_lib" / "libdkv.so"
+
+DKV_OK, DKV_EINVAL, DKV_EALIGN, DKV_ECAPACITY, DKV_EUNSUPPORTED, DKV_ECUDA, DKV_EDEVICE = range(7)
+DKV_FMT_FP16, DKV_FMT_Q4_0, DKV_FMT_DELTA = 0, 1, 2
+DKV_F32, DKV_F16, DKV_BF16 = 0, 1, 2
+DEV_BAD_SEQLEN, DEV_CAPACITY, DEV_TIMEOUT, DEV_BAD_HEADS = 0x1, 0x2, 0x4, 0x8
+FORMATS = {"fp16": DKV_FMT_FP16, "q4": DKV_FMT_Q4_0, "delta": DKV_FMT_DELTA}
+
+
+class DkvError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)} ({status})")
+
+
+class dkv_cache_desc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("kf", ctypes.c_int32),
+                ("max_ctx", ctypes.c_int32), ("fmt", ctypes.c_int32)]
+
+
+class dkv_cache(ctypes.Structure):
+    _fields_ = [("desc", dkv_cache_desc), ("base", ctypes.c_void_p), ("bytes", ctypes.c_size_t),
+                ("seq_stride", ctypes.c_size_t), ("rec_bytes", ctypes.c_size_t),
+                ("n_groups", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+                ("off_data", ctypes.c_size_t), ("off_state", ctypes.c_size_t),
+                ("off_seqlen", ctypes.c_size_t), ("off_header", ctypes.c_size_t)]
+
+
+_lib = None
+EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode", "dkv_append",
+           "dkv_decode_workspace_bytes", "dkv_decode_attn", "dkv_decode_attn_split",
+           "dkv_decode_attn_merge", "dkv_export_canonical", "dkv_dequantize",
+           "dkv_get_device_status", "dkv_status_str"]
+
+
+def load():
+    """Load ``libdkv.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise RuntimeError(f"libdkv.so not built ({LIB_PATH}); run __graft_entry__.build() "
+                           "or python -m delta_quantized_kv_b200.build")
+    lib = ctypes.CDLL(str(LIB_PATH))
+    P, S, I, F = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_float
+    PC = ctypes.POINTER(dkv_cache)
+    PD = ctypes.POINTER(dkv_cache_desc)
+    sig = {
+        "dkv_abi_version": ([], I),
+        "dkv_cache_bytes": ([PD], S),
+        "dkv_cache_init": ([PD, P, S, PC, P], I),
+        "dkv_encode": ([PC, P, P, I, P, I, P], I),
+        "dkv_append": ([PC, P, P, I, I, P], I),
+        "dkv_decode_workspace_bytes": ([PD, I], S),
+        "dkv_decode_attn": ([PC, P, I, I, F, P, P, S, P], I),
+        "dkv_decode_attn_split": ([PC, P, I, I, F, P, S, P], I),
+        "dkv_decode_attn_merge": ([PC, I, P, P, S, P], I),
+        "dkv_export_canonical": ([PC, P, P, P, P, P], I),
+        "dkv_dequantize": ([PC, P, P], I),
+        "dkv_get_device_status": ([PC, ctypes.POINTER(I), P], I),
+        "dkv_status_str": ([I], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def status_str(s: int) -> str:
+    return load().dkv_status_str(int(s)).decode()
+
+
+def _ptr(x):
+    """Device pointer of a tensor (or an int / None)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.float32: DKV_F32, torch.float16: DKV_F16, torch.bfloat16: DKV_BF16}[t]
+
+
+def _check(s: int, what: str):
+    if s != DKV_OK:
+        raise DkvError(s, what)
+
+
+# ---------------------------------------------------------------------------
+# the C functions, same names
+# ---------------------------------------------------------------------------
+def dkv_abi_version() -> int:
+    return load().dkv_abi_version()
+
+
+def dkv_cache_bytes(desc: dkv_cache_desc) -> int:
+    return load().dkv_cache_bytes(ctypes.byref(desc))
+
+
+def dkv_cache_init(desc: dkv_cache_desc, dev, nbytes: int, stream=None) -> dkv_cache:
+    out = dkv_cache()
+    _check(load().dkv_cache_init(ctypes.byref(desc), _ptr(dev), nbytes, ctypes.byref(out),
+                                 _stream(stream)), "dkv_cache_init")
+    return out
+
+
+def dkv_encode(cache: dkv_cache, K, V, dtype=None, seq_lens=None, T=None, stream=None) -> None:
+    dtype = _dtype_code(K.dtype) if dtype is None else dtype
+    T = K.shape[2] if T is None else T
+    _check(load().dkv_encode(ctypes.byref(cache), _ptr(K), _ptr(V), dtype, _ptr(seq_lens), T,
+                             _stream(stream)), "dkv_encode")
+
+
+def dkv_append(cache: dkv_cache, K_new, V_new, dtype=None, n_new=None, stream=None) -> None:
+    dtype = _dtype_code(K_new.dtype) if dtype is None else dtype
+    n_new = K_new.shape[2] if n_new is None else n_new
+    _check(load().dkv_append(ctypes.byref(cache), _ptr(K_new), _ptr(V_new), dtype, n_new,
+                             _stream(stream)), "dkv_append")
+
+
+def dkv_decode_workspace_bytes(desc: dkv_cache_desc, n_q_heads: int) -> int:
+    return load().dkv_decode_workspace_bytes(ctypes.byref(desc), n_q_heads)
+
+
+def dkv_decode_attn(cache: dkv_cache, Q, q_dtype, n_q_heads, softmax_scale, out, workspace,
+                    ws_bytes, stream=None) -> None:
+    _check(load().dkv_decode_attn(ctypes.byref(cache), _ptr(Q), q_dtype, n_q_heads,
+                                  softmax_scale, _ptr(out), _ptr(workspace), ws_bytes,
+                                  _stream(stream)), "dkv_decode_attn")
+
+
+def dkv_decode_attn_split(cache: dkv_cache, Q, q_dtype, n_q_heads, softmax_scale, workspace,
+                          ws_bytes, stream=None) -> None:
+    _check(load().dkv_decode_attn_split(ctypes.byref(cache), _ptr(Q), q_dtype, n_q_heads,
+                                        softmax_scale, _ptr(workspace), ws_bytes,
+                                        _stream(stream)), "dkv_decode_attn_split")
+
+
+def dkv_decode_attn_merge(cache: dkv_cache, n_q_heads, out, workspace, ws_bytes,
+                          stream=None) -> None:
+    _check(load().dkv_decode_attn_merge(ctypes.byref(cache), n_q_heads, _ptr(out),
+                                        _ptr(workspace), ws_bytes, _stream(stream)),
+           "dkv_decode_attn_merge")
+
+
+def dkv_export_canonical(cache: dkv_cache, codes=None, scales=None, keyframes=None, state=None,
+                         stream=None) -> None:
+    _check(load().dkv_export_canonical(ctypes.byref(cache), _ptr(codes), _ptr(scales),
+                                       _ptr(keyframes), _ptr(state), _stream(stream)),
+           "dkv_export_canonical")
+
+
+def dkv_dequantize(cache: dkv_cache, out, stream=None) -> None:
+    _check(load().dkv_dequantize(ctypes.byref(cache), _ptr(out), _stream(stream)),
+           "dkv_dequantize")
+
+
+def dkv_get_device_status(cache: dkv_cache, stream=None) -> int:
+    word = ctypes.c_int32(0)
+    s = load().dkv_get_device_status(ctypes.byref(cache), ctypes.byref(word), _stream(stream))
+    if s not in (DKV_OK, DKV_EDEVICE):
+        raise DkvError(s, "dkv_get_device_status")
+    return word.value
+
+
+# ---------------------------------------------------------------------------
+# convenience wrapper (torch allocations)
+# ---------------------------------------------------------------------------
+class Cache:
+    """A Delta-KV (or comparator) cache in torch-allocated device memory."""
+
+    def __init__(self, batch, n_kv_heads, max_ctx, fmt="delta", kf=32, head_dim=128,
+                 device="cuda", stream=None):
+        import torch
+        self.desc = dkv_cache_desc(batch, n_kv_heads, head_dim, kf, max_ctx,
+                                   FORMATS[fmt] if isinstance(fmt, str) else fmt)
+        nbytes = dkv_cache_bytes(self.desc)
+        if nbytes == 0:
+            raise DkvError(DKV_EINVAL, "dkv_cache_bytes")
+        self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        base = (self.buf.data_ptr() + 255) // 256 * 256
+        self.c = dkv_cache_init(self.desc, base, nbytes, stream)
+        self._ws = None
+        self._ws_heads = None
+        self.device = device
+
+    @property
+    def fmt(self):
+        return self.desc.fmt
+
+    def encode(self, K, V, seq_lens=None, stream=None):
+        dkv_encode(self.c, K, V, seq_lens=seq_lens, stream=stream)
+
+    def append(self, K_new, V_new, stream=None):
+        dkv_append(self.c, K_new, V_new, stream=stream)
+
+    def workspace(self, n_q_heads):
+        import torch
+        if self._ws is None or self._ws_heads != n_q_heads:
+            nb = dkv_decode_workspace_bytes(self.desc, n_q_heads)
+            if nb == 0:
+                raise DkvError(DKV_ECUDA, "dkv_decode_workspace_bytes")
+            self._ws = torch.empty(nb // 4 + 64, dtype=torch.float32, device=self.device)
+            self._ws_heads = n_q_heads
+        return self._ws
+
+    def decode_attn(self, Q, softmax_scale, out=None, stream=None):
+        import torch
+        B, Hq, Dh = Q.shape
+        if out is None:
+            out = torch.empty((B, Hq, Dh), dtype=torch.float32, device=Q.device)
+        ws = self.workspace(Hq)
+        dkv_decode_attn(self.c, Q, _dtype_code(Q.dtype), Hq, softmax_scale, out, ws,
+                        ws.numel() * 4, stream)
+        return out
+
+    def seq_lens(self):
+        import torch
+        n = self.desc.batch
+        base = self.c.base + self.c.off_seqlen
+        off = base - self.buf.data_ptr()
+        return self.buf[off:off + 4 * n].view(torch.int32).clone()
+
+    def export(self, stream=None):
+        """Canonical fields as torch tensors (codes, scales, keyframes, state)."""
+        import torch
+        d = self.desc
+        B, H, cap = d.batch, d.n_kv_heads, d.max_ctx
+        dev = self.device
+        out = {}
+        if d.fmt in (DKV_FMT_DELTA, DKV_FMT_Q4_0):
+            out["codes"] = torch.zeros((B, H, 2, cap, 128), dtype=torch.uint8, device=dev)
+            out["scales"] = torch.zeros((B, H, 2, cap, 4), dtype=torch.int16, device=dev)
+        if d.fmt == DKV_FMT_DELTA:
+            out["keyframes"] = torch.zeros((B, H, 2, self.c.n_groups, 128), dtype=torch.int16,
+                                           device=dev)
+            out["state"] = torch.zeros((B, H, 2, 128), dtype=torch.float32, device=dev)
+        if d.fmt == DKV_FMT_FP16:
+            out["keyframes"] = torch.zeros((B, H, 2, cap, 128), dtype=torch.int16, device=dev)
+        dkv_export_canonical(self.c, out.get("codes"), out.get("scales"), out.get("keyframes"),
+                             out.get("state"), stream)
+        return out
+
+    def dequantize(self, stream=None):
+        import torch
+        d = self.desc
+        out = torch.zeros((d.batch, d.n_kv_heads, 2, d.max_ctx, 128), dtype=torch.float32,
+                          device=self.device)
+        dkv_dequantize(self.c, out, stream)
+        return out
+
+    def device_status(self, stream=None) -> int:
+        return dkv_get_device_status(self.c, stream)

@@ -1,0 +1,274 @@
+// dkv_api.cu -- the C ABI (include/dkv.h): argument validation, cache layout,
+// and the launches.  Nothing here allocates device memory; every launch goes
+// on the caller's stream.
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/dkv.h"
+#include "dkv_common.cuh"
+#include "dkv_internal.h"
+
+namespace {
+
+using dkv::CacheView;
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+struct Layout {
+    size_t seq_stride, rec_bytes, off_data, off_state, off_seqlen, off_header, total;
+    int32_t n_groups;
+};
+
+dkv_status check_desc(const dkv_cache_desc *d) {
+    if (!d) return DKV_EINVAL;
+    if (d->fmt != DKV_FMT_FP16 && d->fmt != DKV_FMT_Q4_0 && d->fmt != DKV_FMT_DELTA)
+        return DKV_EINVAL;
+    if (d->batch < 1 || d->batch > 1024 || d->n_kv_heads < 1 || d->n_kv_heads > 4096)
+        return DKV_EINVAL;
+    if (d->max_ctx < 1 || d->max_ctx > (1 << 28)) return DKV_EINVAL;
+    if (d->fmt == DKV_FMT_DELTA && (d->kf < 1 || d->kf > (1 << 20))) return DKV_EINVAL;
+    if (d->head_dim != dkv::D) return DKV_EUNSUPPORTED;
+    return DKV_OK;
+}
+
+Layout make_layout(const dkv_cache_desc *d) {
+    Layout L{};
+    const size_t cap = (size_t)d->max_ctx;
+    if (d->fmt == DKV_FMT_DELTA) {
+        L.rec_bytes = (size_t)dkv::delta_rec_bytes(d->kf);
+        L.n_groups = (int32_t)((cap + d->kf - 1) / d->kf);
+        L.seq_stride = L.rec_bytes * (size_t)L.n_groups;
+    } else if (d->fmt == DKV_FMT_Q4_0) {
+        L.rec_bytes = 0;
+        L.n_groups = 0;
+        L.seq_stride = cap * dkv::POS_Q4;
+    } else {
+        L.rec_bytes = 0;
+        L.n_groups = 0;
+        L.seq_stride = cap * dkv::POS_F16;
+    }
+    const size_t nseq = (size_t)d->batch * d->n_kv_heads;
+    L.off_data = 0;
+    L.off_state = align_up(nseq * L.seq_stride + 4096, kAlign);
+    L.off_seqlen = align_up(L.off_state + 2 * nseq * 2 * dkv::D * sizeof(float), kAlign);
+    L.off_header = align_up(L.off_seqlen + (size_t)d->batch * sizeof(int32_t), kAlign);
+    L.total = align_up(L.off_header + 16, kAlign);
+    return L;
+}
+
+dkv_status check_cache(const dkv_cache *c) {
+    if (!c || !c->base) return DKV_EINVAL;
+    dkv_status s = check_desc(&c->desc);
+    if (s != DKV_OK) return s;
+    Layout L = make_layout(&c->desc);
+    if (c->bytes < L.total || c->seq_stride != L.seq_stride || c->off_header != L.off_header)
+        return DKV_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(c->base) & (kAlign - 1)) != 0) return DKV_EALIGN;
+    return DKV_OK;
+}
+
+CacheView view_of(const dkv_cache *c) {
+    CacheView v;
+    uint8_t *base = static_cast<uint8_t *>(c->base);
+    v.data = base + c->off_data;
+    v.state = reinterpret_cast<float *>(base + c->off_state);
+    v.seqlen = reinterpret_cast<int32_t *>(base + c->off_seqlen);
+    v.header = reinterpret_cast<int32_t *>(base + c->off_header);
+    v.seq_stride = (int64_t)c->seq_stride;
+    v.rec_bytes = (int64_t)c->rec_bytes;
+    v.B = c->desc.batch;
+    v.Hkv = c->desc.n_kv_heads;
+    v.kf = c->desc.fmt == DKV_FMT_DELTA ? c->desc.kf : 1;
+    v.cap = c->desc.max_ctx;
+    v.fmt = c->desc.fmt;
+    v.n_groups = c->n_groups;
+    return v;
+}
+
+inline dkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DKV_OK : DKV_ECUDA; }
+
+inline bool valid_dtype(int32_t t) { return t == DKV_F32 || t == DKV_F16 || t == DKV_BF16; }
+
+int64_t workspace_floats(const dkv_cache_desc *d, int32_t Hq, bool *ok) {
+    *ok = false;
+    if (check_desc(d) != DKV_OK || Hq < 1 || Hq % d->n_kv_heads != 0) return 0;
+    dkv::SplitGeom g;
+    if (dkv::split_geometry(d->fmt, d->kf, d->batch, &g) != cudaSuccess) return 0;
+    const int G = Hq / d->n_kv_heads;
+    const int64_t nhg = (G + 7) / 8;
+    const int64_t slots = (int64_t)g.ctas * g.warps_per_cta + (int64_t)d->batch * d->n_kv_heads * nhg;
+    *ok = true;
+    return slots * dkv::PARTIAL_FLOATS;
+}
+
+dkv_status check_decode(const dkv_cache *cache, const void *Q, int32_t q_dtype, int32_t Hq,
+                        void *ws, size_t ws_bytes, int64_t *need_floats) {
+    dkv_status s = check_cache(cache);
+    if (s != DKV_OK) return s;
+    if (!ws || (Q == nullptr && q_dtype >= 0)) return DKV_EINVAL;
+    if (q_dtype >= 0 && !valid_dtype(q_dtype)) return DKV_EINVAL;
+    if (Hq < 1 || Hq % cache->desc.n_kv_heads != 0) return DKV_EINVAL;
+    if ((Q && !aligned16(Q)) || !aligned16(ws)) return DKV_EALIGN;
+    bool ok;
+    int64_t need = workspace_floats(&cache->desc, Hq, &ok);
+    if (!ok) return DKV_ECUDA;
+    if (ws_bytes < (size_t)need * sizeof(float)) return DKV_ECAPACITY;
+    *need_floats = need;
+    return DKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t dkv_abi_version(void) { return DKV_ABI_VERSION; }
+
+size_t dkv_cache_bytes(const dkv_cache_desc *desc) {
+    if (check_desc(desc) != DKV_OK) return 0;
+    return make_layout(desc).total;
+}
+
+dkv_status dkv_cache_init(const dkv_cache_desc *desc, void *dev, size_t bytes, dkv_cache *out,
+                          void *stream) {
+    dkv_status s = check_desc(desc);
+    if (s != DKV_OK) return s;
+    if (!dev || !out) return DKV_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(dev) & (kAlign - 1)) != 0) return DKV_EALIGN;
+    Layout L = make_layout(desc);
+    if (bytes < L.total) return DKV_ECAPACITY;
+    std::memset(out, 0, sizeof(*out));
+    out->desc = *desc;
+    out->base = dev;
+    out->bytes = bytes;
+    out->seq_stride = L.seq_stride;
+    out->rec_bytes = L.rec_bytes;
+    out->n_groups = L.n_groups;
+    out->off_data = L.off_data;
+    out->off_state = L.off_state;
+    out->off_seqlen = L.off_seqlen;
+    out->off_header = L.off_header;
+    return cuda_status(cudaMemsetAsync(dev, 0, L.total, static_cast<cudaStream_t>(stream)));
+}
+
+dkv_status dkv_encode(dkv_cache *cache, const void *K, const void *V, int32_t dtype,
+                      const int32_t *seq_lens_dev, int32_t T, void *stream) {
+    dkv_status s = check_cache(cache);
+    if (s != DKV_OK) return s;
+    if (!K || !V || !valid_dtype(dtype) || T < 1) return DKV_EINVAL;
+    if (!aligned16(K) || !aligned16(V) || (seq_lens_dev && !aligned16(seq_lens_dev)))
+        return DKV_EALIGN;
+    if (T > cache->desc.max_ctx) return DKV_ECAPACITY;
+    CacheView v = view_of(cache);
+    return cuda_status(dkv::launch_encode(v, K, V, dtype, seq_lens_dev, T, 0,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+dkv_status dkv_append(dkv_cache *cache, const void *K_new, const void *V_new, int32_t dtype,
+                      int32_t n_new, void *stream) {
+    dkv_status s = check_cache(cache);
+    if (s != DKV_OK) return s;
+    if (!K_new || !V_new || !valid_dtype(dtype) || n_new < 1) return DKV_EINVAL;
+    if (!aligned16(K_new) || !aligned16(V_new)) return DKV_EALIGN;
+    if (n_new > cache->desc.max_ctx) return DKV_ECAPACITY;
+    CacheView v = view_of(cache);
+    return cuda_status(dkv::launch_encode(v, K_new, V_new, dtype, nullptr, n_new, 1,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+size_t dkv_decode_workspace_bytes(const dkv_cache_desc *desc, int32_t n_q_heads) {
+    bool ok;
+    int64_t f = workspace_floats(desc, n_q_heads, &ok);
+    return ok ? (size_t)f * sizeof(float) : 0;
+}
+
+dkv_status dkv_decode_attn_split(const dkv_cache *cache, const void *Q, int32_t q_dtype,
+                                 int32_t n_q_heads, float softmax_scale, void *workspace,
+                                 size_t ws_bytes, void *stream) {
+    int64_t need;
+    if (!Q) return DKV_EINVAL;
+    dkv_status s = check_decode(cache, Q, q_dtype, n_q_heads, workspace, ws_bytes, &need);
+    if (s != DKV_OK) return s;
+    CacheView v = view_of(cache);
+    return cuda_status(dkv::launch_split(v, Q, q_dtype, n_q_heads, softmax_scale,
+                                         static_cast<float *>(workspace), need,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+dkv_status dkv_decode_attn_merge(const dkv_cache *cache, int32_t n_q_heads, float *out,
+                                 void *workspace, size_t ws_bytes, void *stream) {
+    int64_t need;
+    if (!out) return DKV_EINVAL;
+    dkv_status s = check_decode(cache, nullptr, -1, n_q_heads, workspace, ws_bytes, &need);
+    if (s != DKV_OK) return s;
+    if (!aligned16(out)) return DKV_EALIGN;
+    CacheView v = view_of(cache);
+    return cuda_status(dkv::launch_merge(v, n_q_heads, out, static_cast<const float *>(workspace),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+dkv_status dkv_decode_attn(const dkv_cache *cache, const void *Q, int32_t q_dtype,
+                           int32_t n_q_heads, float softmax_scale, float *out, void *workspace,
+                           size_t ws_bytes, void *stream) {
+    if (!out) return DKV_EINVAL;
+    if (!aligned16(out)) return DKV_EALIGN;
+    dkv_status s = dkv_decode_attn_split(cache, Q, q_dtype, n_q_heads, softmax_scale, workspace,
+                                         ws_bytes, stream);
+    if (s != DKV_OK) return s;
+    return dkv_decode_attn_merge(cache, n_q_heads, out, workspace, ws_bytes, stream);
+}
+
+dkv_status dkv_export_canonical(const dkv_cache *cache, uint8_t *codes, uint16_t *scales,
+                                uint16_t *keyframes, float *state, void *stream) {
+    dkv_status s = check_cache(cache);
+    if (s != DKV_OK) return s;
+    if ((codes && !aligned16(codes)) || (scales && !aligned16(scales)) ||
+        (keyframes && !aligned16(keyframes)) || (state && !aligned16(state)))
+        return DKV_EALIGN;
+    CacheView v = view_of(cache);
+    return cuda_status(dkv::launch_readback(v, codes, scales, keyframes, state, nullptr,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+dkv_status dkv_dequantize(const dkv_cache *cache, float *out, void *stream) {
+    dkv_status s = check_cache(cache);
+    if (s != DKV_OK) return s;
+    if (!out) return DKV_EINVAL;
+    if (!aligned16(out)) return DKV_EALIGN;
+    CacheView v = view_of(cache);
+    return cuda_status(dkv::launch_readback(v, nullptr, nullptr, nullptr, nullptr, out,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+dkv_status dkv_get_device_status(const dkv_cache *cache, int32_t *host_out, void *stream) {
+    dkv_status s = check_cache(cache);
+    if (s != DKV_OK) return s;
+    if (!host_out) return DKV_EINVAL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t *word = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(cache->base) + cache->off_header);
+    int32_t h = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, word, sizeof(h), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof(int32_t), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return DKV_ECUDA;
+    *host_out = h;
+    return h ? DKV_EDEVICE : DKV_OK;
+}
+
+const char *dkv_status_str(dkv_status s) {
+    switch (s) {
+        case DKV_OK: return "ok";
+        case DKV_EINVAL: return "invalid argument";
+        case DKV_EALIGN: return "misaligned pointer";
+        case DKV_ECAPACITY: return "capacity or workspace too small";
+        case DKV_EUNSUPPORTED: return "unsupported configuration";
+        case DKV_ECUDA: return "CUDA error";
+        case DKV_EDEVICE: return "device status word set";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,180 @@
+// dkv_common.cuh -- shared device-side definitions of the Delta-KV library:
+// the in-HBM layout of the three cache formats, the channel permutations that
+// put each thread's tensor-core fragment in one contiguous chunk, and thin
+// wrappers over the sm_100a PTX the kernels use (mbarrier, bulk async copy,
+// mma.sync, prmt).
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "../../include/dkv.h"
+
+namespace dkv {
+
+constexpr int D = 128;          // head_dim
+constexpr int NB = 4;           // 32-channel quantisation blocks per token
+constexpr int SEG = 32;         // positions per pipeline stage
+constexpr int KF_BYTES = 512;   // K keyframe (256 B) followed by V keyframe (256 B)
+constexpr int SC_BYTES = 16;    // per position: dK[4] then dV[4], fp16
+constexpr int NIB_BYTES = 64;   // per position per tensor: 128 nibbles
+constexpr int POS_Q4 = SC_BYTES + 2 * NIB_BYTES;   // 144 B per position
+constexpr int POS_F16 = 2 * D * 2;                 // 512 B per position
+
+// ---------------------------------------------------------------------------
+// Layout of one sequence (one batch entry, one kv head):
+//  DELTA: groups of kf positions, each a contiguous record
+//           [K kf 256 B][V kf 256 B][scales (kf-1) x 16 B]
+//           [K nibbles (kf-1) x 64 B][V nibbles (kf-1) x 64 B]
+//         record g holds positions g*kf .. g*kf+kf-1; delta i of the record is
+//         position g*kf + 1 + i.
+//  Q4_0:  [scales cap x 16 B][K nibbles cap x 64 B][V nibbles cap x 64 B]
+//  FP16:  [K cap x 256 B][V cap x 256 B]
+// Every section size and offset is a multiple of 16 B, so 1-D bulk copies
+// (which need 16-B aligned addresses and sizes) can move any run of them.
+// ---------------------------------------------------------------------------
+__host__ __device__ inline int64_t delta_rec_bytes(int kf) {
+    return (int64_t)KF_BYTES + (int64_t)(kf - 1) * POS_Q4;
+}
+
+// ---------------------------------------------------------------------------
+// Channel permutations.  With g = lane / 4 and t = lane % 4:
+//  K nibbles of one position: 16 words; word (t*4 + j) holds block j's
+//   channels {32j + 16s + 8e + 2t + h}, nibble index i = 4h + 2s + e.  A
+//   mask with 0x000F000F of the word (or of the word >> 8 for s = 1) yields the
+//   fp16x2 pair of channels (2t, 2t+1) of k-step 2j+s; 0x00F000F0 yields
+//   (2t+8, 2t+9): exactly the B fragment of mma.m16n8k16 for column g.
+//  V nibbles of one position: 8 chunks of 8 B; byte (g*8 + mt) holds channel
+//   16mt + g (low nibble) and 16mt + g + 8 (high nibble): the rows thread g
+//   owns in the A fragment of m-tile mt.
+//  K keyframe / FP16 K values: halfword (t*32 + 4kk + 2e + h) = channel
+//   16kk + 8e + 2t + h (the B fragment pairs of column g = 0).
+//  V keyframe / FP16 V values: halfword (g*16 + 2mt + e) = channel
+//   16mt + g + 8e.
+// ---------------------------------------------------------------------------
+__host__ __device__ inline void k_nib_pos(int c, int &byte, int &shift) {
+    int j = c >> 5, r = c & 31, s = r >> 4, r2 = r & 15, e = r2 >> 3, r3 = r2 & 7;
+    int t = r3 >> 1, h = r3 & 1;
+    int word = t * 4 + j, i = 4 * h + 2 * s + e;
+    byte = word * 4 + (i >> 1);
+    shift = 4 * (i & 1);
+}
+__host__ __device__ inline void v_nib_pos(int c, int &byte, int &shift) {
+    int mt = c >> 4, r = c & 15, g = r & 7, hi = r >> 3;
+    byte = g * 8 + mt;
+    shift = 4 * hi;
+}
+__host__ __device__ inline int k_half_idx(int c) {
+    int kk = c >> 4, r = c & 15, e = r >> 3, t = (r & 7) >> 1, h = r & 1;
+    return t * 32 + 4 * kk + 2 * e + h;
+}
+__host__ __device__ inline int v_half_idx(int c) {
+    int mt = c >> 4, r = c & 15, g = r & 7, e = r >> 3;
+    return g * 16 + 2 * mt + e;
+}
+
+// Device-side cache view passed by value to kernels.
+struct CacheView {
+    uint8_t *data;
+    float *state;          // [2][B][Hkv][2][D]
+    int32_t *seqlen;       // [B]
+    int32_t *header;       // {status, counter, parity, reserved}
+    int64_t seq_stride;
+    int64_t rec_bytes;
+    int32_t B, Hkv, kf, cap, fmt, n_groups;
+};
+
+__device__ inline void set_status(int32_t *header, int bits) {
+    atomicOr(reinterpret_cast<int *>(header), bits);
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ inline uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ inline void mbar_init(uint64_t *bar, int count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+__device__ inline void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ inline void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ inline void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ inline bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: gives up after ~2^31 cycles (about a second) and returns false.
+__device__ inline bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - t0 > (1ll << 31)) return false;
+    }
+}
+// 1-D bulk async copy global -> shared, completion counted on `bar`.
+__device__ inline void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes,
+                                uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ inline uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+__device__ inline uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
+    return (a & mask) | orv;  // compiles to one LOP3
+}
+__device__ inline uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ inline __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+// D = A(16x16 f16, row) * B(16x8 f16, col) + C, fp32 accumulate.
+__device__ inline void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Dequantise the 4 nibble pairs of one 32-bit word (pairs (bits 0-3,16-19),
+// (4-7,20-23), (8-11,24-27), (12-15,28-31)) to exact fp16x2 values code - 8.
+__device__ inline void dq_word(uint32_t w, uint32_t &p0, uint32_t &p1, uint32_t &p2,
+                               uint32_t &p3) {
+    const uint32_t MAGIC = 0x64006400u;  // fp16 1024.0 in both halves
+    const __half2 SUB_LO = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+    const __half2 MUL_HI = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+    const __half2 SUB_HI = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
+    uint32_t w8 = w >> 8;
+    // (1024 + n) - 1032 = n - 8, exact
+    p0 = h2_as_u32(__hsub2(u32_as_h2(lop_and_or(w, 0x000F000Fu, MAGIC)), SUB_LO));
+    p2 = h2_as_u32(__hsub2(u32_as_h2(lop_and_or(w8, 0x000F000Fu, MAGIC)), SUB_LO));
+    // (1024 + 16 n) / 16 - 72 = n - 8, exact
+    p1 = h2_as_u32(__hfma2(u32_as_h2(lop_and_or(w, 0x00F000F0u, MAGIC)), MUL_HI, SUB_HI));
+    p3 = h2_as_u32(__hfma2(u32_as_h2(lop_and_or(w8, 0x00F000F0u, MAGIC)), MUL_HI, SUB_HI));
+}
+
+}  // namespace dkv

@@ -1,0 +1,33 @@
+// dkv_internal.h -- host-side launchers shared between the C-ABI layer and the
+// kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace dkv {
+
+struct CacheView;
+
+cudaError_t launch_encode(const CacheView &cv, const void *K, const void *V, int dtype,
+                          const int32_t *seq_lens, int T_in, int append, cudaStream_t st);
+cudaError_t launch_readback(const CacheView &cv, uint8_t *codes, uint16_t *scales,
+                            uint16_t *keyframes, float *state, float *xhat, cudaStream_t st);
+
+// Persistent-grid geometry of the split kernel for a cache format on the
+// current device: CTAs and warps per CTA.
+struct SplitGeom {
+    int ctas;
+    int warps_per_cta;
+};
+cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g);
+
+// Floats per partial record: m[8], l[8], o[8][128].
+constexpr int PARTIAL_FLOATS = 8 + 8 + 8 * 128;
+
+cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq,
+                         float softmax_scale, float *ws, int64_t ws_floats, cudaStream_t st);
+cudaError_t launch_merge(const CacheView &cv, int Hq, float *out, const float *ws,
+                         cudaStream_t st);
+
+}  // namespace dkv

@@ -1,0 +1,181 @@
+/*
+ * dkv.h -- C ABI of the Delta-KV decode library for NVIDIA B200 (sm_100a).
+ *
+ * A Delta-KV cache stores every kf-th token of each (batch, kv-head)
+ * sequence as an fp16 keyframe and every other token as a 4-bit, Q4_0-style
+ * quantised difference against the reconstructed previous token (closed
+ * loop).  Sources:
+ *   page "영상 압축 기법을 KV 캐시에 적용해 Q4 양자화 오차를 10,000배 줄인
+ *   Delta-KV" (jeff.news article 892): section "핵심 아이디어" (keyframe +
+ *   4-bit token-to-token differences instead of absolute values), section
+ *   "벤치마크" (kf = 32; Q4_0 and F16 caches as comparators), section
+ *   "컨텍스트 길이에 따른 안정성" (no error build-up with 512 delta frames);
+ *   page "KV 캐시 벡터 양자화와 주의 보존 변환" (llm-wiki), section
+ *   "KV 캐시가 왜 병목인가" (a decode step reads every cached K/V from HBM,
+ *   forms QK^T, softmax and A.V; the read is the bottleneck).
+ *
+ * The Q4_0 block rule (both quantised formats): blocks of 32 channels;
+ * m = signed element of largest |.| (lowest index on ties); d = fp16(m / -8);
+ * code = clamp(trunc(x / d + 8.5), 0, 15) with an IEEE fp32 division by the
+ * stored fp16 d; d == 0 gives code 8; dequantised value (code - 8) * d.
+ *
+ * Conventions for every entry point:
+ *  - The caller owns all memory.  The library never allocates, never frees
+ *    and never synchronises, except dkv_get_device_status (which synchronises
+ *    the stream it is given).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream.
+ *  - Host-side validation happens before any launch; a failed check returns
+ *    an error and launches nothing.  Device pointers must be 16-byte aligned
+ *    (DKV_EALIGN otherwise); the cache base must be 256-byte aligned.
+ *  - Faults found on the device (a sequence length out of range, an append
+ *    past capacity, a pipeline wait that ran out) set a status word inside
+ *    the cache; the kernel skips the affected work and returns.  Nothing
+ *    traps and nothing waits without a bound.  Read and clear the word with
+ *    dkv_get_device_status.
+ *  - head_dim must be 128.  Query head h reads KV head h / (Hq / Hkv).
+ *  - Inputs must be finite and within the fp16 range.
+ */
+#ifndef DKV_H
+#define DKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DKV_ABI_VERSION 1
+
+typedef enum {
+    DKV_OK = 0,
+    DKV_EINVAL = 1,        /* bad argument: null pointer, bad shape, bad enum */
+    DKV_EALIGN = 2,        /* pointer not aligned as required */
+    DKV_ECAPACITY = 3,     /* request exceeds cache capacity or workspace size */
+    DKV_EUNSUPPORTED = 4,  /* valid but not supported (e.g. head_dim != 128) */
+    DKV_ECUDA = 5,         /* a CUDA runtime call or launch failed */
+    DKV_EDEVICE = 6        /* the device status word is non-zero */
+} dkv_status;
+
+typedef enum {
+    DKV_FMT_FP16 = 0,      /* comparator: fp16 values */
+    DKV_FMT_Q4_0 = 1,      /* comparator: Q4_0 on absolute values */
+    DKV_FMT_DELTA = 2      /* keyframe + closed-loop 4-bit deltas */
+} dkv_format;
+
+typedef enum { DKV_F32 = 0, DKV_F16 = 1, DKV_BF16 = 2 } dkv_dtype;
+
+/* Bits of the device status word. */
+#define DKV_DEV_BAD_SEQLEN   0x1   /* a sequence length outside [0, max_ctx] */
+#define DKV_DEV_CAPACITY     0x2   /* an append would pass max_ctx (skipped) */
+#define DKV_DEV_TIMEOUT      0x4   /* a bounded pipeline wait ran out */
+#define DKV_DEV_BAD_HEADS    0x8   /* n_q_heads not a multiple of n_kv_heads */
+
+typedef struct {
+    int32_t batch;         /* B >= 1 (<= 1024) */
+    int32_t n_kv_heads;    /* Hkv >= 1 */
+    int32_t head_dim;      /* D, must be 128 */
+    int32_t kf;            /* keyframe interval >= 1 (DKV_FMT_DELTA only) */
+    int32_t max_ctx;       /* capacity in tokens per sequence, >= 1 */
+    int32_t fmt;           /* dkv_format */
+} dkv_cache_desc;
+
+/* POD view of a cache laid out in caller-owned device memory.  Filled by
+ * dkv_cache_init; all offsets are bytes from `base`. */
+typedef struct {
+    dkv_cache_desc desc;
+    void *base;
+    size_t bytes;
+    size_t seq_stride;     /* bytes of one (batch, kv-head) sequence's data */
+    size_t rec_bytes;      /* DELTA: bytes of one keyframe group record */
+    int32_t n_groups;      /* DELTA: groups per sequence at capacity */
+    int32_t reserved0;
+    size_t off_data;       /* compressed data, B*Hkv*seq_stride bytes */
+    size_t off_state;      /* fp32 reconstruction state [2][B][Hkv][2][D] */
+    size_t off_seqlen;     /* int32 seq_len[B] */
+    size_t off_header;     /* int32 {status, counter, parity, reserved} */
+} dkv_cache;
+
+/* ABI version of the loaded library (DKV_ABI_VERSION). */
+int32_t dkv_abi_version(void);
+
+/* Bytes of device memory a cache with this descriptor needs (0 if the
+ * descriptor is invalid). */
+size_t dkv_cache_bytes(const dkv_cache_desc *desc);
+
+/* Lay a cache out in `dev` (>= dkv_cache_bytes, 256-byte aligned) and zero it
+ * with cudaMemsetAsync on `stream` (every seq_len becomes 0).  Fills *out. */
+dkv_status dkv_cache_init(const dkv_cache_desc *desc, void *dev, size_t bytes,
+                          dkv_cache *out, void *stream);
+
+/* Encode whole sequences, replacing the cache contents.
+ * K, V: [B][Hkv][T][D] contiguous device arrays of `dtype`.
+ * seq_lens_dev: device int32[B] with 0 <= T_b <= T (NULL: every T_b = T).
+ * Positions [0, T_b) of sequence b are encoded; seq_len[b] becomes T_b and
+ * the reconstruction state is that of position T_b - 1.
+ * (Format of the cache: keyframes, 4-bit closed-loop deltas, Q4_0 or fp16.) */
+dkv_status dkv_encode(dkv_cache *cache, const void *K, const void *V, int32_t dtype,
+                      const int32_t *seq_lens_dev, int32_t T, void *stream);
+
+/* Append n_new tokens to every sequence at its current device-side seq_len,
+ * continuing the closed loop from the stored reconstruction state.
+ * K_new, V_new: [B][Hkv][n_new][D] contiguous device arrays of `dtype`.
+ * A batch entry whose seq_len + n_new would pass max_ctx is skipped and sets
+ * DKV_DEV_CAPACITY. */
+dkv_status dkv_append(dkv_cache *cache, const void *K_new, const void *V_new,
+                      int32_t dtype, int32_t n_new, void *stream);
+
+/* Bytes of device workspace dkv_decode_attn needs for n_q_heads query heads on
+ * the current device. */
+size_t dkv_decode_workspace_bytes(const dkv_cache_desc *desc, int32_t n_q_heads);
+
+/* One decode step of GQA attention over the cache: for every batch entry b
+ * and query head h, out[b][h][:] = softmax(softmax_scale * q . k^_p) . v^_p
+ * over the positions p < seq_len[b] (no mask beyond the length; an empty
+ * sequence gives zeros).
+ * Q: [B][n_q_heads][D] device array of q_dtype; out: [B][n_q_heads][D] fp32
+ * device array; workspace: device scratch of >= dkv_decode_workspace_bytes.
+ * Runs dkv_decode_attn_split then dkv_decode_attn_merge. */
+dkv_status dkv_decode_attn(const dkv_cache *cache, const void *Q, int32_t q_dtype,
+                           int32_t n_q_heads, float softmax_scale, float *out,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/* The two launches of dkv_decode_attn, exposed so each can be timed alone:
+ * the split kernel streams the compressed cache and writes per-range partial
+ * (max, sum, unnormalised output) records to the workspace; the merge kernel
+ * combines them (log-sum-exp) into out.  Same arguments as dkv_decode_attn. */
+dkv_status dkv_decode_attn_split(const dkv_cache *cache, const void *Q, int32_t q_dtype,
+                                 int32_t n_q_heads, float softmax_scale,
+                                 void *workspace, size_t ws_bytes, void *stream);
+dkv_status dkv_decode_attn_merge(const dkv_cache *cache, int32_t n_q_heads, float *out,
+                                 void *workspace, size_t ws_bytes, void *stream);
+
+/* Copy the stored fields out in a canonical, layout-independent form (device
+ * destinations; NULL skips a field):
+ *   codes     uint8  [B][Hkv][2][max_ctx][D]   one code per element
+ *   scales    uint16 [B][Hkv][2][max_ctx][D/32] fp16 bits of the block scale
+ *   keyframes uint16 [B][Hkv][2][n_kf][D]     fp16 bits; n_kf = n_groups
+ *                                             (DELTA) or max_ctx (FP16)
+ *   state     float  [B][Hkv][2][D]           reconstruction of the last
+ *                                             encoded position (DELTA)
+ * Rows of keyframe positions in codes/scales are zero (DELTA).  Tensor index
+ * 0 is K, 1 is V. */
+dkv_status dkv_export_canonical(const dkv_cache *cache, uint8_t *codes, uint16_t *scales,
+                                uint16_t *keyframes, float *state, void *stream);
+
+/* Reconstructed values x^ of every stored position, fp32
+ * [B][Hkv][2][max_ctx][D] (positions >= seq_len are left untouched). */
+dkv_status dkv_dequantize(const dkv_cache *cache, float *out, void *stream);
+
+/* Synchronise `stream`, copy the device status word to *host_out and clear
+ * it.  Returns DKV_EDEVICE if it was non-zero, DKV_OK otherwise. */
+dkv_status dkv_get_device_status(const dkv_cache *cache, int32_t *host_out, void *stream);
+
+/* Static description of a status code. */
+const char *dkv_status_str(dkv_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DKV_H */

@@ -1,0 +1,180 @@
+"""CPU-only checks of the C ABI: the library builds and loads, exports every
+function include/dkv.h declares, sizes caches by the documented layout, and
+rejects bad arguments before touching the GPU.  Also checks the host-side
+arithmetic of the decode work split (which warp owns which unit, and the
+partial-record slot of every (warp, sequence) pair)."""
+import ctypes
+import random
+import re
+import subprocess
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+@pytest.fixture(scope="module")
+def dkv():
+    from delta_quantized_kv_b200 import build
+    build.build()
+    import delta_quantized_kv_b200 as m
+    m.load()
+    return m
+
+
+def _declared():
+    text = (ROOT / "include" / "dkv.h").read_text()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(dkv_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol(dkv):
+    names = _declared()
+    assert len(names) >= 13
+    nm = subprocess.run(["nm", "-D", "--defined-only", str(dkv.LIB_PATH)], capture_output=True,
+                        text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (dkv_\w+)", nm))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    assert set(dkv.EXPORTS) <= exported
+
+
+def test_abi_version_and_status_strings(dkv):
+    assert dkv.dkv_abi_version() == 1
+    for s in range(7):
+        assert dkv.status_str(s) and dkv.status_str(s) != "unknown status"
+    assert dkv.status_str(99) == "unknown status"
+
+
+def _desc(dkv, B=16, H=8, D=128, kf=32, cap=32768, fmt=2):
+    return dkv.dkv_cache_desc(B, H, D, kf, cap, fmt)
+
+
+def test_cache_bytes_follow_the_layout(dkv):
+    def expect(B, H, kf, cap, fmt):
+        if fmt == 2:
+            ng = -(-cap // kf)
+            stride = ng * (512 + (kf - 1) * 144)
+        elif fmt == 1:
+            stride = cap * 144
+        else:
+            stride = cap * 512
+        up = lambda x: (x + 255) // 256 * 256
+        off_state = up(B * H * stride + 4096)
+        off_seq = up(off_state + 2 * B * H * 2 * 128 * 4)
+        off_hdr = up(off_seq + 4 * B)
+        return up(off_hdr + 16), stride
+    for (B, H, kf, cap, fmt) in [(16, 8, 32, 32768, 2), (1, 1, 1, 1, 2), (4, 8, 512, 131328, 2),
+                                 (2, 3, 33, 1000, 2), (16, 8, 32, 32768, 1), (16, 8, 32, 32768, 0)]:
+        tot, stride = expect(B, H, kf, cap, fmt)
+        assert dkv.dkv_cache_bytes(_desc(dkv, B, H, 128, kf, cap, fmt)) == tot
+    # the headline cache: 4976 B per 32-token group -> 155.5 B per token per kv head
+    assert expect(16, 8, 32, 32768, 2)[1] * 16 * 8 == 652_214_272
+
+
+@pytest.mark.parametrize("field,val", [("batch", 0), ("batch", 1025), ("n_kv_heads", 0),
+                                       ("kf", 0), ("max_ctx", 0), ("fmt", 7)])
+def test_invalid_descriptors_size_zero(dkv, field, val):
+    d = _desc(dkv)
+    setattr(d, field, val)
+    assert dkv.dkv_cache_bytes(d) == 0
+
+
+def test_head_dim_must_be_128(dkv):
+    d = _desc(dkv, D=64)
+    assert dkv.dkv_cache_bytes(d) == 0
+    out = dkv.dkv_cache()
+    s = dkv.load().dkv_cache_init(ctypes.byref(d), 4096, 1 << 30, ctypes.byref(out), None)
+    assert s == dkv.DKV_EUNSUPPORTED
+
+
+def test_init_rejects_bad_pointers_without_a_launch(dkv):
+    lib = dkv.load()
+    d = _desc(dkv, B=1, H=1, cap=64)
+    out = dkv.dkv_cache()
+    n = dkv.dkv_cache_bytes(d)
+    assert lib.dkv_cache_init(ctypes.byref(d), None, n, ctypes.byref(out), None) == dkv.DKV_EINVAL
+    assert lib.dkv_cache_init(ctypes.byref(d), 4096 + 16, n, ctypes.byref(out), None) == dkv.DKV_EALIGN
+    assert lib.dkv_cache_init(ctypes.byref(d), 4096, n - 1, ctypes.byref(out), None) == dkv.DKV_ECAPACITY
+
+
+def test_calls_on_an_invalid_cache_are_rejected(dkv):
+    lib = dkv.load()
+    c = dkv.dkv_cache()          # base == NULL
+    assert lib.dkv_encode(ctypes.byref(c), 16, 16, 1, None, 8, None) == dkv.DKV_EINVAL
+    assert lib.dkv_append(ctypes.byref(c), 16, 16, 1, 1, None) == dkv.DKV_EINVAL
+    assert lib.dkv_decode_attn(ctypes.byref(c), 16, 1, 8, 1.0, 16, 16, 1 << 20, None) == dkv.DKV_EINVAL
+    assert lib.dkv_dequantize(ctypes.byref(c), 16, None) == dkv.DKV_EINVAL
+    w = ctypes.c_int32(0)
+    assert lib.dkv_get_device_status(ctypes.byref(c), ctypes.byref(w), None) == dkv.DKV_EINVAL
+
+
+def test_bad_dtype_and_sizes_rejected_on_host(dkv):
+    """A well-formed view whose arguments are wrong: nothing is launched."""
+    lib = dkv.load()
+    d = _desc(dkv, B=2, H=2, cap=100)
+    n = dkv.dkv_cache_bytes(d)
+    c = dkv.dkv_cache()
+    c.desc = d
+    c.base = 1 << 20
+    c.bytes = n
+    # replicate the layout the library computes (offsets must agree)
+    up = lambda x: (x + 255) // 256 * 256
+    ng = -(-100 // 32)
+    c.seq_stride = ng * (512 + 31 * 144)
+    c.rec_bytes = 512 + 31 * 144
+    c.n_groups = ng
+    c.off_state = up(4 * c.seq_stride + 4096)
+    c.off_seqlen = up(c.off_state + 2 * 4 * 2 * 128 * 4)
+    c.off_header = up(c.off_seqlen + 8)
+    assert lib.dkv_encode(ctypes.byref(c), 1 << 12, 1 << 12, 9, None, 8, None) == dkv.DKV_EINVAL
+    assert lib.dkv_encode(ctypes.byref(c), (1 << 12) + 2, 1 << 12, 1, None, 8, None) == dkv.DKV_EALIGN
+    assert lib.dkv_encode(ctypes.byref(c), 1 << 12, 1 << 12, 1, None, 101, None) == dkv.DKV_ECAPACITY
+    assert lib.dkv_append(ctypes.byref(c), 1 << 12, 1 << 12, 1, 0, None) == dkv.DKV_EINVAL
+    # n_q_heads not a multiple of n_kv_heads
+    assert lib.dkv_decode_attn(ctypes.byref(c), 1 << 12, 1, 3, 1.0, 1 << 12, 1 << 12, 1 << 30,
+                               None) == dkv.DKV_EINVAL
+
+
+# ---- the decode work split (restated from the kernel's range arithmetic) ----
+def _start(w, NW, T):
+    return (w * T) // NW
+
+
+def _warp_of(x, NW, T):
+    return ((x + 1) * NW - 1) // T
+
+
+def test_work_split_covers_every_unit_once_and_slots_are_unique():
+    rng = random.Random(5)
+    for _ in range(300):
+        nseq = rng.randint(1, 40)
+        units = [rng.choice([0, 1, 2, 3, 7, 50, 1024]) for _ in range(nseq)]
+        T = sum(units)
+        if T == 0:
+            continue
+        NW = rng.choice([1, 3, 4, 37, 592, 1776])
+        owner = {}
+        for w in range(NW):
+            for x in range(_start(w, NW, T), _start(w + 1, NW, T)):
+                assert x not in owner
+                owner[x] = w
+        assert len(owner) == T
+        for x in range(T):
+            assert _warp_of(x, NW, T) == owner[x]
+        # slots (warp + sequence) written by warps that touch a sequence
+        starts = [0]
+        for u in units:
+            starts.append(starts[-1] + u)
+        slots = {}
+        for s in range(nseq):
+            xs, xe = starts[s], starts[s + 1]
+            if xs == xe:
+                continue
+            for w in range(_warp_of(xs, NW, T), _warp_of(xe - 1, NW, T) + 1):
+                if _start(w, NW, T) >= _start(w + 1, NW, T):
+                    continue
+                slot = w + s
+                assert slot not in slots, (slot, slots.get(slot), (w, s))
+                slots[slot] = (w, s)
+                assert slot < NW + nseq
