@@ -49,7 +49,7 @@ _lib = None
 EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode", "dkv_append",
            "dkv_decode_workspace_bytes", "dkv_decode_attn", "dkv_decode_attn_split",
            "dkv_decode_attn_merge", "dkv_export_canonical", "dkv_dequantize",
-           "dkv_get_device_status", "dkv_status_str"]
+           "dkv_get_device_status", "dkv_status_str", "dkv_decode_attn_noalloc"]
 
 
 def load():
@@ -78,6 +78,7 @@ def load():
         "dkv_dequantize": ([PC, P, P], I),
         "dkv_get_device_status": ([PC, ctypes.POINTER(I), P], I),
         "dkv_status_str": ([I], ctypes.c_char_p),
+        "dkv_decode_attn_noalloc": ([PC, P, I, I, F, P, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -174,6 +175,17 @@ def dkv_decode_attn_merge(cache: dkv_cache, n_q_heads, out, workspace, ws_bytes,
     _check(load().dkv_decode_attn_merge(ctypes.byref(cache), n_q_heads, _ptr(out),
                                         _ptr(workspace), ws_bytes, _stream(stream)),
            "dkv_decode_attn_merge")
+
+
+def dkv_decode_attn_noalloc(cache: dkv_cache, Q, q_dtype, n_q_heads, softmax_scale, out,
+                            stream=None) -> None:
+    """Decode step that needs no workspace: the partial records go to a fixed
+    16 MiB array the library keeps on each GPU (for callers that cannot
+    allocate device memory when they decode, e.g. under graph capture).
+    Calls overlapping on the GPU race on that array."""
+    _check(load().dkv_decode_attn_noalloc(ctypes.byref(cache), _ptr(Q), q_dtype, n_q_heads,
+                                          softmax_scale, _ptr(out), _stream(stream)),
+           "dkv_decode_attn_noalloc")
 
 
 def dkv_export_canonical(cache: dkv_cache, codes=None, scales=None, keyframes=None, state=None,

@@ -151,6 +151,25 @@ dkv_status dkv_decode_attn_split(const dkv_cache *cache, const void *Q, int32_t 
 dkv_status dkv_decode_attn_merge(const dkv_cache *cache, int32_t n_q_heads, float *out,
                                  void *workspace, size_t ws_bytes, void *stream);
 
+/* Size of the library-owned scratch array used by dkv_decode_attn_noalloc. */
+#define DKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* dkv_decode_attn for callers that cannot allocate device memory when they
+ * decode (for example code running under CUDA graph capture, where cudaMalloc
+ * is not allowed, or a plugin inside an engine that owns and pre-plans every
+ * device allocation).  The pages have no counterpart: this is a deployment
+ * variant of the same decode step, with the same arguments minus the
+ * workspace.  The partial records go to a fixed 16 MiB array that the library
+ * itself holds on every GPU that loads it, until the process exits.  The
+ * first call on a device looks up that array's address (make it before any
+ * stream capture).  Returns DKV_ECAPACITY when the step needs more than
+ * DKV_NOALLOC_SCRATCH_BYTES of records (see dkv_decode_workspace_bytes).  All
+ * calls share the array: calls that overlap on the GPU race and must be
+ * serialised by the caller.  Allocates and frees nothing. */
+dkv_status dkv_decode_attn_noalloc(const dkv_cache *cache, const void *Q, int32_t q_dtype,
+                                   int32_t n_q_heads, float softmax_scale, float *out,
+                                   void *stream);
+
 /* Copy the stored fields out in a canonical, layout-independent form (device
  * destinations; NULL skips a field):
  *   codes     uint8  [B][Hkv][2][max_ctx][D]   one code per element
