@@ -29,7 +29,7 @@
 // E_s the exclusive prefix of the weights inside the group and R_g the sum of
 // the group's dequantised deltas (an extra MMA against the scales alone).
 //
-// Work split: the (sequence, group) units of all sequences are flattened and
+// Work split: the (sequence, unit) pairs of all sequences are flattened and
 // cut into equal contiguous ranges, one per warp of a persistent grid.  Each
 // warp streams its range through its own ring of shared-memory stages filled
 // by 1-D bulk async copies (cp.async.bulk + mbarrier), keeps an online-softmax
@@ -46,15 +46,32 @@ namespace dkv {
 enum Mode { SUFFIX = 0, PREFIX = 1, PLAIN = 2 };
 
 constexpr int WARPS = 4;                     // warps per CTA (independent pipelines)
-constexpr int MAX_B = 1024;
+
+#ifndef DKV_NIB_MINB
+#define DKV_NIB_MINB 4                       // resident CTAs per SM (nibble formats)
+#endif
+#ifndef DKV_NIB_NS
+#define DKV_NIB_NS 2                         // pipeline stages per warp (nibble formats)
+#endif
 
 template <int FMT> struct FmtCfg;
-template <> struct FmtCfg<DKV_FMT_DELTA> { static constexpr int STAGE = 5120, NS = 3; };
-template <> struct FmtCfg<DKV_FMT_Q4_0>  { static constexpr int STAGE = 5120, NS = 3; };
-template <> struct FmtCfg<DKV_FMT_FP16>  { static constexpr int STAGE = 16384, NS = 2; };
+template <> struct FmtCfg<DKV_FMT_DELTA> { static constexpr int STAGE = 5120, NS = DKV_NIB_NS, MINB = DKV_NIB_MINB; };
+template <> struct FmtCfg<DKV_FMT_Q4_0>  { static constexpr int STAGE = 5120, NS = DKV_NIB_NS, MINB = DKV_NIB_MINB; };
+template <> struct FmtCfg<DKV_FMT_FP16>  { static constexpr int STAGE = 16384, NS = 2, MINB = 1; };
 
-// Stage layout (DELTA / Q4_0): [K kf 256][V kf 256][scales 32x16][K nib 32x64][V nib 32x64]
-constexpr int ST_KF = 0, ST_SC = 512, ST_KN = 1024, ST_VN = 3072;
+// Shared-memory map of the split kernel: [mbarriers WARPS*NS x 8 B]
+// [stage descriptors WARPS*NS x 16 B][stages WARPS*NS x STAGE], each region
+// aligned; the offsets follow from NS so no region can overlap another.
+template <int FMT> struct SmemMap {
+    static constexpr int NS = FmtCfg<FMT>::NS, STAGE = FmtCfg<FMT>::STAGE;
+    static constexpr int BAR_OFF = 0;
+    static constexpr int META_OFF = ((BAR_OFF + 8 * WARPS * NS) + 15) / 16 * 16;
+    static constexpr int STAGE_OFF = ((META_OFF + 16 * WARPS * NS) + 127) / 128 * 128;
+    static constexpr int BYTES = STAGE_OFF + WARPS * NS * STAGE;
+    static_assert(META_OFF >= BAR_OFF + 8 * WARPS * NS, "barriers overlap descriptors");
+    static_assert(STAGE_OFF >= META_OFF + 16 * WARPS * NS, "descriptors overlap stages");
+    static_assert(STAGE % 128 == 0, "stages must stay 128-byte aligned");
+};
 
 struct SplitArgs {
     CacheView cv;
@@ -78,47 +95,75 @@ __host__ __device__ inline int64_t warp_of(int64_t x, int64_t NW, int64_t T) {
     return ((x + 1) * NW - 1) / T;
 }
 
+__device__ inline int clamp_len(const CacheView &cv, int b) {
+    int l = cv.seqlen[b];
+    return (l < 0 || l > cv.cap) ? 0 : l;
+}
+
 // Iterates the (unit, segment) stage items of one warp's range in order.
 struct Cursor {
     int64_t x, x_end;          // flattened unit index, end of range
     int b, vs, g;              // batch entry, sequence within the batch entry, unit
     int units_b;               // units per sequence of batch entry b
     int len_b;                 // tokens of batch entry b
-    int seg, nseg;             // segment within the unit
+    int seg, nseg;             // segment within the unit (kf > 32 only)
     __device__ bool valid() const { return x < x_end; }
 };
 
-__device__ inline int clamp_len(const CacheView &cv, int b) {
-    int l = cv.seqlen[b];
-    return (l < 0 || l > cv.cap) ? 0 : l;
-}
-
+template <int MODE>
 __device__ inline int nseg_of(const CacheView &cv, int len, int g) {
-    if (cv.fmt != DKV_FMT_DELTA) return 1;
-    int glen = min(cv.kf, len - g * cv.kf);
+    if (MODE != PREFIX) return 1;
+    const int glen = min(cv.kf, len - g * cv.kf);
     return (glen + SEG - 1) / SEG;
 }
 
-__device__ inline void cursor_seek(Cursor &c, const CacheView &cv, const int64_t *plan, int nvs) {
-    // find b with plan[b] <= x < plan[b+1]
-    int lo = 0, hi = cv.B;  // invariant plan[lo] <= x < plan[hi]
-    while (hi - lo > 1) {
-        int mid = (lo + hi) >> 1;
-        if (plan[mid] <= c.x) lo = mid; else hi = mid;
+// Warp-wide: total units over all batch entries, and (if 0 <= r < total) the
+// batch entry b containing unit r with the index of its first unit.
+__device__ inline int64_t locate(const CacheView &cv, int nvs, int64_t r, int &b_out,
+                                 int64_t &base_out) {
+    const int lane = threadIdx.x & 31;
+    int64_t base = 0;
+    b_out = -1;
+    base_out = 0;
+    for (int b0 = 0; b0 < cv.B; b0 += 32) {
+        const int b = b0 + lane;
+        const int64_t u = b < cv.B ? (int64_t)nvs * units_of(cv.fmt, cv.kf, clamp_len(cv, b)) : 0;
+        int64_t inc = u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        const int64_t chunk = __shfl_sync(0xffffffffu, inc, 31);
+        if (b_out < 0 && r >= base && r < base + chunk) {
+            const unsigned m = __ballot_sync(0xffffffffu, base + inc > r);
+            const int l = __ffs(m) - 1;
+            b_out = b0 + l;
+            base_out = base + __shfl_sync(0xffffffffu, inc - u, l);
+        }
+        base += chunk;
     }
-    c.b = lo;
-    c.len_b = clamp_len(cv, lo);
+    return base;
+}
+
+template <int MODE>
+__device__ inline void cursor_seek(Cursor &c, const CacheView &cv, int nvs) {
+    int b;
+    int64_t base;
+    locate(cv, nvs, c.x, b, base);
+    c.b = b;
+    c.len_b = clamp_len(cv, b);
     c.units_b = units_of(cv.fmt, cv.kf, c.len_b);
-    int64_t r = c.x - plan[lo];
+    const int64_t r = c.x - base;
     c.vs = (int)(r / c.units_b);
     c.g = (int)(r % c.units_b);
     c.seg = 0;
-    c.nseg = nseg_of(cv, c.len_b, c.g);
-    (void)nvs;
+    c.nseg = nseg_of<MODE>(cv, c.len_b, c.g);
 }
 
+template <int MODE>
 __device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs) {
-    if (++c.seg < c.nseg) return;
+    if (MODE == PREFIX && ++c.seg < c.nseg) return;
     c.seg = 0;
     ++c.x;
     if (!c.valid()) return;
@@ -133,16 +178,70 @@ __device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs) {
             } while (c.units_b == 0);
         }
     }
-    c.nseg = nseg_of(cv, c.len_b, c.g);
+    c.nseg = nseg_of<MODE>(cv, c.len_b, c.g);
+}
+
+// Stage layouts in shared memory (offsets from the stage start):
+//  DELTA, kf <= 32: the whole group record, one copy:
+//      [K kf 256][V kf 256][scales (kf-1)x16][K nib (kf-1)x64][V nib (kf-1)x64]
+//  DELTA, kf > 32 (one 32-position segment) and Q4_0:
+//      [K kf 256][V kf 256][scales 32x16][K nib 32x64][V nib 32x64]
+//  FP16: [K 32x256][V 32x256]
+// For slot s (position a + s) the scale / K nibble / V nibble rows start at
+// sc0 + 16 s, kn0 + 64 s, vn0 + 64 s.
+struct StageMap {
+    int sc0, kn0, vn0;
+};
+template <int FMT, int MODE>
+__device__ inline StageMap stage_map(int kf) {
+    StageMap m;
+    if (FMT == DKV_FMT_DELTA && MODE == SUFFIX) {
+        m.sc0 = KF_BYTES - SC_BYTES;
+        m.kn0 = KF_BYTES + (kf - 1) * SC_BYTES - NIB_BYTES;
+        m.vn0 = KF_BYTES + (kf - 1) * (SC_BYTES + NIB_BYTES) - NIB_BYTES;
+    } else {
+        m.sc0 = 512;
+        m.kn0 = 1024;
+        m.vn0 = 3072;
+    }
+    return m;
+}
+
+// What the consumer needs to know about a stage item, written next to the
+// stage by the issuing lane before it arms the barrier.
+struct StageMeta {
+    int b, vs;                 // batch entry, sequence within it
+    int npos;                  // valid positions in the stage
+    int flags;                 // bit 0: first segment of a group; bit 1: last segment
+};
+
+template <int MODE>
+__device__ inline StageMeta make_meta(const CacheView &cv, const Cursor &c) {
+    StageMeta m;
+    m.b = c.b;
+    m.vs = c.vs;
+    if (cv.fmt == DKV_FMT_DELTA) {
+        const int glen = min(cv.kf, c.len_b - c.g * cv.kf);
+        m.npos = min(SEG, glen - c.seg * SEG);
+        m.flags = (c.seg == 0 ? 1 : 0) | (c.seg == c.nseg - 1 ? 2 : 0);
+    } else {
+        m.npos = min(SEG, c.len_b - c.g * SEG);
+        m.flags = 3;
+    }
+    return m;
 }
 
 // Issue the bulk copies of one stage item (one lane).
-template <int FMT>
-__device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nvs_per_kv,
+template <int FMT, int MODE>
+__device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nhg,
                                    uint8_t *stage, uint64_t *bar) {
-    const int kvh = c.vs / nvs_per_kv;
+    const int kvh = c.vs / nhg;
     const uint8_t *sb = cv.data + ((int64_t)c.b * cv.Hkv + kvh) * cv.seq_stride;
-    if (FMT == DKV_FMT_DELTA) {
+    if (FMT == DKV_FMT_DELTA && MODE == SUFFIX) {
+        const uint32_t bytes = (uint32_t)cv.rec_bytes;
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(stage, sb + (int64_t)c.g * cv.rec_bytes, bytes, bar);
+    } else if (FMT == DKV_FMT_DELTA) {
         const int kf = cv.kf;
         const int glen = min(kf, c.len_b - c.g * kf);
         const int a = c.seg * SEG;
@@ -155,24 +254,24 @@ __device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nvs
         const int s0 = (a == 0) ? 1 : 0;       // slot 0 of segment 0 is the keyframe
         const int nd = npos - s0;
         const int di0 = a + s0 - 1;
-        uint32_t bytes = (a == 0 ? KF_BYTES : 0) + nd * (SC_BYTES + 2 * NIB_BYTES);
+        const uint32_t bytes = (a == 0 ? KF_BYTES : 0) + nd * (SC_BYTES + 2 * NIB_BYTES);
         mbar_arrive_expect_tx(bar, bytes);
-        if (a == 0) bulk_g2s(stage + ST_KF, rec, KF_BYTES, bar);
+        if (a == 0) bulk_g2s(stage, rec, KF_BYTES, bar);
         if (nd > 0) {
-            bulk_g2s(stage + ST_SC + s0 * SC_BYTES, scs + (int64_t)di0 * SC_BYTES, nd * SC_BYTES, bar);
-            bulk_g2s(stage + ST_KN + s0 * NIB_BYTES, kns + (int64_t)di0 * NIB_BYTES,
+            bulk_g2s(stage + 512 + s0 * SC_BYTES, scs + (int64_t)di0 * SC_BYTES, nd * SC_BYTES, bar);
+            bulk_g2s(stage + 1024 + s0 * NIB_BYTES, kns + (int64_t)di0 * NIB_BYTES,
                      nd * NIB_BYTES, bar);
-            bulk_g2s(stage + ST_VN + s0 * NIB_BYTES, vns + (int64_t)di0 * NIB_BYTES,
+            bulk_g2s(stage + 3072 + s0 * NIB_BYTES, vns + (int64_t)di0 * NIB_BYTES,
                      nd * NIB_BYTES, bar);
         }
     } else if (FMT == DKV_FMT_Q4_0) {
         const int p0 = c.g * SEG;
         const int npos = min(SEG, c.len_b - p0);
         mbar_arrive_expect_tx(bar, npos * (SC_BYTES + 2 * NIB_BYTES));
-        bulk_g2s(stage + ST_SC, sb + (int64_t)p0 * SC_BYTES, npos * SC_BYTES, bar);
-        bulk_g2s(stage + ST_KN, sb + (int64_t)cv.cap * SC_BYTES + (int64_t)p0 * NIB_BYTES,
+        bulk_g2s(stage + 512, sb + (int64_t)p0 * SC_BYTES, npos * SC_BYTES, bar);
+        bulk_g2s(stage + 1024, sb + (int64_t)cv.cap * SC_BYTES + (int64_t)p0 * NIB_BYTES,
                  npos * NIB_BYTES, bar);
-        bulk_g2s(stage + ST_VN, sb + (int64_t)cv.cap * (SC_BYTES + NIB_BYTES) + (int64_t)p0 * NIB_BYTES,
+        bulk_g2s(stage + 3072, sb + (int64_t)cv.cap * (SC_BYTES + NIB_BYTES) + (int64_t)p0 * NIB_BYTES,
                  npos * NIB_BYTES, bar);
     } else {
         const int p0 = c.g * SEG;
@@ -188,9 +287,6 @@ __device__ inline uint32_t pack_h2(float lo, float hi) {
 }
 __device__ inline float h_lo(uint32_t u) { return __low2float(u32_as_h2(u)); }
 __device__ inline float h_hi(uint32_t u) { return __high2float(u32_as_h2(u)); }
-__device__ inline uint32_t lds32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
-__device__ inline uint2 lds64(const uint8_t *p) { return *reinterpret_cast<const uint2 *>(p); }
-__device__ inline uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
 
 __device__ inline float q_elem(const void *Q, int dt, int64_t i) {
     if (dt == DKV_F32) return static_cast<const float *>(Q)[i];
@@ -205,18 +301,18 @@ __device__ inline float quad_scan32(float (&x)[4][2], int t) {
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
         x[nt][1] += x[nt][0];
-        float own = x[nt][1];
+        const float own = x[nt][1];
         float inc = own;
         float u = __shfl_up_sync(0xffffffffu, inc, 1, 4);
         if (t >= 1) inc += u;
         u = __shfl_up_sync(0xffffffffu, inc, 2, 4);
         if (t >= 2) inc += u;
-        float ex = inc - own;
+        const float ex = inc - own;
         x[nt][0] += ex;
         x[nt][1] += ex;
         tot[nt] = __shfl_sync(0xffffffffu, inc, 3, 4);
     }
-    float c1 = tot[0], c2 = c1 + tot[1], c3 = c2 + tot[2];
+    const float c1 = tot[0], c2 = c1 + tot[1], c3 = c2 + tot[2];
     x[1][0] += c1; x[1][1] += c1;
     x[2][0] += c2; x[2][1] += c2;
     x[3][0] += c3; x[3][1] += c3;
@@ -224,37 +320,20 @@ __device__ inline float quad_scan32(float (&x)[4][2], int t) {
 }
 
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
+__global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(SplitArgs A) {
     using Cfg = FmtCfg<FMT>;
     constexpr int NS = Cfg::NS, STAGE = Cfg::STAGE;
-    extern __shared__ __align__(128) uint8_t smem[];
-    int64_t *plan = reinterpret_cast<int64_t *>(smem);                       // [MAX_B + 1]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 8 * (MAX_B + 1));   // [WARPS][NS]
-    uint8_t *stages = smem + 8 * (MAX_B + 1) + 8 * WARPS * NS + 64;          // 128-aligned below
-    stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(stages) + 127) & ~uintptr_t(127));
+    extern __shared__ __align__(1024) uint8_t smem[];
 
     const CacheView &cv = A.cv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, tq = lane & 3;          // quad row / column of the fragments
-    const int nvs_per_kv = A.NHG;
     const int nvs = cv.Hkv * A.NHG;                    // sequences per batch entry
+    using Map = SmemMap<FMT>;
+    uint64_t *mybar = reinterpret_cast<uint64_t *>(smem + Map::BAR_OFF) + warp * NS;
+    uint8_t *mystages = smem + Map::STAGE_OFF + warp * NS * STAGE;
+    const StageMap sm = stage_map<FMT, MODE>(cv.kf);
 
-    // ---- plan: prefix over batch entries of units ------------------------
-    if (threadIdx.x == 0) {
-        int64_t acc = 0;
-        for (int b = 0; b < cv.B; ++b) {
-            plan[b] = acc;
-            int l = cv.seqlen[b];
-            if (l < 0 || l > cv.cap) {
-                if (blockIdx.x == 0) set_status(cv.header, DKV_DEV_BAD_SEQLEN);
-                l = 0;
-            }
-            acc += (int64_t)nvs * units_of(cv.fmt, cv.kf, l);
-        }
-        plan[cv.B] = acc;
-    }
-    uint64_t *mybar = bars + warp * NS;
-    uint8_t *mystages = stages + (size_t)warp * NS * STAGE;
     if (lane == 0) {
         for (int s = 0; s < NS; ++s) mbar_init(mybar + s, 1);
         fence_mbar_init();
@@ -263,27 +342,40 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
     for (int i = lane; i < NS * STAGE / 16; i += 32)
         reinterpret_cast<uint4 *>(mystages)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async();
-    __syncthreads();
+    __syncwarp();
 
-    const int64_t total = plan[cv.B];
     const int64_t NW = (int64_t)gridDim.x * WARPS;
     const int64_t gw = (int64_t)blockIdx.x * WARPS + warp;
+    int bdummy;
+    int64_t base_dummy;
+    const int64_t total = locate(cv, nvs, -1, bdummy, base_dummy);
+    if (gw == 0 && lane == 0) {
+        for (int b = 0; b < cv.B; ++b) {
+            const int l = cv.seqlen[b];
+            if (l < 0 || l > cv.cap) set_status(cv.header, DKV_DEV_BAD_SEQLEN);
+        }
+    }
     if (total == 0) return;
     const int64_t r0 = range_start(gw, NW, total), r1 = range_start(gw + 1, NW, total);
     if (r0 >= r1) return;
 
-    Cursor ic, cc;
+    Cursor ic;
     ic.x = r0; ic.x_end = r1;
-    cursor_seek(ic, cv, plan, nvs);
-    cc = ic;
+    cursor_seek<MODE>(ic, cv, nvs);
+    StageMeta *mymeta = reinterpret_cast<StageMeta *>(smem + Map::META_OFF) + warp * NS;
 
     // prologue: fill the ring
     uint32_t phase = 0;                 // bit s = parity to wait for on stage s
+    int issued = 0, consumed = 0;
 #pragma unroll 1
     for (int s = 0; s < NS; ++s) {
         if (ic.valid()) {
-            if (lane == 0) issue_stage<FMT>(cv, ic, nvs_per_kv, mystages + s * STAGE, mybar + s);
-            cursor_next(ic, cv, nvs);
+            if (lane == 0) {
+                mymeta[s] = make_meta<MODE>(cv, ic);
+                issue_stage<FMT, MODE>(cv, ic, A.NHG, mystages + s * STAGE, mybar + s);
+            }
+            cursor_next<MODE>(ic, cv, nvs);
+            ++issued;
         }
     }
 
@@ -311,7 +403,7 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
         float l = l_run;
         l += __shfl_xor_sync(0xffffffffu, l, 1);
         l += __shfl_xor_sync(0xffffffffu, l, 2);
-        const int64_t vseq = ((int64_t)cur_b * cv.Hkv) * A.NHG + cur_vs;
+        const int64_t vseq = (int64_t)cur_b * nvs + cur_vs;
         float *rec = A.ws + (gw + vseq) * PARTIAL_FLOATS;
         if (tq == 0) {
             rec[gq] = m_run;
@@ -328,15 +420,27 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
     };
 
 #pragma unroll 1
-    while (cc.valid()) {
+    while (consumed < issued) {
+        // ---- wait for the stage -------------------------------------------
+        const uint8_t *st = mystages + stage_i * STAGE;
+        if (!dead) {
+            if (!mbar_wait_bounded(mybar + stage_i, (phase >> stage_i) & 1)) {
+                dead = true;
+                if (lane == 0) set_status(cv.header, DKV_DEV_TIMEOUT);
+            }
+        }
+        dead = __any_sync(0xffffffffu, dead);
+        phase ^= 1u << stage_i;
+        const StageMeta meta = mymeta[stage_i];
+
         // ---- sequence change: flush, load q --------------------------------
-        if (cc.b != cur_b || cc.vs != cur_vs) {
+        if (!dead && (meta.b != cur_b || meta.vs != cur_vs)) {
             if (cur_b >= 0) flush();
-            cur_b = cc.b; cur_vs = cc.vs;
-            const int kvh = cc.vs / A.NHG, hg = cc.vs % A.NHG;
+            cur_b = meta.b; cur_vs = meta.vs;
+            const int kvh = meta.vs / A.NHG, hg = meta.vs % A.NHG;
             const int hl = hg * 8 + gq;                  // head within the kv group
             head_ok = hl < A.G;
-            const int64_t qrow = ((int64_t)cc.b * A.Hq + (int64_t)kvh * A.G + (head_ok ? hl : 0)) * D;
+            const int64_t qrow = ((int64_t)meta.b * A.Hq + (int64_t)kvh * A.G + (head_ok ? hl : 0)) * D;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int c = 16 * kk + 2 * tq;
@@ -357,34 +461,14 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
                 for (int j = 0; j < 4; ++j) { o[i][j] = 0.f; racc[i][j] = 0.f; }
         }
 
-        // ---- wait for the stage -------------------------------------------
-        uint8_t *st = mystages + stage_i * STAGE;
-        if (!dead) {
-            if (!mbar_wait_bounded(mybar + stage_i, (phase >> stage_i) & 1)) {
-                dead = true;
-                if (lane == 0) set_status(cv.header, DKV_DEV_TIMEOUT);
-            }
-        }
-        dead = __any_sync(0xffffffffu, dead);
-        phase ^= 1u << stage_i;
-
         if (!dead) {
             // positions of this stage: a + slot, slot < npos valid
-            int a, npos;
-            if (FMT == DKV_FMT_DELTA) {
-                const int glen = min(cv.kf, cc.len_b - cc.g * cv.kf);
-                a = cc.seg * SEG;
-                npos = min(SEG, glen - a);
-            } else {
-                a = 0;
-                npos = min(SEG, cc.len_b - cc.g * SEG);
-            }
-            const bool first_seg = (FMT == DKV_FMT_DELTA) && cc.seg == 0;
-            const bool last_seg = cc.seg == cc.nseg - 1;
+            const int npos = meta.npos;
+            const bool first_seg = (FMT == DKV_FMT_DELTA) && (meta.flags & 1);
+            const bool last_seg = (meta.flags & 2) != 0;
 
             // ================= K side: per-position dot products ============
             float x[4][2];
-            uint32_t dvh[4][2][2];   // dV pairs (blocks 0|1, 2|3) per (nt, e)
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int pc = 8 * nt + gq;            // position of this thread's B column
@@ -393,25 +477,26 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
                     const uint8_t *kp = st + pc * 256 + 64 * tq;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 v = lds128(kp + 16 * q4);
+                        const uint4 v = *reinterpret_cast<const uint4 *>(kp + 16 * q4);
                         bf[2 * q4][0] = v.x; bf[2 * q4][1] = v.y;
                         bf[2 * q4 + 1][0] = v.z; bf[2 * q4 + 1][1] = v.w;
                     }
                 } else {
-                    uint4 kw = lds128(st + ST_KN + pc * NIB_BYTES + 16 * tq);
-                    uint32_t ws4[4] = {kw.x, kw.y, kw.z, kw.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dq_word(ws4[j], bf[2 * j][0], bf[2 * j][1], bf[2 * j + 1][0], bf[2 * j + 1][1]);
                     if (first_seg && nt == 0 && gq == 0) {
                         // position 0 is the keyframe: its fp16 values are the B column
-                        const uint8_t *kp = st + ST_KF + 64 * tq;
+                        const uint8_t *kp = st + 64 * tq;
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
-                            uint4 v = lds128(kp + 16 * q4);
+                            const uint4 v = *reinterpret_cast<const uint4 *>(kp + 16 * q4);
                             bf[2 * q4][0] = v.x; bf[2 * q4][1] = v.y;
                             bf[2 * q4 + 1][0] = v.z; bf[2 * q4 + 1][1] = v.w;
                         }
+                    } else {
+                        const uint4 kw = *reinterpret_cast<const uint4 *>(st + sm.kn0 + pc * NIB_BYTES + 16 * tq);
+                        dq_word(kw.x, bf[0][0], bf[0][1], bf[1][0], bf[1][1]);
+                        dq_word(kw.y, bf[2][0], bf[2][1], bf[3][0], bf[3][1]);
+                        dq_word(kw.z, bf[4][0], bf[4][1], bf[5][0], bf[5][1]);
+                        dq_word(kw.w, bf[6][0], bf[6][1], bf[7][0], bf[7][1]);
                     }
                 }
                 if (FMT == DKV_FMT_FP16) {
@@ -430,33 +515,26 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
                         mma16816(acc[j], qa[2 * j + 1][0], 0u, qa[2 * j + 1][1], 0u, bf[2 * j + 1][0],
                                  bf[2 * j + 1][1]);
                     }
-                    // scales of positions 8nt + 2t + e
+                    // K scales of positions 8nt + 2t + e
                     const int pa = 8 * nt + 2 * tq;
-                    uint4 s0 = lds128(st + ST_SC + pa * SC_BYTES);
-                    uint4 s1 = lds128(st + ST_SC + (pa + 1) * SC_BYTES);
-                    if (first_seg && nt == 0 && tq == 0) {
-                        // keyframe column: unit K weights; V weight 1 (SUFFIX) or 0 (PREFIX)
-                        s0.x = s0.y = 0x3C003C00u;
-                        s0.z = s0.w = (MODE == SUFFIX) ? 0x3C003C00u : 0u;
-                    }
-                    // slots past the end of the unit hold stale data: no V weight
-                    if (pa >= npos) s0.z = s0.w = 0u;
-                    if (pa + 1 >= npos) s1.z = s1.w = 0u;
+                    uint2 s0 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + pa * SC_BYTES);
+                    const uint2 s1 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + (pa + 1) * SC_BYTES);
+                    if (first_seg && nt == 0 && tq == 0) s0.x = s0.y = 0x3C003C00u;  // keyframe: unit weights
                     x[nt][0] = acc[0][0] * h_lo(s0.x) + acc[1][0] * h_hi(s0.x) +
                                acc[2][0] * h_lo(s0.y) + acc[3][0] * h_hi(s0.y);
                     x[nt][1] = acc[0][1] * h_lo(s1.x) + acc[1][1] * h_hi(s1.x) +
                                acc[2][1] * h_lo(s1.y) + acc[3][1] * h_hi(s1.y);
-                    dvh[nt][0][0] = s0.z; dvh[nt][0][1] = s0.w;
-                    dvh[nt][1][0] = s1.z; dvh[nt][1][1] = s1.w;
                 }
             }
 
             // ================= scores, online softmax =======================
             if (MODE != PLAIN) {
                 quad_scan32(x, tq);
+                if (MODE == PREFIX) {
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt) { x[nt][0] += dot_carry; x[nt][1] += dot_carry; }
-                dot_carry = __shfl_sync(0xffffffffu, x[3][1], 3, 4);
+                    for (int nt = 0; nt < 4; ++nt) { x[nt][0] += dot_carry; x[nt][1] += dot_carry; }
+                    dot_carry = __shfl_sync(0xffffffffu, x[3][1], 3, 4);
+                }
             }
             float mx = -INFINITY;
 #pragma unroll
@@ -510,19 +588,22 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
                 for (int nt = 0; nt < 4; ++nt) { wgt[nt][0] = x[nt][0]; wgt[nt][1] = x[nt][1]; }
             }
 
-            // rescale the output accumulators (heads 2t, 2t+1 in the V layout)
-            const float al0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
-            const float al1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
+            // rescale the output accumulators (heads 2t, 2t+1 in the V layout),
+            // only when some head's running max moved
+            if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+                const float al0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
+                const float al1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
+                for (int mt = 0; mt < 8; ++mt) {
+                    o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
+                }
             }
 
             // ================= V side ======================================
             uint32_t vkf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
             if (FMT == DKV_FMT_DELTA && first_seg) {
-                uint4 v0 = lds128(st + ST_KF + 256 + 32 * gq);
-                uint4 v1 = lds128(st + ST_KF + 256 + 32 * gq + 16);
+                const uint4 v0 = *reinterpret_cast<const uint4 *>(st + 256 + 32 * gq);
+                const uint4 v1 = *reinterpret_cast<const uint4 *>(st + 256 + 32 * gq + 16);
                 vkf[0] = v0.x; vkf[1] = v0.y; vkf[2] = v0.z; vkf[3] = v0.w;
                 vkf[4] = v1.x; vkf[5] = v1.y; vkf[6] = v1.z; vkf[7] = v1.w;
                 if (MODE == PREFIX) {
@@ -532,23 +613,35 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
             }
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
-                // B' fragments: rows = positions 16kk + {2t,2t+1} | {2t+8, 2t+9}, col = head g
+                const int sA = 16 * kk + 2 * tq;
+                // V scales of the four positions this thread weights
+                uint2 dv[4] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u),
+                               make_uint2(0u, 0u)};
+                if (FMT != DKV_FMT_FP16) {
+                    const int ps[4] = {sA, sA + 1, sA + 8, sA + 9};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        dv[i] = *reinterpret_cast<const uint2 *>(st + sm.sc0 + ps[i] * SC_BYTES + 8);
+                        if (ps[i] >= npos) dv[i] = make_uint2(0u, 0u);  // stale slot: no weight
+                    }
+                    if (FMT == DKV_FMT_DELTA && first_seg && kk == 0 && tq == 0)
+                        dv[0] = (MODE == SUFFIX) ? make_uint2(0x3C003C00u, 0x3C003C00u)
+                                                 : make_uint2(0u, 0u);  // keyframe row
+                }
                 // B' fragments: rows = positions 16kk + {2t,2t+1} | {2t+8, 2t+9}, col = head g.
                 // For the delta format a weight multiplies a whole dequantised row
                 // (the keyframe row, or a large delta) and its rounding is shared by
                 // every channel, so it is carried as an fp16 hi + lo pair (about
                 // 22 significant bits); the comparators weight one token per row and
                 // use a single fp16 weight, as flash-decoding does.
+                const float w0 = wgt[2 * kk][0], w1 = wgt[2 * kk][1];
+                const float w2 = wgt[2 * kk + 1][0], w3 = wgt[2 * kk + 1][1];
                 auto make_bp = [&](int j, uint32_t (&hi)[2], uint32_t (&lo)[2]) {
-                    const int hw = j >> 1;
-                    auto dv = [&](int nt, int e) {
-                        uint32_t u = dvh[nt][e][hw];
+                    auto d = [&](int i) {
+                        const uint32_t u = (j >> 1) ? dv[i].y : dv[i].x;
                         return (j & 1) ? h_hi(u) : h_lo(u);
                     };
-                    const float v0 = wgt[2 * kk][0] * dv(2 * kk, 0);
-                    const float v1 = wgt[2 * kk][1] * dv(2 * kk, 1);
-                    const float v2 = wgt[2 * kk + 1][0] * dv(2 * kk + 1, 0);
-                    const float v3 = wgt[2 * kk + 1][1] * dv(2 * kk + 1, 1);
+                    const float v0 = w0 * d(0), v1 = w1 * d(1), v2 = w2 * d(2), v3 = w3 * d(3);
                     hi[0] = pack_h2(v0, v1);
                     hi[1] = pack_h2(v2, v3);
                     if (FMT == DKV_FMT_DELTA) {
@@ -558,20 +651,21 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
                 };
                 uint32_t bp[2] = {0u, 0u}, bl[2] = {0u, 0u};
                 if (FMT == DKV_FMT_FP16) {
-                    bp[0] = pack_h2(wgt[2 * kk][0], wgt[2 * kk][1]);
-                    bp[1] = pack_h2(wgt[2 * kk + 1][0], wgt[2 * kk + 1][1]);
-                }
-                const int sA = 16 * kk + 2 * tq;
-                if (FMT == DKV_FMT_FP16) {
+                    bp[0] = pack_h2(w0, w1);
+                    bp[1] = pack_h2(w2, w3);
                     const uint8_t *vb = st + 8192 + 32 * gq;
-                    uint4 A0 = lds128(vb + sA * 256), A1 = lds128(vb + sA * 256 + 16);
-                    uint4 B0 = lds128(vb + (sA + 1) * 256), B1 = lds128(vb + (sA + 1) * 256 + 16);
-                    uint4 C0 = lds128(vb + (sA + 8) * 256), C1 = lds128(vb + (sA + 8) * 256 + 16);
-                    uint4 D0 = lds128(vb + (sA + 9) * 256), D1 = lds128(vb + (sA + 9) * 256 + 16);
-                    uint32_t wa[8] = {A0.x, A0.y, A0.z, A0.w, A1.x, A1.y, A1.z, A1.w};
-                    uint32_t wb[8] = {B0.x, B0.y, B0.z, B0.w, B1.x, B1.y, B1.z, B1.w};
-                    uint32_t wc[8] = {C0.x, C0.y, C0.z, C0.w, C1.x, C1.y, C1.z, C1.w};
-                    uint32_t wd[8] = {D0.x, D0.y, D0.z, D0.w, D1.x, D1.y, D1.z, D1.w};
+                    const uint4 A0 = *reinterpret_cast<const uint4 *>(vb + sA * 256);
+                    const uint4 A1 = *reinterpret_cast<const uint4 *>(vb + sA * 256 + 16);
+                    const uint4 B0 = *reinterpret_cast<const uint4 *>(vb + (sA + 1) * 256);
+                    const uint4 B1 = *reinterpret_cast<const uint4 *>(vb + (sA + 1) * 256 + 16);
+                    const uint4 C0 = *reinterpret_cast<const uint4 *>(vb + (sA + 8) * 256);
+                    const uint4 C1 = *reinterpret_cast<const uint4 *>(vb + (sA + 8) * 256 + 16);
+                    const uint4 D0 = *reinterpret_cast<const uint4 *>(vb + (sA + 9) * 256);
+                    const uint4 D1 = *reinterpret_cast<const uint4 *>(vb + (sA + 9) * 256 + 16);
+                    const uint32_t wa[8] = {A0.x, A0.y, A0.z, A0.w, A1.x, A1.y, A1.z, A1.w};
+                    const uint32_t wb[8] = {B0.x, B0.y, B0.z, B0.w, B1.x, B1.y, B1.z, B1.w};
+                    const uint32_t wc[8] = {C0.x, C0.y, C0.z, C0.w, C1.x, C1.y, C1.z, C1.w};
+                    const uint32_t wd[8] = {D0.x, D0.y, D0.z, D0.w, D1.x, D1.y, D1.z, D1.w};
 #pragma unroll
                     for (int mt = 0; mt < 8; ++mt) {
                         const uint32_t a0 = prmt(wa[mt], wb[mt], 0x5410u);
@@ -581,11 +675,11 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
                         mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
                     }
                 } else {
-                    const uint8_t *vb = st + ST_VN + 8 * gq;
-                    const uint2 wA = lds64(vb + sA * NIB_BYTES);
-                    const uint2 wB = lds64(vb + (sA + 1) * NIB_BYTES);
-                    const uint2 wC = lds64(vb + (sA + 8) * NIB_BYTES);
-                    const uint2 wD = lds64(vb + (sA + 9) * NIB_BYTES);
+                    const uint8_t *vb = st + sm.vn0 + 8 * gq;
+                    const uint2 wA = *reinterpret_cast<const uint2 *>(vb + sA * NIB_BYTES);
+                    const uint2 wB = *reinterpret_cast<const uint2 *>(vb + (sA + 1) * NIB_BYTES);
+                    const uint2 wC = *reinterpret_cast<const uint2 *>(vb + (sA + 8) * NIB_BYTES);
+                    const uint2 wD = *reinterpret_cast<const uint2 *>(vb + (sA + 9) * NIB_BYTES);
                     const bool kfrow = (FMT == DKV_FMT_DELTA) && (MODE == SUFFIX) && first_seg &&
                                        kk == 0 && tq == 0;
                     const uint32_t sel0 = kfrow ? 0x3254u : 0x3210u;
@@ -617,16 +711,12 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
                         if (FMT == DKV_FMT_DELTA) mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
                         if (MODE == PREFIX) {
                             // R += sum_s (code-8) * d_s : B = the scales alone
-                            uint32_t r0, r1;
-                            {
-                                const int hw = j >> 1;
-                                auto dv = [&](int nt, int e) {
-                                    uint32_t u = dvh[nt][e][hw];
-                                    return (j & 1) ? h_hi(u) : h_lo(u);
-                                };
-                                r0 = pack_h2(dv(2 * kk, 0), dv(2 * kk, 1));
-                                r1 = pack_h2(dv(2 * kk + 1, 0), dv(2 * kk + 1, 1));
-                            }
+                            auto d = [&](int i2) {
+                                const uint32_t u = (j >> 1) ? dv[i2].y : dv[i2].x;
+                                return (j & 1) ? h_hi(u) : h_lo(u);
+                            };
+                            const uint32_t r0 = pack_h2(d(0), d(1));
+                            const uint32_t r1 = pack_h2(d(2), d(3));
                             mma16816(racc[mt], a0, a1, a2, a3, r0, r1);
                         }
                     }
@@ -647,30 +737,33 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(SplitArgs A) {
                 }
                 e_carry = 0.f;
                 dot_carry = 0.f;
-            } else if (MODE == SUFFIX) {
-                dot_carry = 0.f;
             }
         }
 
         // ---- release the stage and refill it ------------------------------
         __syncwarp();
-        if (ic.valid()) {
-            if (lane == 0 && !dead) {
+        ++consumed;
+        if (ic.valid() && !dead) {
+            if (lane == 0) {
                 fence_proxy_async();
-                issue_stage<FMT>(cv, ic, nvs_per_kv, mystages + stage_i * STAGE, mybar + stage_i);
+                mymeta[stage_i] = make_meta<MODE>(cv, ic);
+                issue_stage<FMT, MODE>(cv, ic, A.NHG, mystages + stage_i * STAGE, mybar + stage_i);
             }
-            cursor_next(ic, cv, nvs);
+            cursor_next<MODE>(ic, cv, nvs);
+            ++issued;
         }
         stage_i = (stage_i + 1 == NS) ? 0 : stage_i + 1;
-        cursor_next(cc, cv, nvs);
     }
     if (cur_b >= 0) flush();
 
     // A warp that gave up still owns copies in flight: wait for them (bounded)
     // before the CTA can exit and its shared memory be reused.
     if (dead) {
-        for (int s = 0; s < NS; ++s) {
-            if (lane == 0) (void)mbar_wait_bounded(mybar + s, (phase >> s) & 1);
+        int si = stage_i;
+        for (int k = consumed; k < issued; ++k) {
+            if (lane == 0) (void)mbar_wait_bounded(mybar + si, (phase >> si) & 1);
+            phase ^= 1u << si;
+            si = (si + 1 == NS) ? 0 : si + 1;
         }
         __syncwarp();
     }
@@ -683,22 +776,27 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
                                                     int64_t NW, const float *ws, float *out) {
     const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
     const int nvs = cv.Hkv * NHG;
-    __shared__ int64_t sh_plan[2];
-    __shared__ int64_t sh_total;
-    if (threadIdx.x == 0) {
-        int64_t acc = 0, mine = 0;
-        for (int bb = 0; bb < cv.B; ++bb) {
-            if (bb == b) mine = acc;
-            int l = cv.seqlen[bb];
-            if (l < 0 || l > cv.cap) l = 0;
-            acc += (int64_t)nvs * units_of(cv.fmt, cv.kf, l);
+    __shared__ int64_t sh_base, sh_total;
+    if (threadIdx.x < 32) {
+        int bb;
+        int64_t bdummy;
+        const int64_t total = locate(cv, nvs, -1, bb, bdummy);
+        // units of the batch entries before b
+        int64_t mine = 0;
+        for (int b0 = 0; b0 < b; b0 += 32) {
+            const int xb = b0 + (int)threadIdx.x;
+            int64_t u = xb < b ? (int64_t)nvs * units_of(cv.fmt, cv.kf, clamp_len(cv, xb)) : 0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+            mine += u;
         }
-        sh_plan[0] = mine;
-        sh_total = acc;
+        if (threadIdx.x == 0) {
+            sh_base = mine;
+            sh_total = total;
+        }
     }
     __syncthreads();
-    int len = cv.seqlen[b];
-    if (len < 0 || len > cv.cap) len = 0;
+    const int len = clamp_len(cv, b);
     const int ub = units_of(cv.fmt, cv.kf, len);
     float *dst = out + ((int64_t)b * Hq + h) * D;
     if (ub == 0) { dst[c] = 0.f; return; }
@@ -706,7 +804,7 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
     const int vsl = kvh * NHG + hg;
     const int64_t vseq = (int64_t)b * nvs + vsl;
     const int64_t T = sh_total;
-    const int64_t xs = sh_plan[0] + (int64_t)vsl * ub, xe = xs + ub;
+    const int64_t xs = sh_base + (int64_t)vsl * ub, xe = xs + ub;
     const int64_t w0 = warp_of(xs, NW, T), w1 = warp_of(xe - 1, NW, T);
     float M = -INFINITY;
     for (int64_t w = w0; w <= w1; ++w) {
@@ -729,8 +827,7 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
 // ---------------------------------------------------------------------------
 template <int FMT, int MODE>
 static size_t split_smem() {
-    using Cfg = FmtCfg<FMT>;
-    return 8 * (MAX_B + 1) + 8 * WARPS * Cfg::NS + 64 + 128 + (size_t)WARPS * Cfg::NS * Cfg::STAGE;
+    return (size_t)SmemMap<FMT>::BYTES;
 }
 
 template <int FMT, int MODE>
