@@ -102,12 +102,13 @@ __device__ inline int clamp_len(const CacheView &cv, int b) {
 
 // Iterates the (unit, segment) stage items of one warp's range in order.
 struct Cursor {
-    int64_t x, x_end;          // flattened unit index, end of range
+    int64_t left;              // units left in the range, the current one included
     int b, vs, g;              // batch entry, sequence within the batch entry, unit
     int units_b;               // units per sequence of batch entry b
     int len_b;                 // tokens of batch entry b
     int seg, nseg;             // segment within the unit (kf > 32 only)
-    __device__ bool valid() const { return x < x_end; }
+    const uint8_t *seq;        // data of sequence (b, kv head of vs)
+    __device__ bool valid() const { return left > 0; }
 };
 
 template <int MODE>
@@ -146,27 +147,34 @@ __device__ inline int64_t locate(const CacheView &cv, int nvs, int64_t r, int &b
     return base;
 }
 
+__device__ inline const uint8_t *seq_ptr(const CacheView &cv, int b, int vs, int nhg) {
+    const int kvh = nhg == 1 ? vs : vs / nhg;
+    return cv.data + ((int64_t)b * cv.Hkv + kvh) * cv.seq_stride;
+}
+
 template <int MODE>
-__device__ inline void cursor_seek(Cursor &c, const CacheView &cv, int nvs) {
+__device__ inline void cursor_seek(Cursor &c, const CacheView &cv, int nvs, int nhg, int64_t x,
+                                   int64_t count) {
     int b;
     int64_t base;
-    locate(cv, nvs, c.x, b, base);
+    locate(cv, nvs, x, b, base);
+    c.left = count;
     c.b = b;
     c.len_b = clamp_len(cv, b);
     c.units_b = units_of(cv.fmt, cv.kf, c.len_b);
-    const int64_t r = c.x - base;
+    const int64_t r = x - base;
     c.vs = (int)(r / c.units_b);
     c.g = (int)(r % c.units_b);
     c.seg = 0;
     c.nseg = nseg_of<MODE>(cv, c.len_b, c.g);
+    c.seq = seq_ptr(cv, c.b, c.vs, nhg);
 }
 
 template <int MODE>
-__device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs) {
+__device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs, int nhg) {
     if (MODE == PREFIX && ++c.seg < c.nseg) return;
     c.seg = 0;
-    ++c.x;
-    if (!c.valid()) return;
+    if (--c.left == 0) return;
     if (++c.g == c.units_b) {
         c.g = 0;
         if (++c.vs == nvs) {
@@ -177,8 +185,9 @@ __device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs) {
                 c.units_b = units_of(cv.fmt, cv.kf, c.len_b);
             } while (c.units_b == 0);
         }
+        c.seq = seq_ptr(cv, c.b, c.vs, nhg);
     }
-    c.nseg = nseg_of<MODE>(cv, c.len_b, c.g);
+    if (MODE == PREFIX) c.nseg = nseg_of<MODE>(cv, c.len_b, c.g);
 }
 
 // Stage layouts in shared memory (offsets from the stage start):
@@ -235,8 +244,8 @@ __device__ inline StageMeta make_meta(const CacheView &cv, const Cursor &c) {
 template <int FMT, int MODE>
 __device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nhg,
                                    uint8_t *stage, uint64_t *bar) {
-    const int kvh = c.vs / nhg;
-    const uint8_t *sb = cv.data + ((int64_t)c.b * cv.Hkv + kvh) * cv.seq_stride;
+    (void)nhg;
+    const uint8_t *sb = c.seq;
     if (FMT == DKV_FMT_DELTA && MODE == SUFFIX) {
         const uint32_t bytes = (uint32_t)cv.rec_bytes;
         mbar_arrive_expect_tx(bar, bytes);
@@ -294,31 +303,46 @@ __device__ inline float q_elem(const void *Q, int dt, int64_t i) {
     return __bfloat162float(static_cast<const __nv_bfloat16 *>(Q)[i]);
 }
 
-// Inclusive scan over the 32 positions (8*nt + 2*t + e) of one head, held as
-// x[nt][e] across the 4 lanes of a quad.  Returns the total (all lanes).
-__device__ inline float quad_scan32(float (&x)[4][2], int t) {
-    float tot[4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-        x[nt][1] += x[nt][0];
-        const float own = x[nt][1];
-        float inc = own;
-        float u = __shfl_up_sync(0xffffffffu, inc, 1, 4);
-        if (t >= 1) inc += u;
-        u = __shfl_up_sync(0xffffffffu, inc, 2, 4);
-        if (t >= 2) inc += u;
-        const float ex = inc - own;
-        x[nt][0] += ex;
-        x[nt][1] += ex;
-        tot[nt] = __shfl_sync(0xffffffffu, inc, 3, 4);
-    }
-    const float c1 = tot[0], c2 = c1 + tot[1], c3 = c2 + tot[2];
-    x[1][0] += c1; x[1][1] += c1;
-    x[2][0] += c2; x[2][1] += c2;
-    x[3][0] += c3; x[3][1] += c3;
-    return c3 + tot[3];
+__device__ inline uint32_t movm_t(uint32_t a) {
+    uint32_t d;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+    return d;
+}
+__device__ inline float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
 }
 
+// Inclusive prefix over the 32 positions 4g + i (i = 0..3) of one head, held
+// as v[i] by the 8 lanes g of one column (lane % 4).  Returns the total over
+// the 32 positions (every lane).
+__device__ inline float col_scan32(float (&v)[4], int lane) {
+    v[1] += v[0];
+    v[2] += v[1];
+    v[3] += v[2];
+    const float own = v[3];
+    float inc = own;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
+    }
+    const float ex = inc - own;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] += ex;
+    return __shfl_sync(0xffffffffu, inc, 28 + (lane & 3));
+}
+
+// Per stage (up to 32 positions), per thread of lane (g, t4):
+//  K side, tile t: m16n8k16 with rows = positions (row g <-> 4g + 2t, row
+//   g+8 <-> 4g + 2t + 1), k = channels, n = heads; the accumulator holds
+//   x[t][r][e] for position 4g + 2t + r, head 2t4 + e, so each thread owns
+//   the four consecutive positions 4g..4g+3 of two heads.
+//  V side, tile t: m16n8k16 with rows = channels, k = positions
+//   (k 2t4, 2t4+1 <-> 8t4 + 2t, +4; k 2t4+8, 2t4+9 <-> 8t4 + 2t + 1, +5),
+//   n = heads; the weights reach that B layout through an 8x8 transpose
+//   (movmatrix) of the K-side accumulator layout.
 template <int FMT, int MODE>
 __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(SplitArgs A) {
     using Cfg = FmtCfg<FMT>;
@@ -333,6 +357,7 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
     uint64_t *mybar = reinterpret_cast<uint64_t *>(smem + Map::BAR_OFF) + warp * NS;
     uint8_t *mystages = smem + Map::STAGE_OFF + warp * NS * STAGE;
     const StageMap sm = stage_map<FMT, MODE>(cv.kf);
+    const uint32_t magic = magic_1024x2();
 
     if (lane == 0) {
         for (int s = 0; s < NS; ++s) mbar_init(mybar + s, 1);
@@ -360,8 +385,7 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
     if (r0 >= r1) return;
 
     Cursor ic;
-    ic.x = r0; ic.x_end = r1;
-    cursor_seek<MODE>(ic, cv, nvs);
+    cursor_seek<MODE>(ic, cv, nvs, A.NHG, r0, r1 - r0);
     StageMeta *mymeta = reinterpret_cast<StageMeta *>(smem + Map::META_OFF) + warp * NS;
 
     // prologue: fill the ring
@@ -374,7 +398,7 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
                 mymeta[s] = make_meta<MODE>(cv, ic);
                 issue_stage<FMT, MODE>(cv, ic, A.NHG, mystages + s * STAGE, mybar + s);
             }
-            cursor_next<MODE>(ic, cv, nvs);
+            cursor_next<MODE>(ic, cv, nvs, A.NHG);
             ++issued;
         }
     }
@@ -382,14 +406,14 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
     bool dead = false;
     int stage_i = 0;
 
-    // per-sequence state
+    // per-sequence state (heads 2*tq + e of the current head group)
     int cur_b = -1, cur_vs = -1;
-    uint32_t qa[8][2];                  // A fragments of q (rows = heads)
-    bool head_ok = false;
-    float m_run = -1e30f, l_run = 0.f;
+    uint32_t qb[8][2];                  // B fragments of q (column = head gq)
+    bool head_ok[2] = {false, false};
+    float m_run[2] = {-1e30f, -1e30f}, l_run[2] = {0.f, 0.f};
     float o[8][4];
     float racc[8][4];                   // PREFIX: sum of dequantised deltas of the group
-    float dot_carry = 0.f, e_carry = 0.f;
+    float dot_carry[2] = {0.f, 0.f}, e_carry[2] = {0.f, 0.f};
     uint32_t vkf_keep[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -400,14 +424,21 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
 
     auto flush = [&]() {
         // write the partial record of the current sequence
-        float l = l_run;
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float l = l_run[e];
+            l += __shfl_xor_sync(0xffffffffu, l, 4);
+            l += __shfl_xor_sync(0xffffffffu, l, 8);
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
+            l_run[e] = l;
+        }
         const int64_t vseq = (int64_t)cur_b * nvs + cur_vs;
         float *rec = A.ws + (gw + vseq) * PARTIAL_FLOATS;
-        if (tq == 0) {
-            rec[gq] = m_run;
-            rec[8 + gq] = l;
+        if (gq == 0) {
+            rec[2 * tq] = m_run[0];
+            rec[2 * tq + 1] = m_run[1];
+            rec[8 + 2 * tq] = l_run[0];
+            rec[8 + 2 * tq + 1] = l_run[1];
         }
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
@@ -438,23 +469,28 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
             if (cur_b >= 0) flush();
             cur_b = meta.b; cur_vs = meta.vs;
             const int kvh = meta.vs / A.NHG, hg = meta.vs % A.NHG;
-            const int hl = hg * 8 + gq;                  // head within the kv group
-            head_ok = hl < A.G;
-            const int64_t qrow = ((int64_t)meta.b * A.Hq + (int64_t)kvh * A.G + (head_ok ? hl : 0)) * D;
+            const int hl = hg * 8 + gq;                  // head of this thread's q column
+            const bool qok = hl < A.G;
+            head_ok[0] = hg * 8 + 2 * tq < A.G;
+            head_ok[1] = hg * 8 + 2 * tq + 1 < A.G;
+            const int64_t qrow = ((int64_t)meta.b * A.Hq + (int64_t)kvh * A.G + (qok ? hl : 0)) * D;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int c = 16 * kk + 2 * tq;
                 float q0 = 0.f, q1 = 0.f, q8 = 0.f, q9 = 0.f;
-                if (head_ok) {
+                if (qok) {
                     q0 = q_elem(A.Q, A.q_dtype, qrow + c);
                     q1 = q_elem(A.Q, A.q_dtype, qrow + c + 1);
                     q8 = q_elem(A.Q, A.q_dtype, qrow + c + 8);
                     q9 = q_elem(A.Q, A.q_dtype, qrow + c + 9);
                 }
-                qa[kk][0] = pack_h2(q0, q1);
-                qa[kk][1] = pack_h2(q8, q9);
+                qb[kk][0] = pack_h2(q0, q1);
+                qb[kk][1] = pack_h2(q8, q9);
             }
-            m_run = -1e30f; l_run = 0.f; dot_carry = 0.f; e_carry = 0.f;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                m_run[e] = -1e30f; l_run[e] = 0.f; dot_carry[e] = 0.f; e_carry[e] = 0.f;
+            }
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -462,140 +498,149 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
         }
 
         if (!dead) {
-            // positions of this stage: a + slot, slot < npos valid
             const int npos = meta.npos;
             const bool first_seg = (FMT == DKV_FMT_DELTA) && (meta.flags & 1);
             const bool last_seg = (meta.flags & 2) != 0;
+            const bool kfrow = first_seg && gq == 0;   // this thread's row 0 of tile 0 is the keyframe
 
             // ================= K side: per-position dot products ============
-            float x[4][2];
+            float x[2][2][2];                   // [tile][r][e]: position 16t+2g+r, head 2tq+e
+            uint32_t dvw[2][2][2];              // V scales [tile][r][blocks 01 | 23]
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int pc = 8 * nt + gq;            // position of this thread's B column
-                uint32_t bf[8][2];
+            for (int t = 0; t < 2; ++t) {
+                const int p0 = 4 * gq + 2 * t;             // positions p0, p0 + 1
                 if (FMT == DKV_FMT_FP16) {
-                    const uint8_t *kp = st + pc * 256 + 64 * tq;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    const uint8_t *k0 = st + p0 * 256 + 64 * tq;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(kp + 16 * q4);
-                        bf[2 * q4][0] = v.x; bf[2 * q4][1] = v.y;
-                        bf[2 * q4 + 1][0] = v.z; bf[2 * q4 + 1][1] = v.w;
+                        const uint4 u0 = *reinterpret_cast<const uint4 *>(k0 + 16 * q4);
+                        const uint4 u1 = *reinterpret_cast<const uint4 *>(k0 + 256 + 16 * q4);
+                        mma16816(acc, u0.x, u1.x, u0.y, u1.y, qb[2 * q4][0], qb[2 * q4][1]);
+                        mma16816(acc, u0.z, u1.z, u0.w, u1.w, qb[2 * q4 + 1][0], qb[2 * q4 + 1][1]);
                     }
+                    x[t][0][0] = acc[0]; x[t][0][1] = acc[1];
+                    x[t][1][0] = acc[2]; x[t][1][1] = acc[3];
                 } else {
-                    if (first_seg && nt == 0 && gq == 0) {
-                        // position 0 is the keyframe: its fp16 values are the B column
+                    const uint4 w0 = *reinterpret_cast<const uint4 *>(st + sm.kn0 + p0 * NIB_BYTES + 16 * tq);
+                    const uint4 w1 = *reinterpret_cast<const uint4 *>(st + sm.kn0 + (p0 + 1) * NIB_BYTES + 16 * tq);
+                    uint32_t a[8][4];
+                    {
+                        const uint32_t ww0[4] = {w0.x, w0.y, w0.z, w0.w};
+                        const uint32_t ww1[4] = {w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            dq_word(ww0[j], magic, a[2 * j][0], a[2 * j][2], a[2 * j + 1][0], a[2 * j + 1][2]);
+                            dq_word(ww1[j], magic, a[2 * j][1], a[2 * j][3], a[2 * j + 1][1], a[2 * j + 1][3]);
+                        }
+                    }
+                    if (t == 0 && first_seg) {
+                        // position 0 is the keyframe: its fp16 values fill rows g = 0
                         const uint8_t *kp = st + 64 * tq;
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             const uint4 v = *reinterpret_cast<const uint4 *>(kp + 16 * q4);
-                            bf[2 * q4][0] = v.x; bf[2 * q4][1] = v.y;
-                            bf[2 * q4 + 1][0] = v.z; bf[2 * q4 + 1][1] = v.w;
+                            a[2 * q4][0] = kfrow ? v.x : a[2 * q4][0];
+                            a[2 * q4][2] = kfrow ? v.y : a[2 * q4][2];
+                            a[2 * q4 + 1][0] = kfrow ? v.z : a[2 * q4 + 1][0];
+                            a[2 * q4 + 1][2] = kfrow ? v.w : a[2 * q4 + 1][2];
                         }
-                    } else {
-                        const uint4 kw = *reinterpret_cast<const uint4 *>(st + sm.kn0 + pc * NIB_BYTES + 16 * tq);
-                        dq_word(kw.x, bf[0][0], bf[0][1], bf[1][0], bf[1][1]);
-                        dq_word(kw.y, bf[2][0], bf[2][1], bf[3][0], bf[3][1]);
-                        dq_word(kw.z, bf[4][0], bf[4][1], bf[5][0], bf[5][1]);
-                        dq_word(kw.w, bf[6][0], bf[6][1], bf[7][0], bf[7][1]);
                     }
-                }
-                if (FMT == DKV_FMT_FP16) {
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma16816(acc, qa[kk][0], 0u, qa[kk][1], 0u, bf[kk][0], bf[kk][1]);
-                    x[nt][0] = acc[0];
-                    x[nt][1] = acc[1];
-                } else {
                     float acc[4][4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-                        mma16816(acc[j], qa[2 * j][0], 0u, qa[2 * j][1], 0u, bf[2 * j][0], bf[2 * j][1]);
-                        mma16816(acc[j], qa[2 * j + 1][0], 0u, qa[2 * j + 1][1], 0u, bf[2 * j + 1][0],
-                                 bf[2 * j + 1][1]);
+                        mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
+                                 qb[2 * j][0], qb[2 * j][1]);
+                        mma16816(acc[j], a[2 * j + 1][0], a[2 * j + 1][1], a[2 * j + 1][2],
+                                 a[2 * j + 1][3], qb[2 * j + 1][0], qb[2 * j + 1][1]);
                     }
-                    // K scales of positions 8nt + 2t + e
-                    const int pa = 8 * nt + 2 * tq;
-                    uint2 s0 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + pa * SC_BYTES);
-                    const uint2 s1 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + (pa + 1) * SC_BYTES);
-                    if (first_seg && nt == 0 && tq == 0) s0.x = s0.y = 0x3C003C00u;  // keyframe: unit weights
-                    x[nt][0] = acc[0][0] * h_lo(s0.x) + acc[1][0] * h_hi(s0.x) +
-                               acc[2][0] * h_lo(s0.y) + acc[3][0] * h_hi(s0.y);
-                    x[nt][1] = acc[0][1] * h_lo(s1.x) + acc[1][1] * h_hi(s1.x) +
-                               acc[2][1] * h_lo(s1.y) + acc[3][1] * h_hi(s1.y);
+                    // scales of positions p0, p0+1: dK (blocks 0..3) then dV
+                    uint4 s0 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + p0 * SC_BYTES);
+                    uint4 s1 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + (p0 + 1) * SC_BYTES);
+                    if (t == 0 && kfrow) {
+                        s0.x = s0.y = 0x3C003C00u;                          // keyframe: unit K weights
+                        s0.z = s0.w = (MODE == SUFFIX) ? 0x3C003C00u : 0u;  // V: 1 (SUFFIX) / 0 (PREFIX)
+                    }
+                    // slots past the end of the unit hold stale bytes (possibly NaN
+                    // patterns): zero their K and V scales so they add nothing to the
+                    // prefix sums and carry no V weight
+                    if (p0 >= npos) s0 = make_uint4(0u, 0u, 0u, 0u);
+                    if (p0 + 1 >= npos) s1 = make_uint4(0u, 0u, 0u, 0u);
+                    dvw[t][0][0] = s0.z; dvw[t][0][1] = s0.w;
+                    dvw[t][1][0] = s1.z; dvw[t][1][1] = s1.w;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        x[t][0][e] = acc[0][e] * h_lo(s0.x) + acc[1][e] * h_hi(s0.x) +
+                                     acc[2][e] * h_lo(s0.y) + acc[3][e] * h_hi(s0.y);
+                        x[t][1][e] = acc[0][2 + e] * h_lo(s1.x) + acc[1][2 + e] * h_hi(s1.x) +
+                                     acc[2][2 + e] * h_lo(s1.y) + acc[3][2 + e] * h_hi(s1.y);
+                    }
                 }
             }
 
             // ================= scores, online softmax =======================
-            if (MODE != PLAIN) {
-                quad_scan32(x, tq);
-                if (MODE == PREFIX) {
+            float alpha[2];
 #pragma unroll
-                    for (int nt = 0; nt < 4; ++nt) { x[nt][0] += dot_carry; x[nt][1] += dot_carry; }
-                    dot_carry = __shfl_sync(0xffffffffu, x[3][1], 3, 4);
+            for (int e = 0; e < 2; ++e) {
+                // v[i]: position 4g + i  (i = 2t + r)
+                float v[4] = {x[0][0][e], x[0][1][e], x[1][0][e], x[1][1][e]};
+                if (MODE != PLAIN) {
+                    const float tot = col_scan32(v, lane);
+                    if (MODE == PREFIX) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) v[i] += dot_carry[e];
+                        dot_carry[e] += tot;
+                    }
                 }
-            }
-            float mx = -INFINITY;
+                float mx = -INFINITY;
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int slot = 8 * nt + 2 * tq + e;
-                    const bool ok = head_ok && slot < npos;
-                    x[nt][e] = ok ? x[nt][e] * A.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, x[nt][e]);
+                for (int i = 0; i < 4; ++i) {
+                    const bool ok = head_ok[e] && (4 * gq + i) < npos;
+                    v[i] = ok ? v[i] * A.scale_log2 : -INFINITY;
+                    mx = fmaxf(mx, v[i]);
                 }
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m_run, mx);
-            const float alpha = exp2f(m_run - m_new);
-            m_run = m_new;
-            float psum = 0.f;
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float m_new = fmaxf(m_run[e], mx);
+                alpha[e] = ex2(m_run[e] - m_new);
+                m_run[e] = m_new;
+                float psum = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    x[nt][e] = exp2f(x[nt][e] - m_new);
-                    psum += x[nt][e];
+                for (int i = 0; i < 4; ++i) {
+                    v[i] = ex2(v[i] - m_new);
+                    psum += v[i];
                 }
-            l_run = l_run * alpha + psum;
-
-            // weights that multiply each position's dequantised row
-            float wgt[4][2];
-            if (MODE == SUFFIX) {
-                float pin[4][2];
+                l_run[e] = l_run[e] * alpha[e] + psum;
+                // weights that multiply each position's dequantised row
+                float wv[4];
+                if (MODE == SUFFIX) {
+                    float pin[4] = {v[0], v[1], v[2], v[3]};
+                    const float tot = col_scan32(pin, lane);
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt) { pin[nt][0] = x[nt][0]; pin[nt][1] = x[nt][1]; }
-                const float tot = quad_scan32(pin, tq);
+                    for (int i = 0; i < 4; ++i) wv[i] = tot - pin[i] + v[i];
+                } else if (MODE == PREFIX) {
+                    e_carry[e] *= alpha[e];
+                    float pin[4] = {v[0], v[1], v[2], v[3]};
+                    const float tot = col_scan32(pin, lane);
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
+                    for (int i = 0; i < 4; ++i) wv[i] = -(e_carry[e] + pin[i] - v[i]);
+                    e_carry[e] += tot;
+                } else {
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) wgt[nt][e] = tot - pin[nt][e] + x[nt][e];
-            } else if (MODE == PREFIX) {
-                e_carry *= alpha;
-                float pin[4][2];
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) { pin[nt][0] = x[nt][0]; pin[nt][1] = x[nt][1]; }
-                const float tot = quad_scan32(pin, tq);
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) wgt[nt][e] = -(e_carry + pin[nt][e] - x[nt][e]);
-                e_carry += tot;
-            } else {
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) { wgt[nt][0] = x[nt][0]; wgt[nt][1] = x[nt][1]; }
+                    for (int i = 0; i < 4; ++i) wv[i] = v[i];
+                }
+                x[0][0][e] = wv[0]; x[0][1][e] = wv[1]; x[1][0][e] = wv[2]; x[1][1][e] = wv[3];
             }
 
-            // rescale the output accumulators (heads 2t, 2t+1 in the V layout),
-            // only when some head's running max moved
-            if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-                const float al0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
-                const float al1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
+            // rescale the output accumulators (heads 2tq, 2tq+1), only when a
+            // running max moved
+            if (__any_sync(0xffffffffu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
-                    o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
+                    o[mt][0] *= alpha[0]; o[mt][1] *= alpha[1];
+                    o[mt][2] *= alpha[0]; o[mt][3] *= alpha[1];
                 }
             }
 
@@ -612,112 +657,94 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
                 }
             }
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-                const int sA = 16 * kk + 2 * tq;
-                // V scales of the four positions this thread weights
-                uint2 dv[4] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u),
-                               make_uint2(0u, 0u)};
-                if (FMT != DKV_FMT_FP16) {
-                    const int ps[4] = {sA, sA + 1, sA + 8, sA + 9};
+            for (int t = 0; t < 2; ++t) {
+                // B fragments (k = positions, n = head g) of block j: transpose of
+                // the (position, head-pair) layout of W_j = weight * dV_j
+                auto make_b = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2]) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        dv[i] = *reinterpret_cast<const uint2 *>(st + sm.sc0 + ps[i] * SC_BYTES + 8);
-                        if (ps[i] >= npos) dv[i] = make_uint2(0u, 0u);  // stale slot: no weight
-                    }
-                    if (FMT == DKV_FMT_DELTA && first_seg && kk == 0 && tq == 0)
-                        dv[0] = (MODE == SUFFIX) ? make_uint2(0x3C003C00u, 0x3C003C00u)
-                                                 : make_uint2(0u, 0u);  // keyframe row
-                }
-                // B' fragments: rows = positions 16kk + {2t,2t+1} | {2t+8, 2t+9}, col = head g.
-                // For the delta format a weight multiplies a whole dequantised row
-                // (the keyframe row, or a large delta) and its rounding is shared by
-                // every channel, so it is carried as an fp16 hi + lo pair (about
-                // 22 significant bits); the comparators weight one token per row and
-                // use a single fp16 weight, as flash-decoding does.
-                const float w0 = wgt[2 * kk][0], w1 = wgt[2 * kk][1];
-                const float w2 = wgt[2 * kk + 1][0], w3 = wgt[2 * kk + 1][1];
-                auto make_bp = [&](int j, uint32_t (&hi)[2], uint32_t (&lo)[2]) {
-                    auto d = [&](int i) {
-                        const uint32_t u = (j >> 1) ? dv[i].y : dv[i].x;
-                        return (j & 1) ? h_hi(u) : h_lo(u);
-                    };
-                    const float v0 = w0 * d(0), v1 = w1 * d(1), v2 = w2 * d(2), v3 = w3 * d(3);
-                    hi[0] = pack_h2(v0, v1);
-                    hi[1] = pack_h2(v2, v3);
-                    if (FMT == DKV_FMT_DELTA) {
-                        lo[0] = pack_h2(v0 - h_lo(hi[0]), v1 - h_hi(hi[0]));
-                        lo[1] = pack_h2(v2 - h_lo(hi[1]), v3 - h_hi(hi[1]));
+                    for (int r = 0; r < 2; ++r) {
+                        float d = 1.f;
+                        if (FMT != DKV_FMT_FP16) {
+                            const uint32_t u = dvw[t][r][j >> 1];
+                            d = (j & 1) ? h_hi(u) : h_lo(u);
+                        }
+                        const float v0 = x[t][r][0] * d, v1 = x[t][r][1] * d;
+                        const uint32_t hi = pack_h2(v0, v1);
+                        b[r] = movm_t(hi);
+                        if (FMT == DKV_FMT_DELTA && MODE == PREFIX)
+                            bl[r] = movm_t(pack_h2(v0 - h_lo(hi), v1 - h_hi(hi)));
                     }
                 };
-                uint32_t bp[2] = {0u, 0u}, bl[2] = {0u, 0u};
+                uint32_t bp[2], bl[2] = {0u, 0u};
+                // SUFFIX: lo part of the keyframe row's weight (position 0, scale 1)
+                uint32_t bk = 0u;
+                if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0 && first_seg) {
+                    const float r0 = x[0][0][0] - __half2float(__float2half_rn(x[0][0][0]));
+                    const float r1 = x[0][0][1] - __half2float(__float2half_rn(x[0][0][1]));
+                    bk = movm_t(kfrow ? pack_h2(r0, r1) : 0u);
+                }
                 if (FMT == DKV_FMT_FP16) {
-                    bp[0] = pack_h2(w0, w1);
-                    bp[1] = pack_h2(w2, w3);
-                    const uint8_t *vb = st + 8192 + 32 * gq;
-                    const uint4 A0 = *reinterpret_cast<const uint4 *>(vb + sA * 256);
-                    const uint4 A1 = *reinterpret_cast<const uint4 *>(vb + sA * 256 + 16);
-                    const uint4 B0 = *reinterpret_cast<const uint4 *>(vb + (sA + 1) * 256);
-                    const uint4 B1 = *reinterpret_cast<const uint4 *>(vb + (sA + 1) * 256 + 16);
-                    const uint4 C0 = *reinterpret_cast<const uint4 *>(vb + (sA + 8) * 256);
-                    const uint4 C1 = *reinterpret_cast<const uint4 *>(vb + (sA + 8) * 256 + 16);
-                    const uint4 D0 = *reinterpret_cast<const uint4 *>(vb + (sA + 9) * 256);
-                    const uint4 D1 = *reinterpret_cast<const uint4 *>(vb + (sA + 9) * 256 + 16);
-                    const uint32_t wa[8] = {A0.x, A0.y, A0.z, A0.w, A1.x, A1.y, A1.z, A1.w};
-                    const uint32_t wb[8] = {B0.x, B0.y, B0.z, B0.w, B1.x, B1.y, B1.z, B1.w};
-                    const uint32_t wc[8] = {C0.x, C0.y, C0.z, C0.w, C1.x, C1.y, C1.z, C1.w};
-                    const uint32_t wd[8] = {D0.x, D0.y, D0.z, D0.w, D1.x, D1.y, D1.z, D1.w};
+                    make_b(0, bp, bl);
+                    // V values of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
+                    const uint8_t *vb = st + 8192 + (8 * tq + 2 * t) * 256 + 32 * gq;
+                    uint32_t wv[4][8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int dp = (i & 1) + 4 * (i >> 1);
+                        const uint4 lo4 = *reinterpret_cast<const uint4 *>(vb + dp * 256);
+                        const uint4 hi4 = *reinterpret_cast<const uint4 *>(vb + dp * 256 + 16);
+                        wv[i][0] = lo4.x; wv[i][1] = lo4.y; wv[i][2] = lo4.z; wv[i][3] = lo4.w;
+                        wv[i][4] = hi4.x; wv[i][5] = hi4.y; wv[i][6] = hi4.z; wv[i][7] = hi4.w;
+                    }
 #pragma unroll
                     for (int mt = 0; mt < 8; ++mt) {
-                        const uint32_t a0 = prmt(wa[mt], wb[mt], 0x5410u);
-                        const uint32_t a1 = prmt(wa[mt], wb[mt], 0x7632u);
-                        const uint32_t a2 = prmt(wc[mt], wd[mt], 0x5410u);
-                        const uint32_t a3 = prmt(wc[mt], wd[mt], 0x7632u);
+                        const uint32_t a0 = prmt(wv[0][mt], wv[2][mt], 0x5410u);
+                        const uint32_t a1 = prmt(wv[0][mt], wv[2][mt], 0x7632u);
+                        const uint32_t a2 = prmt(wv[1][mt], wv[3][mt], 0x5410u);
+                        const uint32_t a3 = prmt(wv[1][mt], wv[3][mt], 0x7632u);
                         mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
                     }
                 } else {
-                    const uint8_t *vb = st + sm.vn0 + 8 * gq;
-                    const uint2 wA = *reinterpret_cast<const uint2 *>(vb + sA * NIB_BYTES);
-                    const uint2 wB = *reinterpret_cast<const uint2 *>(vb + (sA + 1) * NIB_BYTES);
-                    const uint2 wC = *reinterpret_cast<const uint2 *>(vb + (sA + 8) * NIB_BYTES);
-                    const uint2 wD = *reinterpret_cast<const uint2 *>(vb + (sA + 9) * NIB_BYTES);
-                    const bool kfrow = (FMT == DKV_FMT_DELTA) && (MODE == SUFFIX) && first_seg &&
-                                       kk == 0 && tq == 0;
-                    const uint32_t sel0 = kfrow ? 0x3254u : 0x3210u;
-                    const uint32_t sel1 = kfrow ? 0x3276u : 0x3210u;
+                    // V nibbles of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
+                    const uint8_t *vb = st + sm.vn0 + (8 * tq + 2 * t) * NIB_BYTES + 8 * gq;
+                    const uint2 wP0 = *reinterpret_cast<const uint2 *>(vb);
+                    const uint2 wP1 = *reinterpret_cast<const uint2 *>(vb + NIB_BYTES);
+                    const uint2 wP2 = *reinterpret_cast<const uint2 *>(vb + 4 * NIB_BYTES);
+                    const uint2 wP3 = *reinterpret_cast<const uint2 *>(vb + 5 * NIB_BYTES);
+                    const bool kf_a = (FMT == DKV_FMT_DELTA) && (MODE == SUFFIX) && first_seg &&
+                                      t == 0 && tq == 0;
+                    const uint32_t sel0 = kf_a ? 0x3254u : 0x3210u;
+                    const uint32_t sel1 = kf_a ? 0x3276u : 0x3210u;
 #pragma unroll
                     for (int mt = 0; mt < 8; ++mt) {
                         const int i = mt & 3;
                         const uint32_t sel = (uint32_t)(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
-                        const uint32_t m01 = prmt(mt < 4 ? wA.x : wA.y, mt < 4 ? wB.x : wB.y, sel);
-                        const uint32_t m23 = prmt(mt < 4 ? wC.x : wC.y, mt < 4 ? wD.x : wD.y, sel);
+                        // k pairs: (pos 8tq+2t, +4) | (8tq+2t+1, +5)
+                        const uint32_t m01 = prmt(mt < 4 ? wP0.x : wP0.y, mt < 4 ? wP2.x : wP2.y, sel);
+                        const uint32_t m23 = prmt(mt < 4 ? wP1.x : wP1.y, mt < 4 ? wP3.x : wP3.y, sel);
                         uint32_t a0, a1, a2, a3;
-                        {
-                            const uint32_t MAGIC = 0x64006400u;
-                            const __half2 SUB_LO = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
-                            const __half2 MUL_HI = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
-                            const __half2 SUB_HI = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
-                            a0 = h2_as_u32(__hsub2(u32_as_h2(lop_and_or(m01, 0x000F000Fu, MAGIC)), SUB_LO));
-                            a1 = h2_as_u32(__hfma2(u32_as_h2(lop_and_or(m01, 0x00F000F0u, MAGIC)), MUL_HI, SUB_HI));
-                            a2 = h2_as_u32(__hsub2(u32_as_h2(lop_and_or(m23, 0x000F000Fu, MAGIC)), SUB_LO));
-                            a3 = h2_as_u32(__hfma2(u32_as_h2(lop_and_or(m23, 0x00F000F0u, MAGIC)), MUL_HI, SUB_HI));
-                        }
-                        if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && kk == 0) {
+                        dq_pair(m01, magic, a0, a1);
+                        dq_pair(m23, magic, a2, a3);
+                        if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0) {
                             a0 = prmt(a0, vkf[mt], sel0);
                             a1 = prmt(a1, vkf[mt], sel1);
                         }
                         const int j = mt >> 1;
-                        if ((mt & 1) == 0) make_bp(j, bp, bl);
+                        if ((mt & 1) == 0) make_b(j, bp, bl);
                         mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
-                        if (FMT == DKV_FMT_DELTA) mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
+                        if (MODE == PREFIX) mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
+                        if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0)
+                            mma16816(o[mt], a0, a1, a2, a3, bk, 0u);
                         if (MODE == PREFIX) {
                             // R += sum_s (code-8) * d_s : B = the scales alone
-                            auto d = [&](int i2) {
-                                const uint32_t u = (j >> 1) ? dv[i2].y : dv[i2].x;
-                                return (j & 1) ? h_hi(u) : h_lo(u);
-                            };
-                            const uint32_t r0 = pack_h2(d(0), d(1));
-                            const uint32_t r1 = pack_h2(d(2), d(3));
-                            mma16816(racc[mt], a0, a1, a2, a3, r0, r1);
+                            uint32_t r2[2];
+#pragma unroll
+                            for (int r = 0; r < 2; ++r) {
+                                const uint32_t u = dvw[t][r][j >> 1];
+                                const float d = (j & 1) ? h_hi(u) : h_lo(u);
+                                r2[r] = movm_t(pack_h2(d, d));
+                            }
+                            mma16816(racc[mt], a0, a1, a2, a3, r2[0], r2[1]);
                         }
                     }
                 }
@@ -725,18 +752,16 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
 
             // PREFIX: close the group  o += W_g (v_f + R_g)
             if (MODE == PREFIX && last_seg) {
-                const float w0 = __shfl_sync(0xffffffffu, e_carry, (2 * tq) * 4);
-                const float w1 = __shfl_sync(0xffffffffu, e_carry, (2 * tq + 1) * 4);
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
                     const float v_lo = h_lo(vkf_keep[mt]) + racc[mt][0];   // channel 16mt+g
                     const float v_hi = h_hi(vkf_keep[mt]) + racc[mt][2];   // channel 16mt+g+8
-                    o[mt][0] += w0 * v_lo; o[mt][1] += w1 * v_lo;
-                    o[mt][2] += w0 * v_hi; o[mt][3] += w1 * v_hi;
+                    o[mt][0] += e_carry[0] * v_lo; o[mt][1] += e_carry[1] * v_lo;
+                    o[mt][2] += e_carry[0] * v_hi; o[mt][3] += e_carry[1] * v_hi;
                     racc[mt][0] = racc[mt][1] = racc[mt][2] = racc[mt][3] = 0.f;
                 }
-                e_carry = 0.f;
-                dot_carry = 0.f;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) { e_carry[e] = 0.f; dot_carry[e] = 0.f; }
             }
         }
 
@@ -749,7 +774,7 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
                 mymeta[stage_i] = make_meta<MODE>(cv, ic);
                 issue_stage<FMT, MODE>(cv, ic, A.NHG, mystages + stage_i * STAGE, mybar + stage_i);
             }
-            cursor_next<MODE>(ic, cv, nvs);
+            cursor_next<MODE>(ic, cv, nvs, A.NHG);
             ++issued;
         }
         stage_i = (stage_i + 1 == NS) ? 0 : stage_i + 1;

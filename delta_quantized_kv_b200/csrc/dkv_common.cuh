@@ -153,28 +153,57 @@ __device__ inline __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__hal
 // D = A(16x16 f16, row) * B(16x8 f16, col) + C, fp32 accumulate.
 __device__ inline void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                 uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The fp16 bit pattern of 1024.0 in both halves, as a register value the
+// compiler cannot fold: OR-ing a nibble into it needs the mask as the one
+// immediate operand of a single LOP3 and this value in a register.
+__device__ inline uint32_t magic_1024x2() {
+    uint32_t r;
+    asm volatile("mov.b32 %0, 0x64006400;\n" : "=r"(r));
+    return r;
+}
+// (a & MASK) | c in one LOP3 (LUT 0xEA).
+template <uint32_t MASK>
+__device__ inline uint32_t and_or(uint32_t a, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(d) : "r"(a), "n"(MASK), "r"(c));
+    return d;
+}
+// fp16x2 helpers on raw 32-bit registers
+__device__ inline uint32_t hsub2_1032(uint32_t a) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(0x64086408u));
+    return d;
+}
+__device__ inline uint32_t hfma2_div16_sub72(uint32_t a) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(0x2C002C00u), "r"(0xD480D480u));
+    return d;
+}
+
 // Dequantise the 4 nibble pairs of one 32-bit word (pairs (bits 0-3,16-19),
-// (4-7,20-23), (8-11,24-27), (12-15,28-31)) to exact fp16x2 values code - 8.
-__device__ inline void dq_word(uint32_t w, uint32_t &p0, uint32_t &p1, uint32_t &p2,
-                               uint32_t &p3) {
-    const uint32_t MAGIC = 0x64006400u;  // fp16 1024.0 in both halves
-    const __half2 SUB_LO = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
-    const __half2 MUL_HI = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
-    const __half2 SUB_HI = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
-    uint32_t w8 = w >> 8;
-    // (1024 + n) - 1032 = n - 8, exact
-    p0 = h2_as_u32(__hsub2(u32_as_h2(lop_and_or(w, 0x000F000Fu, MAGIC)), SUB_LO));
-    p2 = h2_as_u32(__hsub2(u32_as_h2(lop_and_or(w8, 0x000F000Fu, MAGIC)), SUB_LO));
-    // (1024 + 16 n) / 16 - 72 = n - 8, exact
-    p1 = h2_as_u32(__hfma2(u32_as_h2(lop_and_or(w, 0x00F000F0u, MAGIC)), MUL_HI, SUB_HI));
-    p3 = h2_as_u32(__hfma2(u32_as_h2(lop_and_or(w8, 0x00F000F0u, MAGIC)), MUL_HI, SUB_HI));
+// (4-7,20-23), (8-11,24-27), (12-15,28-31)) to exact fp16x2 values code - 8:
+// (1024 + n) - 1032 for the low nibbles, (1024 + 16 n) / 16 - 72 for the high.
+__device__ inline void dq_word(uint32_t w, uint32_t magic, uint32_t &p0, uint32_t &p1,
+                               uint32_t &p2, uint32_t &p3) {
+    const uint32_t w8 = w >> 8;
+    p0 = hsub2_1032(and_or<0x000F000Fu>(w, magic));
+    p1 = hfma2_div16_sub72(and_or<0x00F000F0u>(w, magic));
+    p2 = hsub2_1032(and_or<0x000F000Fu>(w8, magic));
+    p3 = hfma2_div16_sub72(and_or<0x00F000F0u>(w8, magic));
+}
+
+// The low-nibble pair (bits 0-3, 16-19) and the high-nibble pair (bits 4-7,
+// 20-23) of one 32-bit word as exact fp16x2 values code - 8.
+__device__ inline void dq_pair(uint32_t w, uint32_t magic, uint32_t &lo, uint32_t &hi) {
+    lo = hsub2_1032(and_or<0x000F000Fu>(w, magic));
+    hi = hfma2_div16_sub72(and_or<0x00F000F0u>(w, magic));
 }
 
 }  // namespace dkv
