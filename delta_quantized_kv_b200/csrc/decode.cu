@@ -16,13 +16,13 @@
 // (position f carries v_f with S_hf = the group's total weight) is a sum of
 // dequantised delta rows weighted by suffix sums of the softmax weights.  Both
 // per-position products are dense tiles for the tensor cores:
-//   K side  D[h][p] = sum_c q[h][c] * code[p][c]  per 32-channel block, m16n8k16
-//           with heads as M (8 of 16 rows used) and positions as N;
+//   K side  D[p][h] = sum_c code[p][c] * q[h][c]  per 32-channel block, m16n8k16
+//           with positions as M, channels as K and heads as N (q stays in
+//           registers as the B operand);
 //   V side  O[c][h] += sum_p code[p][c] * (S[h][p] * d[p][blk(c)]), m16n8k16
 //           with channels as M, positions as K and heads as N.
-// The K-side accumulator layout of a thread (head g, positions 2t, 2t+1) is
-// exactly the V-side B-fragment layout, so the softmax weights flow from one
-// MMA to the other without shuffles.
+// An 8x8 movmatrix transpose turns the K-side accumulator layout (a thread
+// owns positions x heads 2t, 2t+1) into the V-side B fragments.
 //
 // Groups longer than one 32-position stage (kf > 32) use the equivalent
 // forward form  sum_p w_p v^_p = W_g (v_f + R_g) - sum_s delta^_s E_s  with
@@ -47,23 +47,36 @@ enum Mode { SUFFIX = 0, PREFIX = 1, PLAIN = 2 };
 
 constexpr int WARPS = 4;                     // warps per CTA (independent pipelines)
 
-#ifndef DKV_NIB_MINB
-#define DKV_NIB_MINB 4                       // resident CTAs per SM (nibble formats)
+// Nibble formats with kf <= 32: units per stage, stages per warp, CTAs per SM.
+// Two groups per stage and one stage per warp (a warp's next stage is copied
+// while the other warps of the SM compute) measured fastest on B200: the
+// shared memory this frees buys a third CTA per SM.
+#ifndef DKV_NIB_NU
+#define DKV_NIB_NU 2
 #endif
 #ifndef DKV_NIB_NS
-#define DKV_NIB_NS 2                         // pipeline stages per warp (nibble formats)
+#define DKV_NIB_NS 1
+#endif
+#ifndef DKV_NIB_MINB
+#define DKV_NIB_MINB 3
 #endif
 
-template <int FMT> struct FmtCfg;
-template <> struct FmtCfg<DKV_FMT_DELTA> { static constexpr int STAGE = 5120, NS = DKV_NIB_NS, MINB = DKV_NIB_MINB; };
-template <> struct FmtCfg<DKV_FMT_Q4_0>  { static constexpr int STAGE = 5120, NS = DKV_NIB_NS, MINB = DKV_NIB_MINB; };
-template <> struct FmtCfg<DKV_FMT_FP16>  { static constexpr int STAGE = 16384, NS = 2, MINB = 1; };
+// Per (format, mode): units per stage, stage bytes, stages per warp, CTAs/SM.
+// A unit is one keyframe group (delta, kf <= 32), one 32-position segment of
+// a group (delta, kf > 32), or one 32-position chunk (Q4_0, fp16).
+template <int FMT, int MODE> struct KCfg {
+    static constexpr bool NIB = FMT != DKV_FMT_FP16 && MODE != PREFIX;
+    static constexpr int NU = NIB ? DKV_NIB_NU : 1;
+    static constexpr int STAGE = FMT == DKV_FMT_FP16 ? 16384 : NU * 5120;
+    static constexpr int NS = NIB ? DKV_NIB_NS : 2;
+    static constexpr int MINB = FMT == DKV_FMT_FP16 ? 1 : (MODE == PREFIX ? 3 : DKV_NIB_MINB);
+};
 
 // Shared-memory map of the split kernel: [mbarriers WARPS*NS x 8 B]
 // [stage descriptors WARPS*NS x 16 B][stages WARPS*NS x STAGE], each region
 // aligned; the offsets follow from NS so no region can overlap another.
-template <int FMT> struct SmemMap {
-    static constexpr int NS = FmtCfg<FMT>::NS, STAGE = FmtCfg<FMT>::STAGE;
+template <int FMT, int MODE> struct SmemMap {
+    static constexpr int NS = KCfg<FMT, MODE>::NS, STAGE = KCfg<FMT, MODE>::STAGE;
     static constexpr int BAR_OFF = 0;
     static constexpr int META_OFF = ((BAR_OFF + 8 * WARPS * NS) + 15) / 16 * 16;
     static constexpr int STAGE_OFF = ((META_OFF + 16 * WARPS * NS) + 127) / 128 * 128;
@@ -71,6 +84,7 @@ template <int FMT> struct SmemMap {
     static_assert(META_OFF >= BAR_OFF + 8 * WARPS * NS, "barriers overlap descriptors");
     static_assert(STAGE_OFF >= META_OFF + 16 * WARPS * NS, "descriptors overlap stages");
     static_assert(STAGE % 128 == 0, "stages must stay 128-byte aligned");
+    static_assert(BYTES <= 227 * 1024, "shared memory per CTA");
 };
 
 struct SplitArgs {
@@ -78,7 +92,7 @@ struct SplitArgs {
     const void *Q;
     int q_dtype;
     int Hq, G, NHG;            // query heads, heads per kv head, head groups of 8
-    float scale_log2;          // softmax_scale * log2(e)
+    float scale_log2;          // softmax_scale * log2(e), > 0
     float *ws;                 // partial records
 };
 
@@ -190,25 +204,54 @@ __device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs, int 
     if (MODE == PREFIX) c.nseg = nseg_of<MODE>(cv, c.len_b, c.g);
 }
 
-// Stage layouts in shared memory (offsets from the stage start):
-//  DELTA, kf <= 32: the whole group record, one copy:
-//      [K kf 256][V kf 256][scales (kf-1)x16][K nib (kf-1)x64][V nib (kf-1)x64]
-//  DELTA, kf > 32 (one 32-position segment) and Q4_0:
-//      [K kf 256][V kf 256][scales 32x16][K nib 32x64][V nib 32x64]
-//  FP16: [K 32x256][V 32x256]
+// What the consumer needs to know about a stage, written next to the stage by
+// the issuing lane before it arms the barrier.
+struct StageMeta {
+    int b, vs;                 // batch entry, sequence within it
+    int npos;                  // valid positions: unit 0 in bits 0-7, unit 1 in bits 8-15
+    int flags;                 // bit 0: first segment of a group; bit 1: last segment
+};
+
+// Positions of the current unit of c.
+__device__ inline int unit_npos(const CacheView &cv, const Cursor &c, int g) {
+    if (cv.fmt == DKV_FMT_DELTA) {
+        const int glen = min(cv.kf, c.len_b - g * cv.kf);
+        return min(SEG, glen - c.seg * SEG);
+    }
+    return min(SEG, c.len_b - g * SEG);
+}
+
+// Stage layouts in shared memory (offsets from the stage start), unit u:
+//  DELTA, kf <= 32: NU consecutive group records copied as one run, record u
+//      at u * rec: [K kf 256][V kf 256][scales (kf-1)x16][K nib (kf-1)x64]
+//      [V nib (kf-1)x64];
+//  DELTA, kf > 32 (NU = 1, one 32-position segment):
+//      [K kf 256][V kf 256][scales 32x16][K nib 32x64][V nib 32x64];
+//  Q4_0 (NU chunks of 32 positions): [scales NU x 512][K nib NU x 2048]
+//      [V nib NU x 2048];
+//  FP16 (NU = 1): [K 32x256][V 32x256].
 // For slot s (position a + s) the scale / K nibble / V nibble rows start at
-// sc0 + 16 s, kn0 + 64 s, vn0 + 64 s.
+// sc0 + 16 s, kn0 + 64 s, vn0 + 64 s; keyframes at kf0 (K) and kf0 + 256 (V).
 struct StageMap {
-    int sc0, kn0, vn0;
+    int kf0, sc0, kn0, vn0;
 };
 template <int FMT, int MODE>
-__device__ inline StageMap stage_map(int kf) {
+__device__ inline StageMap stage_map(int kf, int64_t rec, int u) {
+    constexpr int NU = KCfg<FMT, MODE>::NU;
     StageMap m;
     if (FMT == DKV_FMT_DELTA && MODE == SUFFIX) {
-        m.sc0 = KF_BYTES - SC_BYTES;
-        m.kn0 = KF_BYTES + (kf - 1) * SC_BYTES - NIB_BYTES;
-        m.vn0 = KF_BYTES + (kf - 1) * (SC_BYTES + NIB_BYTES) - NIB_BYTES;
+        const int base = u * (int)rec;
+        m.kf0 = base;
+        m.sc0 = base + KF_BYTES - SC_BYTES;
+        m.kn0 = base + KF_BYTES + (kf - 1) * SC_BYTES - NIB_BYTES;
+        m.vn0 = base + KF_BYTES + (kf - 1) * (SC_BYTES + NIB_BYTES) - NIB_BYTES;
+    } else if (FMT == DKV_FMT_Q4_0) {
+        m.kf0 = 0;
+        m.sc0 = 512 * u;
+        m.kn0 = 512 * NU + 2048 * u;
+        m.vn0 = 2560 * NU + 2048 * u;
     } else {
+        m.kf0 = 0;
         m.sc0 = 512;
         m.kn0 = 1024;
         m.vn0 = 3072;
@@ -216,38 +259,14 @@ __device__ inline StageMap stage_map(int kf) {
     return m;
 }
 
-// What the consumer needs to know about a stage item, written next to the
-// stage by the issuing lane before it arms the barrier.
-struct StageMeta {
-    int b, vs;                 // batch entry, sequence within it
-    int npos;                  // valid positions in the stage
-    int flags;                 // bit 0: first segment of a group; bit 1: last segment
-};
-
-template <int MODE>
-__device__ inline StageMeta make_meta(const CacheView &cv, const Cursor &c) {
-    StageMeta m;
-    m.b = c.b;
-    m.vs = c.vs;
-    if (cv.fmt == DKV_FMT_DELTA) {
-        const int glen = min(cv.kf, c.len_b - c.g * cv.kf);
-        m.npos = min(SEG, glen - c.seg * SEG);
-        m.flags = (c.seg == 0 ? 1 : 0) | (c.seg == c.nseg - 1 ? 2 : 0);
-    } else {
-        m.npos = min(SEG, c.len_b - c.g * SEG);
-        m.flags = 3;
-    }
-    return m;
-}
-
-// Issue the bulk copies of one stage item (one lane).
+// Issue the bulk copies of one stage (nu units starting at c; one lane).
 template <int FMT, int MODE>
-__device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nhg,
+__device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nu, int npos_all,
                                    uint8_t *stage, uint64_t *bar) {
-    (void)nhg;
+    constexpr int NU = KCfg<FMT, MODE>::NU;
     const uint8_t *sb = c.seq;
     if (FMT == DKV_FMT_DELTA && MODE == SUFFIX) {
-        const uint32_t bytes = (uint32_t)cv.rec_bytes;
+        const uint32_t bytes = (uint32_t)(nu * cv.rec_bytes);
         mbar_arrive_expect_tx(bar, bytes);
         bulk_g2s(stage, sb + (int64_t)c.g * cv.rec_bytes, bytes, bar);
     } else if (FMT == DKV_FMT_DELTA) {
@@ -275,20 +294,44 @@ __device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nhg
         }
     } else if (FMT == DKV_FMT_Q4_0) {
         const int p0 = c.g * SEG;
-        const int npos = min(SEG, c.len_b - p0);
-        mbar_arrive_expect_tx(bar, npos * (SC_BYTES + 2 * NIB_BYTES));
-        bulk_g2s(stage + 512, sb + (int64_t)p0 * SC_BYTES, npos * SC_BYTES, bar);
-        bulk_g2s(stage + 1024, sb + (int64_t)cv.cap * SC_BYTES + (int64_t)p0 * NIB_BYTES,
-                 npos * NIB_BYTES, bar);
-        bulk_g2s(stage + 3072, sb + (int64_t)cv.cap * (SC_BYTES + NIB_BYTES) + (int64_t)p0 * NIB_BYTES,
-                 npos * NIB_BYTES, bar);
+        mbar_arrive_expect_tx(bar, npos_all * (SC_BYTES + 2 * NIB_BYTES));
+        bulk_g2s(stage, sb + (int64_t)p0 * SC_BYTES, npos_all * SC_BYTES, bar);
+        bulk_g2s(stage + 512 * NU, sb + (int64_t)cv.cap * SC_BYTES + (int64_t)p0 * NIB_BYTES,
+                 npos_all * NIB_BYTES, bar);
+        bulk_g2s(stage + 2560 * NU, sb + (int64_t)cv.cap * (SC_BYTES + NIB_BYTES) + (int64_t)p0 * NIB_BYTES,
+                 npos_all * NIB_BYTES, bar);
     } else {
         const int p0 = c.g * SEG;
-        const int npos = min(SEG, c.len_b - p0);
-        mbar_arrive_expect_tx(bar, npos * 512);
-        bulk_g2s(stage, sb + (int64_t)p0 * 256, npos * 256, bar);
-        bulk_g2s(stage + 8192, sb + (int64_t)cv.cap * 256 + (int64_t)p0 * 256, npos * 256, bar);
+        mbar_arrive_expect_tx(bar, npos_all * 512);
+        bulk_g2s(stage, sb + (int64_t)p0 * 256, npos_all * 256, bar);
+        bulk_g2s(stage + 8192, sb + (int64_t)cv.cap * 256 + (int64_t)p0 * 256, npos_all * 256, bar);
     }
+}
+
+// Decide how many units the next stage takes (the units must be consecutive
+// in one sequence), fill its descriptor and (lane 0) issue its copies; every
+// lane advances its cursor identically.
+template <int FMT, int MODE>
+__device__ inline void next_stage(const CacheView &cv, Cursor &c, int nvs, int nhg, uint8_t *stage,
+                                  uint64_t *bar, StageMeta *meta, int lane) {
+    constexpr int NU = KCfg<FMT, MODE>::NU;
+    const int np0 = unit_npos(cv, c, c.g);
+    int nu = 1, np1 = 0;
+    if (NU == 2 && c.left >= 2 && c.g + 1 < c.units_b) {
+        nu = 2;
+        np1 = unit_npos(cv, c, c.g + 1);
+    }
+    if (lane == 0) {
+        StageMeta m;
+        m.b = c.b;
+        m.vs = c.vs;
+        m.npos = np0 | (np1 << 8);
+        m.flags = MODE == PREFIX ? ((c.seg == 0 ? 1 : 0) | (c.seg == c.nseg - 1 ? 2 : 0)) : 3;
+        *meta = m;
+        issue_stage<FMT, MODE>(cv, c, nu, np0 + np1, stage, bar);
+    }
+    cursor_next<MODE>(c, cv, nvs, nhg);
+    if (nu == 2) cursor_next<MODE>(c, cv, nvs, nhg);
 }
 
 __device__ inline uint32_t pack_h2(float lo, float hi) {
@@ -334,7 +377,7 @@ __device__ inline float col_scan32(float (&v)[4], int lane) {
     return __shfl_sync(0xffffffffu, inc, 28 + (lane & 3));
 }
 
-// Per stage (up to 32 positions), per thread of lane (g, t4):
+// Per unit (up to 32 positions), per thread of lane (g, t4):
 //  K side, tile t: m16n8k16 with rows = positions (row g <-> 4g + 2t, row
 //   g+8 <-> 4g + 2t + 1), k = channels, n = heads; the accumulator holds
 //   x[t][r][e] for position 4g + 2t + r, head 2t4 + e, so each thread owns
@@ -343,20 +386,222 @@ __device__ inline float col_scan32(float (&v)[4], int lane) {
 //   (k 2t4, 2t4+1 <-> 8t4 + 2t, +4; k 2t4+8, 2t4+9 <-> 8t4 + 2t + 1, +5),
 //   n = heads; the weights reach that B layout through an 8x8 transpose
 //   (movmatrix) of the K-side accumulator layout.
+
+// K side of one unit: per-position dot products x[t][r][e] (position
+// 4g + 2t + r, head 2tq + e) and the V scales dvw[t][r] of those positions.
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(SplitArgs A) {
-    using Cfg = FmtCfg<FMT>;
-    constexpr int NS = Cfg::NS, STAGE = Cfg::STAGE;
+__device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, bool first_seg,
+                              int gq, int tq, uint32_t magic, const uint32_t (&qb)[8][2],
+                              float (&x)[2][2][2], uint32_t (&dvw)[2][2][2]) {
+    const bool kfrow = first_seg && gq == 0;   // this thread's row 0 of tile 0 is the keyframe
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int p0 = 4 * gq + 2 * t;             // positions p0, p0 + 1
+        if (FMT == DKV_FMT_FP16) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint8_t *k0 = st + p0 * 256 + 64 * tq;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const uint4 u0 = *reinterpret_cast<const uint4 *>(k0 + 16 * q4);
+                const uint4 u1 = *reinterpret_cast<const uint4 *>(k0 + 256 + 16 * q4);
+                mma16816(acc, u0.x, u1.x, u0.y, u1.y, qb[2 * q4][0], qb[2 * q4][1]);
+                mma16816(acc, u0.z, u1.z, u0.w, u1.w, qb[2 * q4 + 1][0], qb[2 * q4 + 1][1]);
+            }
+            x[t][0][0] = acc[0]; x[t][0][1] = acc[1];
+            x[t][1][0] = acc[2]; x[t][1][1] = acc[3];
+            dvw[t][0][0] = dvw[t][0][1] = dvw[t][1][0] = dvw[t][1][1] = 0u;
+        } else {
+            const uint4 w0 = *reinterpret_cast<const uint4 *>(st + sm.kn0 + p0 * NIB_BYTES + 16 * tq);
+            const uint4 w1 = *reinterpret_cast<const uint4 *>(st + sm.kn0 + (p0 + 1) * NIB_BYTES + 16 * tq);
+            uint32_t a[8][4];
+            {
+                const uint32_t ww0[4] = {w0.x, w0.y, w0.z, w0.w};
+                const uint32_t ww1[4] = {w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    dq_word(ww0[j], magic, a[2 * j][0], a[2 * j][2], a[2 * j + 1][0], a[2 * j + 1][2]);
+                    dq_word(ww1[j], magic, a[2 * j][1], a[2 * j][3], a[2 * j + 1][1], a[2 * j + 1][3]);
+                }
+            }
+            if (FMT == DKV_FMT_DELTA && t == 0 && first_seg) {
+                // position 0 is the keyframe: its fp16 values fill rows g = 0
+                const uint8_t *kp = st + sm.kf0 + 64 * tq;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(kp + 16 * q4);
+                    a[2 * q4][0] = kfrow ? v.x : a[2 * q4][0];
+                    a[2 * q4][2] = kfrow ? v.y : a[2 * q4][2];
+                    a[2 * q4 + 1][0] = kfrow ? v.z : a[2 * q4 + 1][0];
+                    a[2 * q4 + 1][2] = kfrow ? v.w : a[2 * q4 + 1][2];
+                }
+            }
+            float acc[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+                mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
+                         qb[2 * j][0], qb[2 * j][1]);
+                mma16816(acc[j], a[2 * j + 1][0], a[2 * j + 1][1], a[2 * j + 1][2],
+                         a[2 * j + 1][3], qb[2 * j + 1][0], qb[2 * j + 1][1]);
+            }
+            // scales of positions p0, p0+1: dK (blocks 0..3) then dV
+            uint4 s0 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + p0 * SC_BYTES);
+            uint4 s1 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + (p0 + 1) * SC_BYTES);
+            if (FMT == DKV_FMT_DELTA && t == 0 && kfrow) {
+                s0.x = s0.y = 0x3C003C00u;                          // keyframe: unit K weights
+                s0.z = s0.w = (MODE == SUFFIX) ? 0x3C003C00u : 0u;  // V: 1 (SUFFIX) / 0 (PREFIX)
+            }
+            // slots past the end of the unit hold stale bytes (possibly NaN
+            // patterns): zero their K and V scales so they add nothing to the
+            // prefix sums and carry no V weight
+            if (p0 >= npos) s0 = make_uint4(0u, 0u, 0u, 0u);
+            if (p0 + 1 >= npos) s1 = make_uint4(0u, 0u, 0u, 0u);
+            dvw[t][0][0] = s0.z; dvw[t][0][1] = s0.w;
+            dvw[t][1][0] = s1.z; dvw[t][1][1] = s1.w;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                x[t][0][e] = acc[0][e] * h_lo(s0.x) + acc[1][e] * h_hi(s0.x) +
+                             acc[2][e] * h_lo(s0.y) + acc[3][e] * h_hi(s0.y);
+                x[t][1][e] = acc[0][2 + e] * h_lo(s1.x) + acc[1][2 + e] * h_hi(s1.x) +
+                             acc[2][2 + e] * h_lo(s1.y) + acc[3][2 + e] * h_hi(s1.y);
+            }
+        }
+    }
+}
+
+// V side of one unit: o += sum over positions of dequantised V rows times the
+// weights w[t][r][e] (position 4g + 2t + r, head 2tq + e) and their V scales.
+template <int FMT, int MODE>
+__device__ inline void v_side(const uint8_t *st, const StageMap &sm, bool first_seg, int gq, int tq,
+                              uint32_t magic, const float (&w)[2][2][2],
+                              const uint32_t (&dvw)[2][2][2], float (&o)[8][4],
+                              float (&racc)[8][4], uint32_t (&vkf_keep)[8]) {
+    const bool kfrow = first_seg && gq == 0;
+    uint32_t vkf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (FMT == DKV_FMT_DELTA && first_seg) {
+        const uint4 v0 = *reinterpret_cast<const uint4 *>(st + sm.kf0 + 256 + 32 * gq);
+        const uint4 v1 = *reinterpret_cast<const uint4 *>(st + sm.kf0 + 256 + 32 * gq + 16);
+        vkf[0] = v0.x; vkf[1] = v0.y; vkf[2] = v0.z; vkf[3] = v0.w;
+        vkf[4] = v1.x; vkf[5] = v1.y; vkf[6] = v1.z; vkf[7] = v1.w;
+        if (MODE == PREFIX) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) vkf_keep[i] = vkf[i];
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        // B fragments (k = positions, n = head g) of block j: transpose of the
+        // (position, head-pair) layout of W_j = weight * dV_j.  A delta row's
+        // weight rounding is shared by every channel of the row: the keyframe
+        // row (the group's total weight times v_f) gets an fp16 hi + lo pair;
+        // with kf > 32 the prefix weights -E_s aggregate up to kf positions, so
+        // every row gets the pair; the comparators weight one token per row
+        // with one fp16 weight, as flash-decoding does.
+        auto make_b = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2]) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                float d = 1.f;
+                if (FMT != DKV_FMT_FP16) {
+                    const uint32_t u = dvw[t][r][j >> 1];
+                    d = (j & 1) ? h_hi(u) : h_lo(u);
+                }
+                const float v0 = w[t][r][0] * d, v1 = w[t][r][1] * d;
+                const uint32_t hi = pack_h2(v0, v1);
+                b[r] = movm_t(hi);
+                if (FMT == DKV_FMT_DELTA && MODE == PREFIX)
+                    bl[r] = movm_t(pack_h2(v0 - h_lo(hi), v1 - h_hi(hi)));
+            }
+        };
+        uint32_t bp[2], bl[2] = {0u, 0u};
+        // kf <= 32: lo part of the keyframe row's weight (position 0, scale 1)
+        uint32_t bk = 0u;
+        if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0 && first_seg) {
+            const float r0 = w[0][0][0] - __half2float(__float2half_rn(w[0][0][0]));
+            const float r1 = w[0][0][1] - __half2float(__float2half_rn(w[0][0][1]));
+            bk = movm_t(kfrow ? pack_h2(r0, r1) : 0u);
+        }
+        if (FMT == DKV_FMT_FP16) {
+            make_b(0, bp, bl);
+            // V values of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
+            const uint8_t *vb = st + 8192 + (8 * tq + 2 * t) * 256 + 32 * gq;
+            uint32_t wv[4][8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int dp = (i & 1) + 4 * (i >> 1);
+                const uint4 lo4 = *reinterpret_cast<const uint4 *>(vb + dp * 256);
+                const uint4 hi4 = *reinterpret_cast<const uint4 *>(vb + dp * 256 + 16);
+                wv[i][0] = lo4.x; wv[i][1] = lo4.y; wv[i][2] = lo4.z; wv[i][3] = lo4.w;
+                wv[i][4] = hi4.x; wv[i][5] = hi4.y; wv[i][6] = hi4.z; wv[i][7] = hi4.w;
+            }
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                const uint32_t a0 = prmt(wv[0][mt], wv[2][mt], 0x5410u);
+                const uint32_t a1 = prmt(wv[0][mt], wv[2][mt], 0x7632u);
+                const uint32_t a2 = prmt(wv[1][mt], wv[3][mt], 0x5410u);
+                const uint32_t a3 = prmt(wv[1][mt], wv[3][mt], 0x7632u);
+                mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
+            }
+        } else {
+            // V nibbles of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
+            const uint8_t *vb = st + sm.vn0 + (8 * tq + 2 * t) * NIB_BYTES + 8 * gq;
+            const uint2 wP0 = *reinterpret_cast<const uint2 *>(vb);
+            const uint2 wP1 = *reinterpret_cast<const uint2 *>(vb + NIB_BYTES);
+            const uint2 wP2 = *reinterpret_cast<const uint2 *>(vb + 4 * NIB_BYTES);
+            const uint2 wP3 = *reinterpret_cast<const uint2 *>(vb + 5 * NIB_BYTES);
+            const bool kf_a = (FMT == DKV_FMT_DELTA) && (MODE == SUFFIX) && first_seg && t == 0 &&
+                              tq == 0;
+            const uint32_t sel0 = kf_a ? 0x3254u : 0x3210u;
+            const uint32_t sel1 = kf_a ? 0x3276u : 0x3210u;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                const int i = mt & 3;
+                const uint32_t sel = (uint32_t)(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
+                // k pairs: (pos 8tq+2t, +4) | (8tq+2t+1, +5)
+                const uint32_t m01 = prmt(mt < 4 ? wP0.x : wP0.y, mt < 4 ? wP2.x : wP2.y, sel);
+                const uint32_t m23 = prmt(mt < 4 ? wP1.x : wP1.y, mt < 4 ? wP3.x : wP3.y, sel);
+                uint32_t a0, a1, a2, a3;
+                dq_pair(m01, magic, a0, a1);
+                dq_pair(m23, magic, a2, a3);
+                if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0) {
+                    a0 = prmt(a0, vkf[mt], sel0);
+                    a1 = prmt(a1, vkf[mt], sel1);
+                }
+                const int j = mt >> 1;
+                if ((mt & 1) == 0) make_b(j, bp, bl);
+                mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
+                if (MODE == PREFIX) mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
+                if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0)
+                    mma16816(o[mt], a0, a1, a2, a3, bk, 0u);
+                if (MODE == PREFIX) {
+                    // R += sum_s (code-8) * d_s : B = the scales alone
+                    uint32_t r2[2];
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const uint32_t u = dvw[t][r][j >> 1];
+                        const float d = (j & 1) ? h_hi(u) : h_lo(u);
+                        r2[r] = movm_t(pack_h2(d, d));
+                    }
+                    mma16816(racc[mt], a0, a1, a2, a3, r2[0], r2[1]);
+                }
+            }
+        }
+    }
+}
+
+template <int FMT, int MODE>
+__global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_kernel(SplitArgs A) {
+    using Cfg = KCfg<FMT, MODE>;
+    constexpr int NS = Cfg::NS, STAGE = Cfg::STAGE, NU = Cfg::NU;
+    using Map = SmemMap<FMT, MODE>;
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const CacheView &cv = A.cv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, tq = lane & 3;          // quad row / column of the fragments
     const int nvs = cv.Hkv * A.NHG;                    // sequences per batch entry
-    using Map = SmemMap<FMT>;
     uint64_t *mybar = reinterpret_cast<uint64_t *>(smem + Map::BAR_OFF) + warp * NS;
+    StageMeta *mymeta = reinterpret_cast<StageMeta *>(smem + Map::META_OFF) + warp * NS;
     uint8_t *mystages = smem + Map::STAGE_OFF + warp * NS * STAGE;
-    const StageMap sm = stage_map<FMT, MODE>(cv.kf);
     const uint32_t magic = magic_1024x2();
 
     if (lane == 0) {
@@ -386,7 +631,6 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
 
     Cursor ic;
     cursor_seek<MODE>(ic, cv, nvs, A.NHG, r0, r1 - r0);
-    StageMeta *mymeta = reinterpret_cast<StageMeta *>(smem + Map::META_OFF) + warp * NS;
 
     // prologue: fill the ring
     uint32_t phase = 0;                 // bit s = parity to wait for on stage s
@@ -394,11 +638,7 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
 #pragma unroll 1
     for (int s = 0; s < NS; ++s) {
         if (ic.valid()) {
-            if (lane == 0) {
-                mymeta[s] = make_meta<MODE>(cv, ic);
-                issue_stage<FMT, MODE>(cv, ic, A.NHG, mystages + s * STAGE, mybar + s);
-            }
-            cursor_next<MODE>(ic, cv, nvs, A.NHG);
+            next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + s * STAGE, mybar + s, mymeta + s, lane);
             ++issued;
         }
     }
@@ -498,140 +738,96 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
         }
 
         if (!dead) {
-            const int npos = meta.npos;
-            const bool first_seg = (FMT == DKV_FMT_DELTA) && (meta.flags & 1);
-            const bool last_seg = (meta.flags & 2) != 0;
-            const bool kfrow = first_seg && gq == 0;   // this thread's row 0 of tile 0 is the keyframe
+            int npos[NU];
+#pragma unroll
+            for (int u = 0; u < NU; ++u) npos[u] = (meta.npos >> (8 * u)) & 0xff;
+            // kf <= 32: every unit is a whole group, so it starts with its keyframe
+            const bool first_seg = (FMT == DKV_FMT_DELTA) && (MODE == SUFFIX || (meta.flags & 1));
+            const bool last_seg = MODE != PREFIX || (meta.flags & 2) != 0;
 
-            // ================= K side: per-position dot products ============
-            float x[2][2][2];                   // [tile][r][e]: position 16t+2g+r, head 2tq+e
-            uint32_t dvw[2][2][2];              // V scales [tile][r][blocks 01 | 23]
+            // ================= K side ======================================
+            float x[NU][2][2][2];
+            uint32_t dvw[NU][2][2][2];
+            // Both units go through the same straight-line code; a unit the stage
+            // does not hold has npos 0, so all its slots are masked and its scales
+            // zeroed (its shared-memory bytes are an older stage's, always finite).
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const int p0 = 4 * gq + 2 * t;             // positions p0, p0 + 1
-                if (FMT == DKV_FMT_FP16) {
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    const uint8_t *k0 = st + p0 * 256 + 64 * tq;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const uint4 u0 = *reinterpret_cast<const uint4 *>(k0 + 16 * q4);
-                        const uint4 u1 = *reinterpret_cast<const uint4 *>(k0 + 256 + 16 * q4);
-                        mma16816(acc, u0.x, u1.x, u0.y, u1.y, qb[2 * q4][0], qb[2 * q4][1]);
-                        mma16816(acc, u0.z, u1.z, u0.w, u1.w, qb[2 * q4 + 1][0], qb[2 * q4 + 1][1]);
-                    }
-                    x[t][0][0] = acc[0]; x[t][0][1] = acc[1];
-                    x[t][1][0] = acc[2]; x[t][1][1] = acc[3];
-                } else {
-                    const uint4 w0 = *reinterpret_cast<const uint4 *>(st + sm.kn0 + p0 * NIB_BYTES + 16 * tq);
-                    const uint4 w1 = *reinterpret_cast<const uint4 *>(st + sm.kn0 + (p0 + 1) * NIB_BYTES + 16 * tq);
-                    uint32_t a[8][4];
-                    {
-                        const uint32_t ww0[4] = {w0.x, w0.y, w0.z, w0.w};
-                        const uint32_t ww1[4] = {w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            dq_word(ww0[j], magic, a[2 * j][0], a[2 * j][2], a[2 * j + 1][0], a[2 * j + 1][2]);
-                            dq_word(ww1[j], magic, a[2 * j][1], a[2 * j][3], a[2 * j + 1][1], a[2 * j + 1][3]);
-                        }
-                    }
-                    if (t == 0 && first_seg) {
-                        // position 0 is the keyframe: its fp16 values fill rows g = 0
-                        const uint8_t *kp = st + 64 * tq;
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const uint4 v = *reinterpret_cast<const uint4 *>(kp + 16 * q4);
-                            a[2 * q4][0] = kfrow ? v.x : a[2 * q4][0];
-                            a[2 * q4][2] = kfrow ? v.y : a[2 * q4][2];
-                            a[2 * q4 + 1][0] = kfrow ? v.z : a[2 * q4 + 1][0];
-                            a[2 * q4 + 1][2] = kfrow ? v.w : a[2 * q4 + 1][2];
-                        }
-                    }
-                    float acc[4][4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-                        mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
-                                 qb[2 * j][0], qb[2 * j][1]);
-                        mma16816(acc[j], a[2 * j + 1][0], a[2 * j + 1][1], a[2 * j + 1][2],
-                                 a[2 * j + 1][3], qb[2 * j + 1][0], qb[2 * j + 1][1]);
-                    }
-                    // scales of positions p0, p0+1: dK (blocks 0..3) then dV
-                    uint4 s0 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + p0 * SC_BYTES);
-                    uint4 s1 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + (p0 + 1) * SC_BYTES);
-                    if (t == 0 && kfrow) {
-                        s0.x = s0.y = 0x3C003C00u;                          // keyframe: unit K weights
-                        s0.z = s0.w = (MODE == SUFFIX) ? 0x3C003C00u : 0u;  // V: 1 (SUFFIX) / 0 (PREFIX)
-                    }
-                    // slots past the end of the unit hold stale bytes (possibly NaN
-                    // patterns): zero their K and V scales so they add nothing to the
-                    // prefix sums and carry no V weight
-                    if (p0 >= npos) s0 = make_uint4(0u, 0u, 0u, 0u);
-                    if (p0 + 1 >= npos) s1 = make_uint4(0u, 0u, 0u, 0u);
-                    dvw[t][0][0] = s0.z; dvw[t][0][1] = s0.w;
-                    dvw[t][1][0] = s1.z; dvw[t][1][1] = s1.w;
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        x[t][0][e] = acc[0][e] * h_lo(s0.x) + acc[1][e] * h_hi(s0.x) +
-                                     acc[2][e] * h_lo(s0.y) + acc[3][e] * h_hi(s0.y);
-                        x[t][1][e] = acc[0][2 + e] * h_lo(s1.x) + acc[1][2 + e] * h_hi(s1.x) +
-                                     acc[2][2 + e] * h_lo(s1.y) + acc[3][2 + e] * h_hi(s1.y);
-                    }
-                }
+            for (int u = 0; u < NU; ++u) {
+                const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
+                k_side<FMT, MODE>(st, sm, npos[u], first_seg, gq, tq, magic, qb, x[u], dvw[u]);
             }
 
             // ================= scores, online softmax =======================
+            // valid slots of this thread: positions 4g + i with i < lim[u]
+            int lim[NU];
+#pragma unroll
+            for (int u = 0; u < NU; ++u) lim[u] = npos[u] - 4 * gq;
             float alpha[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                // v[i]: position 4g + i  (i = 2t + r)
-                float v[4] = {x[0][0][e], x[0][1][e], x[1][0][e], x[1][1][e]};
-                if (MODE != PLAIN) {
-                    const float tot = col_scan32(v, lane);
-                    if (MODE == PREFIX) {
+                // v[u][i]: position 4g + i of unit u  (i = 2t + r)
+                float v[NU][4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) v[i] += dot_carry[e];
-                        dot_carry[e] += tot;
+                for (int u = 0; u < NU; ++u) {
+                    v[u][0] = x[u][0][0][e]; v[u][1] = x[u][0][1][e];
+                    v[u][2] = x[u][1][0][e]; v[u][3] = x[u][1][1][e];
+                    if (MODE != PLAIN) {
+                        const float tot = col_scan32(v[u], lane);
+                        if (MODE == PREFIX) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) v[u][i] += dot_carry[e];
+                            dot_carry[e] += tot;
+                        }
                     }
                 }
                 float mx = -INFINITY;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const bool ok = head_ok[e] && (4 * gq + i) < npos;
-                    v[i] = ok ? v[i] * A.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, v[i]);
-                }
+                for (int u = 0; u < NU; ++u)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        v[u][i] = (head_ok[e] && i < lim[u]) ? v[u][i] : -INFINITY;
+                        mx = fmaxf(mx, v[u][i]);
+                    }
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                const float m_new = fmaxf(m_run[e], mx);
+                // scores in log2 units: x * scale_log2 (scale_log2 > 0, so the max
+                // of the raw dots scales to the max of the scores)
+                const float m_new = fmaxf(m_run[e], mx * A.scale_log2);
                 alpha[e] = ex2(m_run[e] - m_new);
                 m_run[e] = m_new;
                 float psum = 0.f;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    v[i] = ex2(v[i] - m_new);
-                    psum += v[i];
-                }
+                for (int u = 0; u < NU; ++u)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        v[u][i] = ex2(fmaf(v[u][i], A.scale_log2, -m_new));
+                        psum += v[u][i];
+                    }
                 l_run[e] = l_run[e] * alpha[e] + psum;
                 // weights that multiply each position's dequantised row
-                float wv[4];
-                if (MODE == SUFFIX) {
-                    float pin[4] = {v[0], v[1], v[2], v[3]};
-                    const float tot = col_scan32(pin, lane);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) wv[i] = tot - pin[i] + v[i];
-                } else if (MODE == PREFIX) {
-                    e_carry[e] *= alpha[e];
-                    float pin[4] = {v[0], v[1], v[2], v[3]};
-                    const float tot = col_scan32(pin, lane);
+                for (int u = 0; u < NU; ++u) {
+                    float wv[4];
+                    if (MODE == SUFFIX) {
+                        float pin[4] = {v[u][0], v[u][1], v[u][2], v[u][3]};
+                        const float tot = col_scan32(pin, lane);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) wv[i] = -(e_carry[e] + pin[i] - v[i]);
-                    e_carry[e] += tot;
-                } else {
+                        for (int i = 0; i < 4; ++i) wv[i] = tot - pin[i] + v[u][i];
+                    } else if (MODE == PREFIX) {
+                        e_carry[e] *= alpha[e];
+                        float pin[4] = {v[u][0], v[u][1], v[u][2], v[u][3]};
+                        const float tot = col_scan32(pin, lane);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) wv[i] = v[i];
+                        for (int i = 0; i < 4; ++i) wv[i] = -(e_carry[e] + pin[i] - v[u][i]);
+                        e_carry[e] += tot;
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) wv[i] = v[u][i];
+                    }
+                    x[u][0][0][e] = wv[0]; x[u][0][1][e] = wv[1];
+                    x[u][1][0][e] = wv[2]; x[u][1][1][e] = wv[3];
                 }
-                x[0][0][e] = wv[0]; x[0][1][e] = wv[1]; x[1][0][e] = wv[2]; x[1][1][e] = wv[3];
             }
 
             // rescale the output accumulators (heads 2tq, 2tq+1), only when a
@@ -645,109 +841,11 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
             }
 
             // ================= V side ======================================
-            uint32_t vkf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-            if (FMT == DKV_FMT_DELTA && first_seg) {
-                const uint4 v0 = *reinterpret_cast<const uint4 *>(st + 256 + 32 * gq);
-                const uint4 v1 = *reinterpret_cast<const uint4 *>(st + 256 + 32 * gq + 16);
-                vkf[0] = v0.x; vkf[1] = v0.y; vkf[2] = v0.z; vkf[3] = v0.w;
-                vkf[4] = v1.x; vkf[5] = v1.y; vkf[6] = v1.z; vkf[7] = v1.w;
-                if (MODE == PREFIX) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) vkf_keep[i] = vkf[i];
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                // B fragments (k = positions, n = head g) of block j: transpose of
-                // the (position, head-pair) layout of W_j = weight * dV_j
-                auto make_b = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2]) {
-#pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        float d = 1.f;
-                        if (FMT != DKV_FMT_FP16) {
-                            const uint32_t u = dvw[t][r][j >> 1];
-                            d = (j & 1) ? h_hi(u) : h_lo(u);
-                        }
-                        const float v0 = x[t][r][0] * d, v1 = x[t][r][1] * d;
-                        const uint32_t hi = pack_h2(v0, v1);
-                        b[r] = movm_t(hi);
-                        if (FMT == DKV_FMT_DELTA && MODE == PREFIX)
-                            bl[r] = movm_t(pack_h2(v0 - h_lo(hi), v1 - h_hi(hi)));
-                    }
-                };
-                uint32_t bp[2], bl[2] = {0u, 0u};
-                // SUFFIX: lo part of the keyframe row's weight (position 0, scale 1)
-                uint32_t bk = 0u;
-                if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0 && first_seg) {
-                    const float r0 = x[0][0][0] - __half2float(__float2half_rn(x[0][0][0]));
-                    const float r1 = x[0][0][1] - __half2float(__float2half_rn(x[0][0][1]));
-                    bk = movm_t(kfrow ? pack_h2(r0, r1) : 0u);
-                }
-                if (FMT == DKV_FMT_FP16) {
-                    make_b(0, bp, bl);
-                    // V values of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
-                    const uint8_t *vb = st + 8192 + (8 * tq + 2 * t) * 256 + 32 * gq;
-                    uint32_t wv[4][8];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int dp = (i & 1) + 4 * (i >> 1);
-                        const uint4 lo4 = *reinterpret_cast<const uint4 *>(vb + dp * 256);
-                        const uint4 hi4 = *reinterpret_cast<const uint4 *>(vb + dp * 256 + 16);
-                        wv[i][0] = lo4.x; wv[i][1] = lo4.y; wv[i][2] = lo4.z; wv[i][3] = lo4.w;
-                        wv[i][4] = hi4.x; wv[i][5] = hi4.y; wv[i][6] = hi4.z; wv[i][7] = hi4.w;
-                    }
-#pragma unroll
-                    for (int mt = 0; mt < 8; ++mt) {
-                        const uint32_t a0 = prmt(wv[0][mt], wv[2][mt], 0x5410u);
-                        const uint32_t a1 = prmt(wv[0][mt], wv[2][mt], 0x7632u);
-                        const uint32_t a2 = prmt(wv[1][mt], wv[3][mt], 0x5410u);
-                        const uint32_t a3 = prmt(wv[1][mt], wv[3][mt], 0x7632u);
-                        mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
-                    }
-                } else {
-                    // V nibbles of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
-                    const uint8_t *vb = st + sm.vn0 + (8 * tq + 2 * t) * NIB_BYTES + 8 * gq;
-                    const uint2 wP0 = *reinterpret_cast<const uint2 *>(vb);
-                    const uint2 wP1 = *reinterpret_cast<const uint2 *>(vb + NIB_BYTES);
-                    const uint2 wP2 = *reinterpret_cast<const uint2 *>(vb + 4 * NIB_BYTES);
-                    const uint2 wP3 = *reinterpret_cast<const uint2 *>(vb + 5 * NIB_BYTES);
-                    const bool kf_a = (FMT == DKV_FMT_DELTA) && (MODE == SUFFIX) && first_seg &&
-                                      t == 0 && tq == 0;
-                    const uint32_t sel0 = kf_a ? 0x3254u : 0x3210u;
-                    const uint32_t sel1 = kf_a ? 0x3276u : 0x3210u;
-#pragma unroll
-                    for (int mt = 0; mt < 8; ++mt) {
-                        const int i = mt & 3;
-                        const uint32_t sel = (uint32_t)(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
-                        // k pairs: (pos 8tq+2t, +4) | (8tq+2t+1, +5)
-                        const uint32_t m01 = prmt(mt < 4 ? wP0.x : wP0.y, mt < 4 ? wP2.x : wP2.y, sel);
-                        const uint32_t m23 = prmt(mt < 4 ? wP1.x : wP1.y, mt < 4 ? wP3.x : wP3.y, sel);
-                        uint32_t a0, a1, a2, a3;
-                        dq_pair(m01, magic, a0, a1);
-                        dq_pair(m23, magic, a2, a3);
-                        if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0) {
-                            a0 = prmt(a0, vkf[mt], sel0);
-                            a1 = prmt(a1, vkf[mt], sel1);
-                        }
-                        const int j = mt >> 1;
-                        if ((mt & 1) == 0) make_b(j, bp, bl);
-                        mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
-                        if (MODE == PREFIX) mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
-                        if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0)
-                            mma16816(o[mt], a0, a1, a2, a3, bk, 0u);
-                        if (MODE == PREFIX) {
-                            // R += sum_s (code-8) * d_s : B = the scales alone
-                            uint32_t r2[2];
-#pragma unroll
-                            for (int r = 0; r < 2; ++r) {
-                                const uint32_t u = dvw[t][r][j >> 1];
-                                const float d = (j & 1) ? h_hi(u) : h_lo(u);
-                                r2[r] = movm_t(pack_h2(d, d));
-                            }
-                            mma16816(racc[mt], a0, a1, a2, a3, r2[0], r2[1]);
-                        }
-                    }
-                }
+            for (int u = 0; u < NU; ++u) {
+                const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
+                v_side<FMT, MODE>(st, sm, first_seg, gq, tq, magic, x[u], dvw[u], o, racc,
+                                  vkf_keep);
             }
 
             // PREFIX: close the group  o += W_g (v_f + R_g)
@@ -769,12 +867,9 @@ __global__ void __launch_bounds__(WARPS * 32, FmtCfg<FMT>::MINB) split_kernel(Sp
         __syncwarp();
         ++consumed;
         if (ic.valid() && !dead) {
-            if (lane == 0) {
-                fence_proxy_async();
-                mymeta[stage_i] = make_meta<MODE>(cv, ic);
-                issue_stage<FMT, MODE>(cv, ic, A.NHG, mystages + stage_i * STAGE, mybar + stage_i);
-            }
-            cursor_next<MODE>(ic, cv, nvs, A.NHG);
+            if (lane == 0) fence_proxy_async();
+            next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + stage_i * STAGE, mybar + stage_i,
+                                  mymeta + stage_i, lane);
             ++issued;
         }
         stage_i = (stage_i + 1 == NS) ? 0 : stage_i + 1;
@@ -852,7 +947,7 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
 // ---------------------------------------------------------------------------
 template <int FMT, int MODE>
 static size_t split_smem() {
-    return (size_t)SmemMap<FMT>::BYTES;
+    return (size_t)SmemMap<FMT, MODE>::BYTES;
 }
 
 template <int FMT, int MODE>

@@ -189,6 +189,7 @@ dkv_status dkv_decode_attn_split(const dkv_cache *cache, const void *Q, int32_t 
                                  size_t ws_bytes, void *stream) {
     int64_t need;
     if (!Q) return DKV_EINVAL;
+    if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return DKV_EINVAL;  // finite, > 0
     dkv_status s = check_decode(cache, Q, q_dtype, n_q_heads, workspace, ws_bytes, &need);
     if (s != DKV_OK) return s;
     CacheView v = view_of(cache);

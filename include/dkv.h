@@ -135,7 +135,8 @@ size_t dkv_decode_workspace_bytes(const dkv_cache_desc *desc, int32_t n_q_heads)
  * over the positions p < seq_len[b] (no mask beyond the length; an empty
  * sequence gives zeros).
  * Q: [B][n_q_heads][D] device array of q_dtype; out: [B][n_q_heads][D] fp32
- * device array; workspace: device scratch of >= dkv_decode_workspace_bytes.
+ * device array; workspace: device scratch of >= dkv_decode_workspace_bytes;
+ * softmax_scale must be finite and > 0 (DKV_EINVAL otherwise).
  * Runs dkv_decode_attn_split then dkv_decode_attn_merge. */
 dkv_status dkv_decode_attn(const dkv_cache *cache, const void *Q, int32_t q_dtype,
                            int32_t n_q_heads, float softmax_scale, float *out,
