@@ -472,8 +472,8 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
 // V side of one unit: o += sum over positions of dequantised V rows times the
 // weights w[t][r][e] (position 4g + 2t + r, head 2tq + e) and their V scales.
 template <int FMT, int MODE>
-__device__ inline void v_side(const uint8_t *st, const StageMap &sm, bool first_seg, int gq, int tq,
-                              uint32_t magic, const float (&w)[2][2][2],
+__device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, bool first_seg,
+                              int gq, int tq, uint32_t magic, const float (&w)[2][2][2],
                               const uint32_t (&dvw)[2][2][2], float (&o)[8][4],
                               float (&racc)[8][4], uint32_t (&vkf_keep)[8]) {
     const bool kfrow = first_seg && gq == 0;
@@ -513,6 +513,35 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, bool first_
             }
         };
         uint32_t bp[2], bl[2] = {0u, 0u};
+        // Q4_0: transpose the weights once per tile and apply block j's V scale
+        // in the transposed layout, where row k of the B fragment is one of the
+        // positions whose V nibbles this thread loads (k 2tq, 2tq+1 <-> P0,
+        // P0+4; k 2tq+8, 2tq+9 <-> P0+1, P0+5).  (Measured faster for Q4_0; the
+        // delta format keeps one fp32 product and one rounding per weight.)
+        constexpr bool TSCALE = FMT == DKV_FMT_Q4_0;
+        uint32_t wt[2] = {0u, 0u};
+        uint2 dq[4] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u),
+                       make_uint2(0u, 0u)};
+        if (TSCALE) {
+            wt[0] = movm_t(pack_h2(w[t][0][0], w[t][0][1]));
+            wt[1] = movm_t(pack_h2(w[t][1][0], w[t][1][1]));
+            const int P0 = 8 * tq + 2 * t;
+            const int ps[4] = {P0, P0 + 4, P0 + 1, P0 + 5};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                dq[i] = *reinterpret_cast<const uint2 *>(st + sm.sc0 + ps[i] * SC_BYTES + 8);
+                if (ps[i] >= npos) dq[i] = make_uint2(0u, 0u);  // stale slot: no weight
+            }
+            if (FMT == DKV_FMT_DELTA && t == 0 && tq == 0 && first_seg)
+                dq[0] = make_uint2(0x3C003C00u, 0x3C003C00u);   // keyframe row: scale 1
+        }
+        auto make_bt = [&](int j, uint32_t (&b)[2]) {
+            const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
+            const uint32_t d01 = prmt((j >> 1) ? dq[0].y : dq[0].x, (j >> 1) ? dq[1].y : dq[1].x, sel);
+            const uint32_t d23 = prmt((j >> 1) ? dq[2].y : dq[2].x, (j >> 1) ? dq[3].y : dq[3].x, sel);
+            b[0] = h2_as_u32(__hmul2(u32_as_h2(wt[0]), u32_as_h2(d01)));
+            b[1] = h2_as_u32(__hmul2(u32_as_h2(wt[1]), u32_as_h2(d23)));
+        };
         // kf <= 32: lo part of the keyframe row's weight (position 0, scale 1)
         uint32_t bk = 0u;
         if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0 && first_seg) {
@@ -567,7 +596,10 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, bool first_
                     a1 = prmt(a1, vkf[mt], sel1);
                 }
                 const int j = mt >> 1;
-                if ((mt & 1) == 0) make_b(j, bp, bl);
+                if ((mt & 1) == 0) {
+                    if (TSCALE) make_bt(j, bp);
+                    else make_b(j, bp, bl);
+                }
                 mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
                 if (MODE == PREFIX) mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
                 if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0)
@@ -844,7 +876,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
-                v_side<FMT, MODE>(st, sm, first_seg, gq, tq, magic, x[u], dvw[u], o, racc,
+                v_side<FMT, MODE>(st, sm, npos[u], first_seg, gq, tq, magic, x[u], dvw[u], o, racc,
                                   vkf_keep);
             }
 
