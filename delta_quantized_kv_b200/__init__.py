@@ -49,7 +49,8 @@ _lib = None
 EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode", "dkv_append",
            "dkv_decode_workspace_bytes", "dkv_decode_attn", "dkv_decode_attn_split",
            "dkv_decode_attn_merge", "dkv_export_canonical", "dkv_dequantize",
-           "dkv_get_device_status", "dkv_status_str", "dkv_decode_attn_noalloc"]
+           "dkv_get_device_status", "dkv_status_str", "dkv_decode_attn_noalloc",
+           "dkv_debug_set_fault"]
 
 
 def load():
@@ -79,6 +80,7 @@ def load():
         "dkv_get_device_status": ([PC, ctypes.POINTER(I), P], I),
         "dkv_status_str": ([I], ctypes.c_char_p),
         "dkv_decode_attn_noalloc": ([PC, P, I, I, F, P, P], I),
+        "dkv_debug_set_fault": ([I], None),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -198,6 +200,11 @@ def dkv_export_canonical(cache: dkv_cache, codes=None, scales=None, keyframes=No
 def dkv_dequantize(cache: dkv_cache, out, stream=None) -> None:
     _check(load().dkv_dequantize(ctypes.byref(cache), _ptr(out), _stream(stream)),
            "dkv_dequantize")
+
+
+def dkv_debug_set_fault(mode: int) -> None:
+    """Test support: mode 1 makes later split launches time out by design."""
+    load().dkv_debug_set_fault(int(mode))
 
 
 def dkv_get_device_status(cache: dkv_cache, stream=None) -> int:

@@ -94,6 +94,7 @@ struct SplitArgs {
     int Hq, G, NHG;            // query heads, heads per kv head, head groups of 8
     float scale_log2;          // softmax_scale * log2(e), > 0
     float *ws;                 // partial records
+    int fault;                 // test support: 1 = arm the copy barriers but issue no copy
 };
 
 __host__ __device__ inline int units_of(int fmt, int kf, int len) {
@@ -262,9 +263,15 @@ __device__ inline StageMap stage_map(int kf, int64_t rec, int u) {
 // Issue the bulk copies of one stage (nu units starting at c; one lane).
 template <int FMT, int MODE>
 __device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nu, int npos_all,
-                                   uint8_t *stage, uint64_t *bar) {
+                                   uint8_t *stage, uint64_t *bar, int fault) {
     constexpr int NU = KCfg<FMT, MODE>::NU;
     const uint8_t *sb = c.seq;
+    if (fault) {
+        // test support: expect bytes that never come, so the consumer's bounded
+        // wait runs out and reports DKV_DEV_TIMEOUT
+        mbar_arrive_expect_tx(bar, 16);
+        return;
+    }
     if (FMT == DKV_FMT_DELTA && MODE == SUFFIX) {
         const uint32_t bytes = (uint32_t)(nu * cv.rec_bytes);
         mbar_arrive_expect_tx(bar, bytes);
@@ -313,7 +320,7 @@ __device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nu,
 // lane advances its cursor identically.
 template <int FMT, int MODE>
 __device__ inline void next_stage(const CacheView &cv, Cursor &c, int nvs, int nhg, uint8_t *stage,
-                                  uint64_t *bar, StageMeta *meta, int lane) {
+                                  uint64_t *bar, StageMeta *meta, int lane, int fault) {
     constexpr int NU = KCfg<FMT, MODE>::NU;
     const int np0 = unit_npos(cv, c, c.g);
     int nu = 1, np1 = 0;
@@ -328,7 +335,7 @@ __device__ inline void next_stage(const CacheView &cv, Cursor &c, int nvs, int n
         m.npos = np0 | (np1 << 8);
         m.flags = MODE == PREFIX ? ((c.seg == 0 ? 1 : 0) | (c.seg == c.nseg - 1 ? 2 : 0)) : 3;
         *meta = m;
-        issue_stage<FMT, MODE>(cv, c, nu, np0 + np1, stage, bar);
+        issue_stage<FMT, MODE>(cv, c, nu, np0 + np1, stage, bar, fault);
     }
     cursor_next<MODE>(c, cv, nvs, nhg);
     if (nu == 2) cursor_next<MODE>(c, cv, nvs, nhg);
@@ -670,7 +677,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
 #pragma unroll 1
     for (int s = 0; s < NS; ++s) {
         if (ic.valid()) {
-            next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + s * STAGE, mybar + s, mymeta + s, lane);
+            next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + s * STAGE, mybar + s, mymeta + s, lane, A.fault);
             ++issued;
         }
     }
@@ -901,7 +908,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
         if (ic.valid() && !dead) {
             if (lane == 0) fence_proxy_async();
             next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + stage_i * STAGE, mybar + stage_i,
-                                  mymeta + stage_i, lane);
+                                  mymeta + stage_i, lane, A.fault);
             ++issued;
         }
         stage_i = (stage_i + 1 == NS) ? 0 : stage_i + 1;
@@ -1026,9 +1033,11 @@ static cudaError_t launch_split_t(const SplitArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq,
-                         float softmax_scale, float *ws, int64_t ws_floats, cudaStream_t st) {
+                         float softmax_scale, float *ws, int64_t ws_floats, int fault,
+                         cudaStream_t st) {
     (void)ws_floats;
     SplitArgs a;
+    a.fault = fault;
     a.cv = cv;
     a.Q = Q;
     a.q_dtype = q_dtype;

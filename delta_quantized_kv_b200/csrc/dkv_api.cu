@@ -90,6 +90,8 @@ CacheView view_of(const dkv_cache *c) {
 
 inline dkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DKV_OK : DKV_ECUDA; }
 
+int g_debug_fault = 0;   // dkv_debug_set_fault
+
 inline bool valid_dtype(int32_t t) { return t == DKV_F32 || t == DKV_F16 || t == DKV_BF16; }
 
 int64_t workspace_floats(const dkv_cache_desc *d, int32_t Hq, bool *ok) {
@@ -194,7 +196,7 @@ dkv_status dkv_decode_attn_split(const dkv_cache *cache, const void *Q, int32_t 
     if (s != DKV_OK) return s;
     CacheView v = view_of(cache);
     return cuda_status(dkv::launch_split(v, Q, q_dtype, n_q_heads, softmax_scale,
-                                         static_cast<float *>(workspace), need,
+                                         static_cast<float *>(workspace), need, g_debug_fault,
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -258,6 +260,8 @@ dkv_status dkv_get_device_status(const dkv_cache *cache, int32_t *host_out, void
     *host_out = h;
     return h ? DKV_EDEVICE : DKV_OK;
 }
+
+void dkv_debug_set_fault(int32_t mode) { g_debug_fault = mode == 1 ? 1 : 0; }
 
 const char *dkv_status_str(dkv_status s) {
     switch (s) {

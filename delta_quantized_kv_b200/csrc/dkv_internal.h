@@ -26,7 +26,8 @@ cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g);
 constexpr int PARTIAL_FLOATS = 8 + 8 + 8 * 128;
 
 cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq,
-                         float softmax_scale, float *ws, int64_t ws_floats, cudaStream_t st);
+                         float softmax_scale, float *ws, int64_t ws_floats, int fault,
+                         cudaStream_t st);
 cudaError_t launch_merge(const CacheView &cv, int Hq, float *out, const float *ws,
                          cudaStream_t st);
 

@@ -192,6 +192,15 @@ dkv_status dkv_dequantize(const dkv_cache *cache, float *out, void *stream);
  * it.  Returns DKV_EDEVICE if it was non-zero, DKV_OK otherwise. */
 dkv_status dkv_get_device_status(const dkv_cache *cache, int32_t *host_out, void *stream);
 
+/* Test support for failure detection (no counterpart on the pages).  With
+ * mode 1, later decode-attention split launches from this process arm their
+ * copy barriers without issuing the copies, so every bounded pipeline wait
+ * runs out (after about a second) and the kernel records DKV_DEV_TIMEOUT in
+ * the status word and returns, instead of hanging; the outputs of such a
+ * launch are meaningless.  Mode 0 restores normal operation.  Nothing traps
+ * or faults either way.  Not thread-safe; meant for tests. */
+void dkv_debug_set_fault(int32_t mode);
+
 /* Static description of a status code. */
 const char *dkv_status_str(dkv_status s);
 

@@ -1,0 +1,76 @@
+"""Multi-rank host logic of bench.py on CPU with the gloo backend
+(world size 2): the timing reduction takes the max over ranks, the barrier
+completes, and only rank 0 runs the reference arm."""
+import io
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+from pathlib import Path
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, str(ROOT))
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        bench.barrier(world)
+        got = bench.max_over_ranks(1.5 + rank, world)
+        r, w, l = bench.dist_env()
+        q.put((rank, got, r, w, l))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_env_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [2.5, 2.5]
+    assert [(r[2], r[3], r[4]) for r in res] == [(0, 2, 0), (1, 2, 1)]
+
+
+def test_reference_arm_other_ranks_exit_silently(monkeypatch):
+    sys.path.insert(0, str(ROOT))
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        rc = bench.main(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"])
+    assert rc == 0 and buf.getvalue() == ""
+
+
+def test_kv_bytes_model():
+    sys.path.insert(0, str(ROOT))
+    import bench
+    # headline cache: 4,194,304 (token, kv head) units at 155.5 B each
+    assert bench.kv_bytes("delta", [32768] * 16, 8, 32) == 652_214_272
+    assert bench.kv_bytes("q4", [32768] * 16, 8, 32) == 603_979_776
+    assert bench.kv_bytes("fp16", [32768] * 16, 8, 32) == 2_147_483_648
+    # a partial last group still pays a whole keyframe
+    assert bench.kv_bytes("delta", [33], 1, 32) == 2 * 512 + 31 * 144

@@ -124,3 +124,32 @@ def test_workspace_too_small_is_rejected(dkv_gpu):
     with pytest.raises(dkv_gpu.DkvError) as e:
         dkv_gpu.dkv_decode_attn(cache.c, q, dkv_gpu.DKV_F16, 1, 1.0, out, ws, 64)
     assert e.value.status == dkv_gpu.DKV_ECAPACITY
+
+
+def test_pipeline_wait_timeout_is_reported_not_hung(dkv_gpu):
+    """Failure detection without a GPU fault: with the copies dropped on
+    purpose, every bounded wait runs out (~1 s), the kernel records
+    DKV_DEV_TIMEOUT and returns; the context stays usable afterwards."""
+    import time
+    w = S.WORKLOADS["llama3_8b_layer"].with_(T=256)
+    K, V = S.gen_kv(w)
+    q = S.gen_q(w).to(DEV)
+    cache = dkv_gpu.Cache(w.B, w.Hkv, w.T, "delta", kf=32)
+    cache.encode(K.to(DEV), V.to(DEV))
+    good = cache.decode_attn(q, 0.088).clone()
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    dkv_gpu.dkv_debug_set_fault(1)
+    try:
+        t0 = time.time()
+        cache.decode_attn(q, 0.088)
+        st = cache.device_status()          # synchronises
+        dt = time.time() - t0
+    finally:
+        dkv_gpu.dkv_debug_set_fault(0)
+    assert st & dkv_gpu.DEV_TIMEOUT
+    assert dt < 30.0
+    again = cache.decode_attn(q, 0.088)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    assert torch.equal(again, good)
