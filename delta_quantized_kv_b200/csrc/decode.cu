@@ -45,7 +45,10 @@ namespace dkv {
 
 enum Mode { SUFFIX = 0, PREFIX = 1, PLAIN = 2 };
 
-constexpr int WARPS = 4;                     // warps per CTA (independent pipelines)
+#ifndef DKV_WARPS
+#define DKV_WARPS 4
+#endif
+constexpr int WARPS = DKV_WARPS;             // warps per CTA (independent pipelines)
 
 // Nibble formats with kf <= 32: units per stage, stages per warp, CTAs per SM.
 // Two groups per stage and one stage per warp (a warp's next stage is copied
@@ -59,6 +62,27 @@ constexpr int WARPS = 4;                     // warps per CTA (independent pipel
 #endif
 #ifndef DKV_NIB_MINB
 #define DKV_NIB_MINB 3
+#endif
+// Nibble formats with kf <= 32: remove the dequantisation biases inside the
+// K-side MMAs (accumulator input) / the V-side MMAs (one extra MMA per tile);
+// build the V-side B fragments with one fp16x2 multiply.
+#ifndef DKV_KBIAS
+#define DKV_KBIAS 0
+#endif
+#ifndef DKV_VBIAS
+#define DKV_VBIAS 0
+#endif
+#ifndef DKV_HMUL_B
+#define DKV_HMUL_B 1
+#endif
+// Delta, kf <= 32: the keyframe row's V contribution as an fp32 rank-1 update
+// (v_f times the group's total weight) instead of an fp16 hi + lo pair of MMAs.
+#ifndef DKV_KF_FFMA
+#define DKV_KF_FFMA 1
+#endif
+// Nibble formats: skip the tail masks of stages whose units are all full.
+#ifndef DKV_FULL_FAST
+#define DKV_FULL_FAST 0
 #endif
 
 // Per (format, mode): units per stage, stage bytes, stages per warp, CTAs/SM.
@@ -77,12 +101,16 @@ template <int FMT, int MODE> struct KCfg {
 // aligned; the offsets follow from NS so no region can overlap another.
 template <int FMT, int MODE> struct SmemMap {
     static constexpr int NS = KCfg<FMT, MODE>::NS, STAGE = KCfg<FMT, MODE>::STAGE;
+    static constexpr int KBT = 256 + 32;      // per warp: K-side bias table, keyframe terms
     static constexpr int BAR_OFF = 0;
     static constexpr int META_OFF = ((BAR_OFF + 8 * WARPS * NS) + 15) / 16 * 16;
-    static constexpr int STAGE_OFF = ((META_OFF + 16 * WARPS * NS) + 127) / 128 * 128;
+    static constexpr int KBT_OFF = ((META_OFF + 16 * WARPS * NS) + 15) / 16 * 16;
+    static constexpr int STAGE_OFF = ((KBT_OFF + KBT * WARPS) + 127) / 128 * 128;
     static constexpr int BYTES = STAGE_OFF + WARPS * NS * STAGE;
     static_assert(META_OFF >= BAR_OFF + 8 * WARPS * NS, "barriers overlap descriptors");
-    static_assert(STAGE_OFF >= META_OFF + 16 * WARPS * NS, "descriptors overlap stages");
+    static_assert(KBT_OFF >= META_OFF + 16 * WARPS * NS, "descriptors overlap the bias tables");
+    static_assert(STAGE_OFF >= KBT_OFF + KBT * WARPS, "bias tables overlap stages");
+    static_assert(KBT % 16 == 0, "bias table rows are 16-byte loads");
     static_assert(STAGE % 128 == 0, "stages must stay 128-byte aligned");
     static_assert(BYTES <= 227 * 1024, "shared memory per CTA");
 };
@@ -394,12 +422,53 @@ __device__ inline float col_scan32(float (&v)[4], int lane) {
 //   n = heads; the weights reach that B layout through an 8x8 transpose
 //   (movmatrix) of the K-side accumulator layout.
 
+// K-side bias removal (nibble formats, whole groups per unit).  A low-nibble
+// channel dequantises to 1024 + n and a high-nibble channel to 64 + n, so for
+// head h and 32-channel block j
+//     sum_c (n_c - 8) q_hc = sum_c A_c q_hc - (1032 sum_low q_hc + 72 sum_high q_hc);
+// the bracket, of the fp16 q the tensor cores multiply, enters negated as the
+// accumulator input of the block's first MMA.  Per warp, a shared-memory table
+// holds it where the MMA wants it: row (tq, j) = {-B_j(2tq), -B_j(2tq+1),
+// -B_j(2tq), -B_j(2tq+1)} (16 B, one load per block), then per tq the pair
+// sum_j B_j(2tq + e) that gives the keyframe row (raw fp16 values, no bias) its
+// biases back.
+__device__ inline void write_kbias(const uint32_t (&qb)[8][2], int gq, int tq, float *tab) {
+    float part[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // this thread's 8 channels of block j for head gq: k rows 2tq, 2tq+1
+        // (low nibbles) and 2tq+8, 2tq+9 (high nibbles) of k-steps 2j, 2j+1
+        const uint32_t l0 = qb[2 * j][0], h0 = qb[2 * j][1];
+        const uint32_t l1 = qb[2 * j + 1][0], h1 = qb[2 * j + 1][1];
+        const float sl = (h_lo(l0) + h_hi(l0)) + (h_lo(l1) + h_hi(l1));
+        const float sh = (h_lo(h0) + h_hi(h0)) + (h_lo(h1) + h_hi(h1));
+        float v = 1032.f * sl + 72.f * sh;
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        part[j] = v;                                   // B_j(head gq), every lane of quad gq
+    }
+    if (tq == 0) {
+        const int r = gq >> 1, e = gq & 1;             // head gq sits in column e of tq = r
+        float tot = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            tab[(r * 4 + j) * 4 + e] = -part[j];
+            tab[(r * 4 + j) * 4 + 2 + e] = -part[j];
+            tot += part[j];
+        }
+        tab[64 + 2 * r + e] = tot;
+    }
+    __syncwarp();
+}
+
 // K side of one unit: per-position dot products x[t][r][e] (position
 // 4g + 2t + r, head 2tq + e) and the V scales dvw[t][r] of those positions.
 template <int FMT, int MODE>
 __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, bool first_seg,
-                              int gq, int tq, uint32_t magic, const uint32_t (&qb)[8][2],
-                              float (&x)[2][2][2], uint32_t (&dvw)[2][2][2]) {
+                              int gq, int tq, uint32_t m1024, uint32_t m64,
+                              const uint32_t (&qb)[8][2], const float *kbt, float (&x)[2][2][2],
+                              uint32_t (&dvw)[2][2][2]) {
+    constexpr bool BIASED = KCfg<FMT, MODE>::NIB && DKV_KBIAS;
     const bool kfrow = first_seg && gq == 0;   // this thread's row 0 of tile 0 is the keyframe
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
@@ -426,8 +495,17 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
                 const uint32_t ww1[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    dq_word(ww0[j], magic, a[2 * j][0], a[2 * j][2], a[2 * j + 1][0], a[2 * j + 1][2]);
-                    dq_word(ww1[j], magic, a[2 * j][1], a[2 * j][3], a[2 * j + 1][1], a[2 * j + 1][3]);
+                    if (BIASED) {
+                        dq_word_biased(ww0[j], m1024, m64, a[2 * j][0], a[2 * j][2], a[2 * j + 1][0],
+                                       a[2 * j + 1][2]);
+                        dq_word_biased(ww1[j], m1024, m64, a[2 * j][1], a[2 * j][3], a[2 * j + 1][1],
+                                       a[2 * j + 1][3]);
+                    } else {
+                        dq_word(ww0[j], m1024, m64, a[2 * j][0], a[2 * j][2], a[2 * j + 1][0],
+                                a[2 * j + 1][2]);
+                        dq_word(ww1[j], m1024, m64, a[2 * j][1], a[2 * j][3], a[2 * j + 1][1],
+                                a[2 * j + 1][3]);
+                    }
                 }
             }
             if (FMT == DKV_FMT_DELTA && t == 0 && first_seg) {
@@ -445,9 +523,15 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
             float acc[4][4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-                mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
-                         qb[2 * j][0], qb[2 * j][1]);
+                if (BIASED) {
+                    const float4 c = *reinterpret_cast<const float4 *>(kbt + (tq * 4 + j) * 4);
+                    mma16816c(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
+                              qb[2 * j][0], qb[2 * j][1], c.x, c.y, c.z, c.w);
+                } else {
+                    acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+                    mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
+                             qb[2 * j][0], qb[2 * j][1]);
+                }
                 mma16816(acc[j], a[2 * j + 1][0], a[2 * j + 1][1], a[2 * j + 1][2],
                          a[2 * j + 1][3], qb[2 * j + 1][0], qb[2 * j + 1][1]);
             }
@@ -455,22 +539,34 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
             uint4 s0 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + p0 * SC_BYTES);
             uint4 s1 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + (p0 + 1) * SC_BYTES);
             if (FMT == DKV_FMT_DELTA && t == 0 && kfrow) {
-                s0.x = s0.y = 0x3C003C00u;                          // keyframe: unit K weights
-                s0.z = s0.w = (MODE == SUFFIX) ? 0x3C003C00u : 0u;  // V: 1 (SUFFIX) / 0 (PREFIX)
+                // keyframe: unit K weights; V weight 1 when its row goes through
+                // the MMA (SUFFIX), else 0 (added apart)
+                s0.x = s0.y = 0x3C003C00u;
+                s0.z = s0.w = (MODE == SUFFIX && !DKV_KF_FFMA) ? 0x3C003C00u : 0u;
             }
             // slots past the end of the unit hold stale bytes (possibly NaN
             // patterns): zero their K and V scales so they add nothing to the
             // prefix sums and carry no V weight
-            if (p0 >= npos) s0 = make_uint4(0u, 0u, 0u, 0u);
-            if (p0 + 1 >= npos) s1 = make_uint4(0u, 0u, 0u, 0u);
+            if (!DKV_FULL_FAST || !KCfg<FMT, MODE>::NIB || npos < SEG) {
+                if (p0 >= npos) s0 = make_uint4(0u, 0u, 0u, 0u);
+                if (p0 + 1 >= npos) s1 = make_uint4(0u, 0u, 0u, 0u);
+            }
             dvw[t][0][0] = s0.z; dvw[t][0][1] = s0.w;
             dvw[t][1][0] = s1.z; dvw[t][1][1] = s1.w;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                x[t][0][e] = acc[0][e] * h_lo(s0.x) + acc[1][e] * h_hi(s0.x) +
-                             acc[2][e] * h_lo(s0.y) + acc[3][e] * h_hi(s0.y);
-                x[t][1][e] = acc[0][2 + e] * h_lo(s1.x) + acc[1][2 + e] * h_hi(s1.x) +
-                             acc[2][2 + e] * h_lo(s1.y) + acc[3][2 + e] * h_hi(s1.y);
+                float x0;
+                if (BIASED && FMT == DKV_FMT_DELTA && t == 0)
+                    x0 = fmaf(acc[0][e], h_lo(s0.x), kfrow ? kbt[64 + 2 * tq + e] : 0.f);
+                else
+                    x0 = acc[0][e] * h_lo(s0.x);
+                x0 = fmaf(acc[1][e], h_hi(s0.x), x0);
+                x0 = fmaf(acc[2][e], h_lo(s0.y), x0);
+                x[t][0][e] = fmaf(acc[3][e], h_hi(s0.y), x0);
+                float x1 = acc[0][2 + e] * h_lo(s1.x);
+                x1 = fmaf(acc[1][2 + e], h_hi(s1.x), x1);
+                x1 = fmaf(acc[2][2 + e], h_lo(s1.y), x1);
+                x[t][1][e] = fmaf(acc[3][2 + e], h_hi(s1.y), x1);
             }
         }
     }
@@ -480,9 +576,10 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
 // weights w[t][r][e] (position 4g + 2t + r, head 2tq + e) and their V scales.
 template <int FMT, int MODE>
 __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, bool first_seg,
-                              int gq, int tq, uint32_t magic, const float (&w)[2][2][2],
-                              const uint32_t (&dvw)[2][2][2], float (&o)[8][4],
-                              float (&racc)[8][4], uint32_t (&vkf_keep)[8]) {
+                              int gq, int tq, uint32_t m1024, uint32_t m64,
+                              const float (&w)[2][2][2], const uint32_t (&dvw)[2][2][2],
+                              float (&o)[8][4], float (&racc)[8][4], uint32_t (&vkf_keep)[8]) {
+    constexpr bool VBIASED = KCfg<FMT, MODE>::NIB && DKV_VBIAS;
     const bool kfrow = first_seg && gq == 0;
     uint32_t vkf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     if (FMT == DKV_FMT_DELTA && first_seg) {
@@ -497,67 +594,11 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
     }
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        // B fragments (k = positions, n = head g) of block j: transpose of the
-        // (position, head-pair) layout of W_j = weight * dV_j.  A delta row's
-        // weight rounding is shared by every channel of the row: the keyframe
-        // row (the group's total weight times v_f) gets an fp16 hi + lo pair;
-        // with kf > 32 the prefix weights -E_s aggregate up to kf positions, so
-        // every row gets the pair; the comparators weight one token per row
-        // with one fp16 weight, as flash-decoding does.
-        auto make_b = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2]) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                float d = 1.f;
-                if (FMT != DKV_FMT_FP16) {
-                    const uint32_t u = dvw[t][r][j >> 1];
-                    d = (j & 1) ? h_hi(u) : h_lo(u);
-                }
-                const float v0 = w[t][r][0] * d, v1 = w[t][r][1] * d;
-                const uint32_t hi = pack_h2(v0, v1);
-                b[r] = movm_t(hi);
-                if (FMT == DKV_FMT_DELTA && MODE == PREFIX)
-                    bl[r] = movm_t(pack_h2(v0 - h_lo(hi), v1 - h_hi(hi)));
-            }
-        };
-        uint32_t bp[2], bl[2] = {0u, 0u};
-        // Q4_0: transpose the weights once per tile and apply block j's V scale
-        // in the transposed layout, where row k of the B fragment is one of the
-        // positions whose V nibbles this thread loads (k 2tq, 2tq+1 <-> P0,
-        // P0+4; k 2tq+8, 2tq+9 <-> P0+1, P0+5).  (Measured faster for Q4_0; the
-        // delta format keeps one fp32 product and one rounding per weight.)
-        constexpr bool TSCALE = FMT == DKV_FMT_Q4_0;
-        uint32_t wt[2] = {0u, 0u};
-        uint2 dq[4] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u),
-                       make_uint2(0u, 0u)};
-        if (TSCALE) {
-            wt[0] = movm_t(pack_h2(w[t][0][0], w[t][0][1]));
-            wt[1] = movm_t(pack_h2(w[t][1][0], w[t][1][1]));
-            const int P0 = 8 * tq + 2 * t;
-            const int ps[4] = {P0, P0 + 4, P0 + 1, P0 + 5};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                dq[i] = *reinterpret_cast<const uint2 *>(st + sm.sc0 + ps[i] * SC_BYTES + 8);
-                if (ps[i] >= npos) dq[i] = make_uint2(0u, 0u);  // stale slot: no weight
-            }
-            if (FMT == DKV_FMT_DELTA && t == 0 && tq == 0 && first_seg)
-                dq[0] = make_uint2(0x3C003C00u, 0x3C003C00u);   // keyframe row: scale 1
-        }
-        auto make_bt = [&](int j, uint32_t (&b)[2]) {
-            const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
-            const uint32_t d01 = prmt((j >> 1) ? dq[0].y : dq[0].x, (j >> 1) ? dq[1].y : dq[1].x, sel);
-            const uint32_t d23 = prmt((j >> 1) ? dq[2].y : dq[2].x, (j >> 1) ? dq[3].y : dq[3].x, sel);
-            b[0] = h2_as_u32(__hmul2(u32_as_h2(wt[0]), u32_as_h2(d01)));
-            b[1] = h2_as_u32(__hmul2(u32_as_h2(wt[1]), u32_as_h2(d23)));
-        };
-        // kf <= 32: lo part of the keyframe row's weight (position 0, scale 1)
-        uint32_t bk = 0u;
-        if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0 && first_seg) {
-            const float r0 = w[0][0][0] - __half2float(__float2half_rn(w[0][0][0]));
-            const float r1 = w[0][0][1] - __half2float(__float2half_rn(w[0][0][1]));
-            bk = movm_t(kfrow ? pack_h2(r0, r1) : 0u);
-        }
         if (FMT == DKV_FMT_FP16) {
-            make_b(0, bp, bl);
+            // one token per row: one fp16 weight, as flash-decoding does
+            uint32_t bp[2];
+            bp[0] = movm_t(pack_h2(w[t][0][0], w[t][0][1]));
+            bp[1] = movm_t(pack_h2(w[t][1][0], w[t][1][1]));
             // V values of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
             const uint8_t *vb = st + 8192 + (8 * tq + 2 * t) * 256 + 32 * gq;
             uint32_t wv[4][8];
@@ -577,51 +618,131 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
                 const uint32_t a3 = prmt(wv[1][mt], wv[3][mt], 0x7632u);
                 mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
             }
-        } else {
-            // V nibbles of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
-            const uint8_t *vb = st + sm.vn0 + (8 * tq + 2 * t) * NIB_BYTES + 8 * gq;
-            const uint2 wP0 = *reinterpret_cast<const uint2 *>(vb);
-            const uint2 wP1 = *reinterpret_cast<const uint2 *>(vb + NIB_BYTES);
-            const uint2 wP2 = *reinterpret_cast<const uint2 *>(vb + 4 * NIB_BYTES);
-            const uint2 wP3 = *reinterpret_cast<const uint2 *>(vb + 5 * NIB_BYTES);
-            const bool kf_a = (FMT == DKV_FMT_DELTA) && (MODE == SUFFIX) && first_seg && t == 0 &&
-                              tq == 0;
-            const uint32_t sel0 = kf_a ? 0x3254u : 0x3210u;
-            const uint32_t sel1 = kf_a ? 0x3276u : 0x3210u;
+            continue;
+        }
+        // V nibbles of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
+        const uint8_t *vb = st + sm.vn0 + (8 * tq + 2 * t) * NIB_BYTES + 8 * gq;
+        const uint2 wP0 = *reinterpret_cast<const uint2 *>(vb);
+        const uint2 wP1 = *reinterpret_cast<const uint2 *>(vb + NIB_BYTES);
+        const uint2 wP2 = *reinterpret_cast<const uint2 *>(vb + 4 * NIB_BYTES);
+        const uint2 wP3 = *reinterpret_cast<const uint2 *>(vb + 5 * NIB_BYTES);
+        auto codes = [&](int mt, bool biased, uint32_t &a0, uint32_t &a1, uint32_t &a2,
+                         uint32_t &a3) {
+            const int i = mt & 3;
+            const uint32_t sel = (uint32_t)(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
+            // k pairs: (pos 8tq+2t, +4) | (8tq+2t+1, +5)
+            const uint32_t m01 = prmt(mt < 4 ? wP0.x : wP0.y, mt < 4 ? wP2.x : wP2.y, sel);
+            const uint32_t m23 = prmt(mt < 4 ? wP1.x : wP1.y, mt < 4 ? wP3.x : wP3.y, sel);
+            if (biased) {
+                dq_pair_biased(m01, m1024, m64, a0, a1);
+                dq_pair_biased(m23, m1024, m64, a2, a3);
+            } else {
+                dq_pair(m01, m1024, m64, a0, a1);
+                dq_pair(m23, m1024, m64, a2, a3);
+            }
+        };
+        if (MODE != PREFIX) {
+            constexpr bool VB = VBIASED;
+            // B fragments (k = positions, n = head g) of block j: the 8x8
+            // transpose of the weights times block j's V scale, in fp16 (one
+            // token per row for Q4_0; for the delta format the keyframe row gets
+            // an extra lo fragment below).
+            const uint32_t wp0 = pack_h2(w[t][0][0], w[t][0][1]);
+            const uint32_t wp1 = pack_h2(w[t][1][0], w[t][1][1]);
+            auto make_b = [&](int j, uint32_t (&b)[2]) {
+                const uint32_t u0 = dvw[t][0][j >> 1], u1 = dvw[t][1][j >> 1];
+                if (DKV_HMUL_B) {
+                    const __half2 d0 = (j & 1) ? __high2half2(u32_as_h2(u0)) : __low2half2(u32_as_h2(u0));
+                    const __half2 d1 = (j & 1) ? __high2half2(u32_as_h2(u1)) : __low2half2(u32_as_h2(u1));
+                    b[0] = movm_t(h2_as_u32(__hmul2(u32_as_h2(wp0), d0)));
+                    b[1] = movm_t(h2_as_u32(__hmul2(u32_as_h2(wp1), d1)));
+                } else {
+                    const float d0 = (j & 1) ? h_hi(u0) : h_lo(u0);
+                    const float d1 = (j & 1) ? h_hi(u1) : h_lo(u1);
+                    b[0] = movm_t(pack_h2(w[t][0][0] * d0, w[t][0][1] * d0));
+                    b[1] = movm_t(pack_h2(w[t][1][0] * d1, w[t][1][1] * d1));
+                }
+            };
+            // delta: the keyframe row's weight (the group total, scale 1) as fp16
+            // hi (in the B fragment) + lo (this extra fragment, nonzero only at
+            // the keyframe's k slot)
+            constexpr bool KF = FMT == DKV_FMT_DELTA && !DKV_KF_FFMA;
+            uint32_t bk = 0u;
+            if (KF && t == 0) {
+                const float r0 = w[0][0][0] - h_lo(wp0);
+                const float r1 = w[0][0][1] - h_hi(wp0);
+                bk = movm_t(kfrow ? pack_h2(r0, r1) : 0u);
+            }
+            // bias removal: A rows -1032 (rows g: low nibbles) and -72 (rows g+8:
+            // high nibbles) against the same B fragments; the keyframe slot
+            // (k = 2tq of t = 0, tq = 0) holds raw fp16 values and no bias
+            const bool kslot = KF && t == 0 && tq == 0;
+            const uint32_t cl = 0xE408E408u, ch = 0xD480D480u;
+            const uint32_t cl0 = kslot ? 0xE4080000u : cl;
+            const uint32_t ch0 = kslot ? 0xD4800000u : ch;
+            const uint32_t sel0 = kslot ? 0x3254u : 0x3210u;
+            const uint32_t sel1 = kslot ? 0x3276u : 0x3210u;
+            uint32_t bp[2];
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
-                const int i = mt & 3;
-                const uint32_t sel = (uint32_t)(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
-                // k pairs: (pos 8tq+2t, +4) | (8tq+2t+1, +5)
-                const uint32_t m01 = prmt(mt < 4 ? wP0.x : wP0.y, mt < 4 ? wP2.x : wP2.y, sel);
-                const uint32_t m23 = prmt(mt < 4 ? wP1.x : wP1.y, mt < 4 ? wP3.x : wP3.y, sel);
                 uint32_t a0, a1, a2, a3;
-                dq_pair(m01, magic, a0, a1);
-                dq_pair(m23, magic, a2, a3);
-                if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0) {
+                codes(mt, VB, a0, a1, a2, a3);
+                if (KF && t == 0) {
                     a0 = prmt(a0, vkf[mt], sel0);
                     a1 = prmt(a1, vkf[mt], sel1);
                 }
-                const int j = mt >> 1;
-                if ((mt & 1) == 0) {
-                    if (TSCALE) make_bt(j, bp);
-                    else make_b(j, bp, bl);
-                }
+                if ((mt & 1) == 0) make_b(mt >> 1, bp);
                 mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
-                if (MODE == PREFIX) mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
-                if (FMT == DKV_FMT_DELTA && MODE == SUFFIX && t == 0)
-                    mma16816(o[mt], a0, a1, a2, a3, bk, 0u);
-                if (MODE == PREFIX) {
-                    // R += sum_s (code-8) * d_s : B = the scales alone
-                    uint32_t r2[2];
+                if (VB) mma16816(o[mt], cl0, ch0, cl, ch, bp[0], bp[1]);
+                if (KF && t == 0) mma16816(o[mt], a0, a1, a2, a3, bk, 0u);
+            }
+            if (FMT == DKV_FMT_DELTA && DKV_KF_FFMA && t == 0) {
+                // keyframe row: o += v_f * (the group's total weight), in fp32;
+                // the total of heads 2tq + e sits in w[0][0][e] of lane tq (g = 0)
+                const float S0 = __shfl_sync(0xffffffffu, w[0][0][0], tq);
+                const float S1 = __shfl_sync(0xffffffffu, w[0][0][1], tq);
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const uint32_t u = dvw[t][r][j >> 1];
-                        const float d = (j & 1) ? h_hi(u) : h_lo(u);
-                        r2[r] = movm_t(pack_h2(d, d));
-                    }
-                    mma16816(racc[mt], a0, a1, a2, a3, r2[0], r2[1]);
+                for (int mt = 0; mt < 8; ++mt) {
+                    const float vl = h_lo(vkf[mt]), vh = h_hi(vkf[mt]);
+                    o[mt][0] = fmaf(vl, S0, o[mt][0]);
+                    o[mt][1] = fmaf(vl, S1, o[mt][1]);
+                    o[mt][2] = fmaf(vh, S0, o[mt][2]);
+                    o[mt][3] = fmaf(vh, S1, o[mt][3]);
                 }
+            }
+        } else {
+            // PREFIX (kf > 32): the prefix weights -E_s aggregate up to kf
+            // positions, so every row's weight (times its V scale, in fp32) is an
+            // fp16 hi + lo pair.
+            auto make_b = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2]) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const uint32_t u = dvw[t][r][j >> 1];
+                    const float d = (j & 1) ? h_hi(u) : h_lo(u);
+                    const float v0 = w[t][r][0] * d, v1 = w[t][r][1] * d;
+                    const uint32_t hi = pack_h2(v0, v1);
+                    b[r] = movm_t(hi);
+                    bl[r] = movm_t(pack_h2(v0 - h_lo(hi), v1 - h_hi(hi)));
+                }
+            };
+            uint32_t bp[2], bl[2];
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                uint32_t a0, a1, a2, a3;
+                codes(mt, false, a0, a1, a2, a3);
+                const int j = mt >> 1;
+                if ((mt & 1) == 0) make_b(j, bp, bl);
+                mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
+                mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
+                // R += sum_s (code-8) * d_s : B = the scales alone
+                uint32_t r2[2];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const uint32_t u = dvw[t][r][j >> 1];
+                    const float d = (j & 1) ? h_hi(u) : h_lo(u);
+                    r2[r] = movm_t(pack_h2(d, d));
+                }
+                mma16816(racc[mt], a0, a1, a2, a3, r2[0], r2[1]);
             }
         }
     }
@@ -641,7 +762,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
     uint64_t *mybar = reinterpret_cast<uint64_t *>(smem + Map::BAR_OFF) + warp * NS;
     StageMeta *mymeta = reinterpret_cast<StageMeta *>(smem + Map::META_OFF) + warp * NS;
     uint8_t *mystages = smem + Map::STAGE_OFF + warp * NS * STAGE;
-    const uint32_t magic = magic_1024x2();
+    const uint32_t m1024 = magic_1024x2(), m64 = magic_64x2();
 
     if (lane == 0) {
         for (int s = 0; s < NS; ++s) mbar_init(mybar + s, 1);
@@ -688,6 +809,8 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
     // per-sequence state (heads 2*tq + e of the current head group)
     int cur_b = -1, cur_vs = -1;
     uint32_t qb[8][2];                  // B fragments of q (column = head gq)
+    float *kbt = reinterpret_cast<float *>(smem + Map::KBT_OFF + warp * Map::KBT);
+    bool heads_all = false;             // all 8 heads of the head group exist
     bool head_ok[2] = {false, false};
     float m_run[2] = {-1e30f, -1e30f}, l_run[2] = {0.f, 0.f};
     float o[8][4];
@@ -766,6 +889,8 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
                 qb[kk][0] = pack_h2(q0, q1);
                 qb[kk][1] = pack_h2(q8, q9);
             }
+            heads_all = hg * 8 + 8 <= A.G;
+            if (Cfg::NIB && DKV_KBIAS) write_kbias(qb, gq, tq, kbt);
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 m_run[e] = -1e30f; l_run[e] = 0.f; dot_carry[e] = 0.f; e_carry[e] = 0.f;
@@ -793,7 +918,8 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
-                k_side<FMT, MODE>(st, sm, npos[u], first_seg, gq, tq, magic, qb, x[u], dvw[u]);
+                k_side<FMT, MODE>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, qb, kbt, x[u],
+                                  dvw[u]);
             }
 
             // ================= scores, online softmax =======================
@@ -801,6 +927,13 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
             int lim[NU];
 #pragma unroll
             for (int u = 0; u < NU; ++u) lim[u] = npos[u] - 4 * gq;
+            // every slot valid: no tail masks (nibble formats; a warp-uniform test)
+            bool full = false;
+            if (DKV_FULL_FAST && Cfg::NIB) {
+                full = heads_all;
+#pragma unroll
+                for (int u = 0; u < NU; ++u) full = full && npos[u] == SEG;
+            }
             float alpha[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -820,13 +953,17 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
                     }
                 }
                 float mx = -INFINITY;
+                if (!full) {
+#pragma unroll
+                    for (int u = 0; u < NU; ++u)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            v[u][i] = (head_ok[e] && i < lim[u]) ? v[u][i] : -INFINITY;
+                }
 #pragma unroll
                 for (int u = 0; u < NU; ++u)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        v[u][i] = (head_ok[e] && i < lim[u]) ? v[u][i] : -INFINITY;
-                        mx = fmaxf(mx, v[u][i]);
-                    }
+                    for (int i = 0; i < 4; ++i) mx = fmaxf(mx, v[u][i]);
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -883,8 +1020,8 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
-                v_side<FMT, MODE>(st, sm, npos[u], first_seg, gq, tq, magic, x[u], dvw[u], o, racc,
-                                  vkf_keep);
+                v_side<FMT, MODE>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, x[u], dvw[u], o,
+                                  racc, vkf_keep);
             }
 
             // PREFIX: close the group  o += W_g (v_f + R_g)
@@ -935,7 +1072,17 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
                                                     int64_t NW, const float *ws, float *out) {
     const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
     const int nvs = cv.Hkv * NHG;
-    __shared__ int64_t sh_base, sh_total;
+    const int len = clamp_len(cv, b);
+    const int ub = units_of(cv.fmt, cv.kf, len);
+    float *dst = out + ((int64_t)b * Hq + h) * D;
+    if (ub == 0) {                      // uniform over the block
+        dst[c] = 0.f;
+        return;
+    }
+    const int kvh = h / G, hl = h % G, hg = hl >> 3, j = hl & 7;
+    const int vsl = kvh * NHG + hg;
+    // the warps whose unit ranges touch this sequence: found once per block
+    __shared__ int64_t sh_w0, sh_w1, sh_total;
     if (threadIdx.x < 32) {
         int bb;
         int64_t bdummy;
@@ -950,29 +1097,27 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
             mine += u;
         }
         if (threadIdx.x == 0) {
-            sh_base = mine;
+            const int64_t xs = mine + (int64_t)vsl * ub, xe = xs + ub;
+            sh_w0 = warp_of(xs, NW, total);
+            sh_w1 = warp_of(xe - 1, NW, total);
             sh_total = total;
         }
     }
     __syncthreads();
-    const int len = clamp_len(cv, b);
-    const int ub = units_of(cv.fmt, cv.kf, len);
-    float *dst = out + ((int64_t)b * Hq + h) * D;
-    if (ub == 0) { dst[c] = 0.f; return; }
-    const int kvh = h / G, hl = h % G, hg = hl >> 3, j = hl & 7;
-    const int vsl = kvh * NHG + hg;
     const int64_t vseq = (int64_t)b * nvs + vsl;
-    const int64_t T = sh_total;
-    const int64_t xs = sh_base + (int64_t)vsl * ub, xe = xs + ub;
-    const int64_t w0 = warp_of(xs, NW, T), w1 = warp_of(xe - 1, NW, T);
+    const int64_t T = sh_total, w0 = sh_w0, w1 = sh_w1;
+    // with at least one unit per warp every range is non-empty; otherwise
+    // skip the warps that own no unit (they wrote no record)
+    const bool dense = T >= NW;
     float M = -INFINITY;
     for (int64_t w = w0; w <= w1; ++w) {
-        if (range_start(w, NW, T) >= range_start(w + 1, NW, T)) continue;
+        if (!dense && range_start(w, NW, T) >= range_start(w + 1, NW, T)) continue;
         M = fmaxf(M, ws[(w + vseq) * PARTIAL_FLOATS + j]);
     }
     float L = 0.f, O = 0.f;
+#pragma unroll 4
     for (int64_t w = w0; w <= w1; ++w) {
-        if (range_start(w, NW, T) >= range_start(w + 1, NW, T)) continue;
+        if (!dense && range_start(w, NW, T) >= range_start(w + 1, NW, T)) continue;
         const float *rec = ws + (w + vseq) * PARTIAL_FLOATS;
         const float sc = exp2f(rec[j] - M);
         L += rec[8 + j] * sc;

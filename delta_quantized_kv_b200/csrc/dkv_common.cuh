@@ -160,6 +160,17 @@ __device__ inline void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D = A * B + C with the accumulator input C in other registers than D.
+__device__ inline void mma16816c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                 uint32_t b0, uint32_t b1, float c0, float c1, float c2, float c3) {
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%11,%12,%13};\n"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2),
+          "f"(c3));
+}
+
 // The fp16 bit pattern of 1024.0 in both halves, as a register value the
 // compiler cannot fold: OR-ing a nibble into it needs the mask as the one
 // immediate operand of a single LOP3 and this value in a register.
@@ -168,6 +179,22 @@ __device__ inline uint32_t magic_1024x2() {
     asm volatile("mov.b32 %0, 0x64006400;\n" : "=r"(r));
     return r;
 }
+// fp16 64.0 in both halves: its ulp is 1/16, so a nibble OR-ed into mantissa
+// bits 4-7 reads as 64 + n exactly.
+__device__ inline uint32_t magic_64x2() {
+    uint32_t r;
+    asm volatile("mov.b32 %0, 0x54005400;\n" : "=r"(r));
+    return r;
+}
+
+// Biased dequantisation: one LOP3 per fp16x2 pair, no arithmetic.  The pairs
+// read 1024 + n (nibbles at bits 0-3 / 16-19, over the 1024 magic) and 64 + n
+// (bits 4-7 / 20-23, over the 64 magic); the callers remove the biases
+// 1032 = 1024 + 8 and 72 = 64 + 8 inside the tensor-core products.
+__device__ inline void dq_word_biased(uint32_t w, uint32_t m1024, uint32_t m64, uint32_t &p0,
+                                      uint32_t &p1, uint32_t &p2, uint32_t &p3);
+__device__ inline void dq_pair_biased(uint32_t w, uint32_t m1024, uint32_t m64, uint32_t &lo,
+                                      uint32_t &hi);
 // (a & MASK) | c in one LOP3 (LUT 0xEA).
 template <uint32_t MASK>
 __device__ inline uint32_t and_or(uint32_t a, uint32_t c) {
@@ -181,29 +208,45 @@ __device__ inline uint32_t hsub2_1032(uint32_t a) {
     asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(0x64086408u));
     return d;
 }
-__device__ inline uint32_t hfma2_div16_sub72(uint32_t a) {
+__device__ inline uint32_t hsub2_72(uint32_t a) {
     uint32_t d;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(0x2C002C00u), "r"(0xD480D480u));
+    asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(0x54805480u));
     return d;
 }
 
-// Dequantise the 4 nibble pairs of one 32-bit word (pairs (bits 0-3,16-19),
-// (4-7,20-23), (8-11,24-27), (12-15,28-31)) to exact fp16x2 values code - 8:
-// (1024 + n) - 1032 for the low nibbles, (1024 + 16 n) / 16 - 72 for the high.
-__device__ inline void dq_word(uint32_t w, uint32_t magic, uint32_t &p0, uint32_t &p1,
-                               uint32_t &p2, uint32_t &p3) {
+__device__ inline void dq_word_biased(uint32_t w, uint32_t m1024, uint32_t m64, uint32_t &p0,
+                                      uint32_t &p1, uint32_t &p2, uint32_t &p3) {
     const uint32_t w8 = w >> 8;
-    p0 = hsub2_1032(and_or<0x000F000Fu>(w, magic));
-    p1 = hfma2_div16_sub72(and_or<0x00F000F0u>(w, magic));
-    p2 = hsub2_1032(and_or<0x000F000Fu>(w8, magic));
-    p3 = hfma2_div16_sub72(and_or<0x00F000F0u>(w8, magic));
+    p0 = and_or<0x000F000Fu>(w, m1024);
+    p1 = and_or<0x00F000F0u>(w, m64);
+    p2 = and_or<0x000F000Fu>(w8, m1024);
+    p3 = and_or<0x00F000F0u>(w8, m64);
+}
+__device__ inline void dq_pair_biased(uint32_t w, uint32_t m1024, uint32_t m64, uint32_t &lo,
+                                      uint32_t &hi) {
+    lo = and_or<0x000F000Fu>(w, m1024);
+    hi = and_or<0x00F000F0u>(w, m64);
+}
+
+// Exact dequantisation of the 4 nibble pairs of one 32-bit word (pairs (bits
+// 0-3,16-19), (4-7,20-23), (8-11,24-27), (12-15,28-31)) to fp16x2 values
+// code - 8: (1024 + n) - 1032 for the low nibbles, (64 + n) - 72 for the high.
+__device__ inline void dq_word(uint32_t w, uint32_t m1024, uint32_t m64, uint32_t &p0,
+                               uint32_t &p1, uint32_t &p2, uint32_t &p3) {
+    dq_word_biased(w, m1024, m64, p0, p1, p2, p3);
+    p0 = hsub2_1032(p0);
+    p1 = hsub2_72(p1);
+    p2 = hsub2_1032(p2);
+    p3 = hsub2_72(p3);
 }
 
 // The low-nibble pair (bits 0-3, 16-19) and the high-nibble pair (bits 4-7,
 // 20-23) of one 32-bit word as exact fp16x2 values code - 8.
-__device__ inline void dq_pair(uint32_t w, uint32_t magic, uint32_t &lo, uint32_t &hi) {
-    lo = hsub2_1032(and_or<0x000F000Fu>(w, magic));
-    hi = hfma2_div16_sub72(and_or<0x00F000F0u>(w, magic));
+__device__ inline void dq_pair(uint32_t w, uint32_t m1024, uint32_t m64, uint32_t &lo,
+                               uint32_t &hi) {
+    dq_pair_biased(w, m1024, m64, lo, hi);
+    lo = hsub2_1032(lo);
+    hi = hsub2_72(hi);
 }
 
 }  // namespace dkv

@@ -217,18 +217,25 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
 
     // The last block to finish publishes the new lengths and flips the state
     // slot; every block has read seq_len and the old state before it arrives.
+    __shared__ int last;
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        unsigned total = gridDim.x * gridDim.y * gridDim.z;
-        unsigned prev = atomicAdd(reinterpret_cast<unsigned *>(cv.header + 1), 1u);
-        if (prev == total - 1) {
-            __threadfence();
-            for (int bb = 0; bb < cv.B; ++bb) {
-                int s0, nn;
-                encode_range(a, bb, s0, nn);
-                if (nn >= 0) cv.seqlen[bb] = s0 + nn;
-            }
+        const unsigned total = gridDim.x * gridDim.y * gridDim.z;
+        const unsigned prev = atomicAdd(reinterpret_cast<unsigned *>(cv.header + 1), 1u);
+        last = prev == total - 1;
+    }
+    __syncthreads();
+    if (last) {
+        __threadfence();
+        // one thread per batch entry: each reads and then writes its own seq_len
+        for (int bb = threadIdx.x; bb < cv.B; bb += blockDim.x) {
+            int s0, nn;
+            encode_range(a, bb, s0, nn);
+            if (nn >= 0) cv.seqlen[bb] = s0 + nn;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
             cv.header[2] ^= 1;
             cv.header[1] = 0;
             __threadfence();
