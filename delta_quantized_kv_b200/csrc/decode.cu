@@ -63,27 +63,6 @@ constexpr int WARPS = DKV_WARPS;             // warps per CTA (independent pipel
 #ifndef DKV_NIB_MINB
 #define DKV_NIB_MINB 3
 #endif
-// Nibble formats with kf <= 32: remove the dequantisation biases inside the
-// K-side MMAs (accumulator input) / the V-side MMAs (one extra MMA per tile);
-// build the V-side B fragments with one fp16x2 multiply.
-#ifndef DKV_KBIAS
-#define DKV_KBIAS 0
-#endif
-#ifndef DKV_VBIAS
-#define DKV_VBIAS 0
-#endif
-#ifndef DKV_HMUL_B
-#define DKV_HMUL_B 1
-#endif
-// Delta, kf <= 32: the keyframe row's V contribution as an fp32 rank-1 update
-// (v_f times the group's total weight) instead of an fp16 hi + lo pair of MMAs.
-#ifndef DKV_KF_FFMA
-#define DKV_KF_FFMA 1
-#endif
-// Nibble formats: skip the tail masks of stages whose units are all full.
-#ifndef DKV_FULL_FAST
-#define DKV_FULL_FAST 0
-#endif
 
 // Per (format, mode): units per stage, stage bytes, stages per warp, CTAs/SM.
 // A unit is one keyframe group (delta, kf <= 32), one 32-position segment of
@@ -101,16 +80,12 @@ template <int FMT, int MODE> struct KCfg {
 // aligned; the offsets follow from NS so no region can overlap another.
 template <int FMT, int MODE> struct SmemMap {
     static constexpr int NS = KCfg<FMT, MODE>::NS, STAGE = KCfg<FMT, MODE>::STAGE;
-    static constexpr int KBT = 256 + 32;      // per warp: K-side bias table, keyframe terms
     static constexpr int BAR_OFF = 0;
     static constexpr int META_OFF = ((BAR_OFF + 8 * WARPS * NS) + 15) / 16 * 16;
-    static constexpr int KBT_OFF = ((META_OFF + 16 * WARPS * NS) + 15) / 16 * 16;
-    static constexpr int STAGE_OFF = ((KBT_OFF + KBT * WARPS) + 127) / 128 * 128;
+    static constexpr int STAGE_OFF = ((META_OFF + 16 * WARPS * NS) + 127) / 128 * 128;
     static constexpr int BYTES = STAGE_OFF + WARPS * NS * STAGE;
     static_assert(META_OFF >= BAR_OFF + 8 * WARPS * NS, "barriers overlap descriptors");
-    static_assert(KBT_OFF >= META_OFF + 16 * WARPS * NS, "descriptors overlap the bias tables");
-    static_assert(STAGE_OFF >= KBT_OFF + KBT * WARPS, "bias tables overlap stages");
-    static_assert(KBT % 16 == 0, "bias table rows are 16-byte loads");
+    static_assert(STAGE_OFF >= META_OFF + 16 * WARPS * NS, "descriptors overlap stages");
     static_assert(STAGE % 128 == 0, "stages must stay 128-byte aligned");
     static_assert(BYTES <= 227 * 1024, "shared memory per CTA");
 };
@@ -262,7 +237,7 @@ __device__ inline int unit_npos(const CacheView &cv, const Cursor &c, int g) {
 // For slot s (position a + s) the scale / K nibble / V nibble rows start at
 // sc0 + 16 s, kn0 + 64 s, vn0 + 64 s; keyframes at kf0 (K) and kf0 + 256 (V).
 struct StageMap {
-    int kf0, sc0, kn0, vn0;
+    int kf0, sc0, kn0, vk0, vn0;
 };
 template <int FMT, int MODE>
 __device__ inline StageMap stage_map(int kf, int64_t rec, int u) {
@@ -273,16 +248,19 @@ __device__ inline StageMap stage_map(int kf, int64_t rec, int u) {
         m.kf0 = base;
         m.sc0 = base + KF_BYTES - SC_BYTES;
         m.kn0 = base + KF_BYTES + (kf - 1) * SC_BYTES - NIB_BYTES;
+        m.vk0 = base + 256;
         m.vn0 = base + KF_BYTES + (kf - 1) * (SC_BYTES + NIB_BYTES) - NIB_BYTES;
     } else if (FMT == DKV_FMT_Q4_0) {
         m.kf0 = 0;
         m.sc0 = 512 * u;
         m.kn0 = 512 * NU + 2048 * u;
+        m.vk0 = 256;
         m.vn0 = 2560 * NU + 2048 * u;
     } else {
         m.kf0 = 0;
         m.sc0 = 512;
         m.kn0 = 1024;
+        m.vk0 = 256;
         m.vn0 = 3072;
     }
     return m;
@@ -346,9 +324,12 @@ __device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nu,
 // Decide how many units the next stage takes (the units must be consecutive
 // in one sequence), fill its descriptor and (lane 0) issue its copies; every
 // lane advances its cursor identically.
+// With one stage per warp the descriptor stays in registers (every lane
+// computes it); with more it goes to the stage's shared-memory slot.
 template <int FMT, int MODE>
-__device__ inline void next_stage(const CacheView &cv, Cursor &c, int nvs, int nhg, uint8_t *stage,
-                                  uint64_t *bar, StageMeta *meta, int lane, int fault) {
+__device__ inline StageMeta next_stage(const CacheView &cv, Cursor &c, int nvs, int nhg,
+                                       uint8_t *stage, uint64_t *bar, StageMeta *meta, int lane,
+                                       int fault) {
     constexpr int NU = KCfg<FMT, MODE>::NU;
     const int np0 = unit_npos(cv, c, c.g);
     int nu = 1, np1 = 0;
@@ -356,17 +337,18 @@ __device__ inline void next_stage(const CacheView &cv, Cursor &c, int nvs, int n
         nu = 2;
         np1 = unit_npos(cv, c, c.g + 1);
     }
+    StageMeta m;
+    m.b = c.b;
+    m.vs = c.vs;
+    m.npos = np0 | (np1 << 8);
+    m.flags = MODE == PREFIX ? ((c.seg == 0 ? 1 : 0) | (c.seg == c.nseg - 1 ? 2 : 0)) : 3;
     if (lane == 0) {
-        StageMeta m;
-        m.b = c.b;
-        m.vs = c.vs;
-        m.npos = np0 | (np1 << 8);
-        m.flags = MODE == PREFIX ? ((c.seg == 0 ? 1 : 0) | (c.seg == c.nseg - 1 ? 2 : 0)) : 3;
-        *meta = m;
+        if (KCfg<FMT, MODE>::NS > 1) *meta = m;
         issue_stage<FMT, MODE>(cv, c, nu, np0 + np1, stage, bar, fault);
     }
     cursor_next<MODE>(c, cv, nvs, nhg);
     if (nu == 2) cursor_next<MODE>(c, cv, nvs, nhg);
+    return m;
 }
 
 __device__ inline uint32_t pack_h2(float lo, float hi) {
@@ -422,53 +404,18 @@ __device__ inline float col_scan32(float (&v)[4], int lane) {
 //   n = heads; the weights reach that B layout through an 8x8 transpose
 //   (movmatrix) of the K-side accumulator layout.
 
-// K-side bias removal (nibble formats, whole groups per unit).  A low-nibble
-// channel dequantises to 1024 + n and a high-nibble channel to 64 + n, so for
-// head h and 32-channel block j
-//     sum_c (n_c - 8) q_hc = sum_c A_c q_hc - (1032 sum_low q_hc + 72 sum_high q_hc);
-// the bracket, of the fp16 q the tensor cores multiply, enters negated as the
-// accumulator input of the block's first MMA.  Per warp, a shared-memory table
-// holds it where the MMA wants it: row (tq, j) = {-B_j(2tq), -B_j(2tq+1),
-// -B_j(2tq), -B_j(2tq+1)} (16 B, one load per block), then per tq the pair
-// sum_j B_j(2tq + e) that gives the keyframe row (raw fp16 values, no bias) its
-// biases back.
-__device__ inline void write_kbias(const uint32_t (&qb)[8][2], int gq, int tq, float *tab) {
-    float part[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        // this thread's 8 channels of block j for head gq: k rows 2tq, 2tq+1
-        // (low nibbles) and 2tq+8, 2tq+9 (high nibbles) of k-steps 2j, 2j+1
-        const uint32_t l0 = qb[2 * j][0], h0 = qb[2 * j][1];
-        const uint32_t l1 = qb[2 * j + 1][0], h1 = qb[2 * j + 1][1];
-        const float sl = (h_lo(l0) + h_hi(l0)) + (h_lo(l1) + h_hi(l1));
-        const float sh = (h_lo(h0) + h_hi(h0)) + (h_lo(h1) + h_hi(h1));
-        float v = 1032.f * sl + 72.f * sh;
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        part[j] = v;                                   // B_j(head gq), every lane of quad gq
-    }
-    if (tq == 0) {
-        const int r = gq >> 1, e = gq & 1;             // head gq sits in column e of tq = r
-        float tot = 0.f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            tab[(r * 4 + j) * 4 + e] = -part[j];
-            tab[(r * 4 + j) * 4 + 2 + e] = -part[j];
-            tot += part[j];
-        }
-        tab[64 + 2 * r + e] = tot;
-    }
-    __syncwarp();
-}
-
 // K side of one unit: per-position dot products x[t][r][e] (position
 // 4g + 2t + r, head 2tq + e) and the V scales dvw[t][r] of those positions.
-template <int FMT, int MODE>
+// ZT: zero the scales of slots past the unit's end.  Needed where such a slot
+// can read bytes that are not scale rows (kf < 32: the next record's nibbles,
+// whose fp16 reading may be NaN); with kf = 32 and for Q4_0 a slot past the end
+// reads a scale row of the cache (zeroed at init, else written by the encoder)
+// or of an older stage, always finite, and the softmax mask alone handles it.
+template <int FMT, int MODE, bool ZT>
 __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, bool first_seg,
                               int gq, int tq, uint32_t m1024, uint32_t m64,
-                              const uint32_t (&qb)[8][2], const float *kbt, float (&x)[2][2][2],
+                              const uint32_t (&qb)[8][2], float (&x)[2][2][2],
                               uint32_t (&dvw)[2][2][2]) {
-    constexpr bool BIASED = KCfg<FMT, MODE>::NIB && DKV_KBIAS;
     const bool kfrow = first_seg && gq == 0;   // this thread's row 0 of tile 0 is the keyframe
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
@@ -495,43 +442,31 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
                 const uint32_t ww1[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    if (BIASED) {
-                        dq_word_biased(ww0[j], m1024, m64, a[2 * j][0], a[2 * j][2], a[2 * j + 1][0],
-                                       a[2 * j + 1][2]);
-                        dq_word_biased(ww1[j], m1024, m64, a[2 * j][1], a[2 * j][3], a[2 * j + 1][1],
-                                       a[2 * j + 1][3]);
-                    } else {
-                        dq_word(ww0[j], m1024, m64, a[2 * j][0], a[2 * j][2], a[2 * j + 1][0],
-                                a[2 * j + 1][2]);
-                        dq_word(ww1[j], m1024, m64, a[2 * j][1], a[2 * j][3], a[2 * j + 1][1],
-                                a[2 * j + 1][3]);
-                    }
+                    dq_word(ww0[j], m1024, m64, a[2 * j][0], a[2 * j][2], a[2 * j + 1][0],
+                            a[2 * j + 1][2]);
+                    dq_word(ww1[j], m1024, m64, a[2 * j][1], a[2 * j][3], a[2 * j + 1][1],
+                            a[2 * j + 1][3]);
                 }
             }
-            if (FMT == DKV_FMT_DELTA && t == 0 && first_seg) {
+            if (FMT == DKV_FMT_DELTA && t == 0 && first_seg && kfrow) {
                 // position 0 is the keyframe: its fp16 values fill rows g = 0
+                // (loaded by those lanes only, straight into the A fragment)
                 const uint8_t *kp = st + sm.kf0 + 64 * tq;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const uint4 v = *reinterpret_cast<const uint4 *>(kp + 16 * q4);
-                    a[2 * q4][0] = kfrow ? v.x : a[2 * q4][0];
-                    a[2 * q4][2] = kfrow ? v.y : a[2 * q4][2];
-                    a[2 * q4 + 1][0] = kfrow ? v.z : a[2 * q4 + 1][0];
-                    a[2 * q4 + 1][2] = kfrow ? v.w : a[2 * q4 + 1][2];
+                    a[2 * q4][0] = v.x;
+                    a[2 * q4][2] = v.y;
+                    a[2 * q4 + 1][0] = v.z;
+                    a[2 * q4 + 1][2] = v.w;
                 }
             }
             float acc[4][4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                if (BIASED) {
-                    const float4 c = *reinterpret_cast<const float4 *>(kbt + (tq * 4 + j) * 4);
-                    mma16816c(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
-                              qb[2 * j][0], qb[2 * j][1], c.x, c.y, c.z, c.w);
-                } else {
-                    acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-                    mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
-                             qb[2 * j][0], qb[2 * j][1]);
-                }
+                acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+                mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
+                         qb[2 * j][0], qb[2 * j][1]);
                 mma16816(acc[j], a[2 * j + 1][0], a[2 * j + 1][1], a[2 * j + 1][2],
                          a[2 * j + 1][3], qb[2 * j + 1][0], qb[2 * j + 1][1]);
             }
@@ -539,15 +474,12 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
             uint4 s0 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + p0 * SC_BYTES);
             uint4 s1 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + (p0 + 1) * SC_BYTES);
             if (FMT == DKV_FMT_DELTA && t == 0 && kfrow) {
-                // keyframe: unit K weights; V weight 1 when its row goes through
-                // the MMA (SUFFIX), else 0 (added apart)
+                // keyframe: unit K weights; no V weight in the MMAs (its V
+                // contribution is added apart, in fp32)
                 s0.x = s0.y = 0x3C003C00u;
-                s0.z = s0.w = (MODE == SUFFIX && !DKV_KF_FFMA) ? 0x3C003C00u : 0u;
+                s0.z = s0.w = 0u;
             }
-            // slots past the end of the unit hold stale bytes (possibly NaN
-            // patterns): zero their K and V scales so they add nothing to the
-            // prefix sums and carry no V weight
-            if (!DKV_FULL_FAST || !KCfg<FMT, MODE>::NIB || npos < SEG) {
+            if (ZT) {
                 if (p0 >= npos) s0 = make_uint4(0u, 0u, 0u, 0u);
                 if (p0 + 1 >= npos) s1 = make_uint4(0u, 0u, 0u, 0u);
             }
@@ -555,11 +487,7 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
             dvw[t][1][0] = s1.z; dvw[t][1][1] = s1.w;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                float x0;
-                if (BIASED && FMT == DKV_FMT_DELTA && t == 0)
-                    x0 = fmaf(acc[0][e], h_lo(s0.x), kfrow ? kbt[64 + 2 * tq + e] : 0.f);
-                else
-                    x0 = acc[0][e] * h_lo(s0.x);
+                float x0 = acc[0][e] * h_lo(s0.x);
                 x0 = fmaf(acc[1][e], h_hi(s0.x), x0);
                 x0 = fmaf(acc[2][e], h_lo(s0.y), x0);
                 x[t][0][e] = fmaf(acc[3][e], h_hi(s0.y), x0);
@@ -579,12 +507,10 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
                               int gq, int tq, uint32_t m1024, uint32_t m64,
                               const float (&w)[2][2][2], const uint32_t (&dvw)[2][2][2],
                               float (&o)[8][4], float (&racc)[8][4], uint32_t (&vkf_keep)[8]) {
-    constexpr bool VBIASED = KCfg<FMT, MODE>::NIB && DKV_VBIAS;
-    const bool kfrow = first_seg && gq == 0;
     uint32_t vkf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     if (FMT == DKV_FMT_DELTA && first_seg) {
-        const uint4 v0 = *reinterpret_cast<const uint4 *>(st + sm.kf0 + 256 + 32 * gq);
-        const uint4 v1 = *reinterpret_cast<const uint4 *>(st + sm.kf0 + 256 + 32 * gq + 16);
+        const uint4 v0 = *reinterpret_cast<const uint4 *>(st + sm.vk0 + 32 * gq);
+        const uint4 v1 = *reinterpret_cast<const uint4 *>(st + sm.vk0 + 32 * gq + 16);
         vkf[0] = v0.x; vkf[1] = v0.y; vkf[2] = v0.z; vkf[3] = v0.w;
         vkf[4] = v1.x; vkf[5] = v1.y; vkf[6] = v1.z; vkf[7] = v1.w;
         if (MODE == PREFIX) {
@@ -626,77 +552,38 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
         const uint2 wP1 = *reinterpret_cast<const uint2 *>(vb + NIB_BYTES);
         const uint2 wP2 = *reinterpret_cast<const uint2 *>(vb + 4 * NIB_BYTES);
         const uint2 wP3 = *reinterpret_cast<const uint2 *>(vb + 5 * NIB_BYTES);
-        auto codes = [&](int mt, bool biased, uint32_t &a0, uint32_t &a1, uint32_t &a2,
-                         uint32_t &a3) {
+        // A fragment of m-tile mt: exact code - 8 of channels 16mt + g (rows g)
+        // and 16mt + g + 8 (rows g + 8), k pairs (pos 8tq+2t, +4) | (+1, +5)
+        auto codes = [&](int mt, uint32_t &a0, uint32_t &a1, uint32_t &a2, uint32_t &a3) {
             const int i = mt & 3;
             const uint32_t sel = (uint32_t)(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
-            // k pairs: (pos 8tq+2t, +4) | (8tq+2t+1, +5)
             const uint32_t m01 = prmt(mt < 4 ? wP0.x : wP0.y, mt < 4 ? wP2.x : wP2.y, sel);
             const uint32_t m23 = prmt(mt < 4 ? wP1.x : wP1.y, mt < 4 ? wP3.x : wP3.y, sel);
-            if (biased) {
-                dq_pair_biased(m01, m1024, m64, a0, a1);
-                dq_pair_biased(m23, m1024, m64, a2, a3);
-            } else {
-                dq_pair(m01, m1024, m64, a0, a1);
-                dq_pair(m23, m1024, m64, a2, a3);
-            }
+            dq_pair(m01, m1024, m64, a0, a1);
+            dq_pair(m23, m1024, m64, a2, a3);
         };
         if (MODE != PREFIX) {
-            constexpr bool VB = VBIASED;
-            // B fragments (k = positions, n = head g) of block j: the 8x8
-            // transpose of the weights times block j's V scale, in fp16 (one
-            // token per row for Q4_0; for the delta format the keyframe row gets
-            // an extra lo fragment below).
+            // B fragments (k = positions, n = head g) of block j: the weights
+            // packed to fp16 once, times block j's V scale in one fp16x2
+            // multiply, then the 8x8 transpose into the B layout
             const uint32_t wp0 = pack_h2(w[t][0][0], w[t][0][1]);
             const uint32_t wp1 = pack_h2(w[t][1][0], w[t][1][1]);
             auto make_b = [&](int j, uint32_t (&b)[2]) {
                 const uint32_t u0 = dvw[t][0][j >> 1], u1 = dvw[t][1][j >> 1];
-                if (DKV_HMUL_B) {
-                    const __half2 d0 = (j & 1) ? __high2half2(u32_as_h2(u0)) : __low2half2(u32_as_h2(u0));
-                    const __half2 d1 = (j & 1) ? __high2half2(u32_as_h2(u1)) : __low2half2(u32_as_h2(u1));
-                    b[0] = movm_t(h2_as_u32(__hmul2(u32_as_h2(wp0), d0)));
-                    b[1] = movm_t(h2_as_u32(__hmul2(u32_as_h2(wp1), d1)));
-                } else {
-                    const float d0 = (j & 1) ? h_hi(u0) : h_lo(u0);
-                    const float d1 = (j & 1) ? h_hi(u1) : h_lo(u1);
-                    b[0] = movm_t(pack_h2(w[t][0][0] * d0, w[t][0][1] * d0));
-                    b[1] = movm_t(pack_h2(w[t][1][0] * d1, w[t][1][1] * d1));
-                }
+                const __half2 d0 = (j & 1) ? __high2half2(u32_as_h2(u0)) : __low2half2(u32_as_h2(u0));
+                const __half2 d1 = (j & 1) ? __high2half2(u32_as_h2(u1)) : __low2half2(u32_as_h2(u1));
+                b[0] = movm_t(h2_as_u32(__hmul2(u32_as_h2(wp0), d0)));
+                b[1] = movm_t(h2_as_u32(__hmul2(u32_as_h2(wp1), d1)));
             };
-            // delta: the keyframe row's weight (the group total, scale 1) as fp16
-            // hi (in the B fragment) + lo (this extra fragment, nonzero only at
-            // the keyframe's k slot)
-            constexpr bool KF = FMT == DKV_FMT_DELTA && !DKV_KF_FFMA;
-            uint32_t bk = 0u;
-            if (KF && t == 0) {
-                const float r0 = w[0][0][0] - h_lo(wp0);
-                const float r1 = w[0][0][1] - h_hi(wp0);
-                bk = movm_t(kfrow ? pack_h2(r0, r1) : 0u);
-            }
-            // bias removal: A rows -1032 (rows g: low nibbles) and -72 (rows g+8:
-            // high nibbles) against the same B fragments; the keyframe slot
-            // (k = 2tq of t = 0, tq = 0) holds raw fp16 values and no bias
-            const bool kslot = KF && t == 0 && tq == 0;
-            const uint32_t cl = 0xE408E408u, ch = 0xD480D480u;
-            const uint32_t cl0 = kslot ? 0xE4080000u : cl;
-            const uint32_t ch0 = kslot ? 0xD4800000u : ch;
-            const uint32_t sel0 = kslot ? 0x3254u : 0x3210u;
-            const uint32_t sel1 = kslot ? 0x3276u : 0x3210u;
             uint32_t bp[2];
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 uint32_t a0, a1, a2, a3;
-                codes(mt, VB, a0, a1, a2, a3);
-                if (KF && t == 0) {
-                    a0 = prmt(a0, vkf[mt], sel0);
-                    a1 = prmt(a1, vkf[mt], sel1);
-                }
+                codes(mt, a0, a1, a2, a3);
                 if ((mt & 1) == 0) make_b(mt >> 1, bp);
                 mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
-                if (VB) mma16816(o[mt], cl0, ch0, cl, ch, bp[0], bp[1]);
-                if (KF && t == 0) mma16816(o[mt], a0, a1, a2, a3, bk, 0u);
             }
-            if (FMT == DKV_FMT_DELTA && DKV_KF_FFMA && t == 0) {
+            if (FMT == DKV_FMT_DELTA && t == 0) {
                 // keyframe row: o += v_f * (the group's total weight), in fp32;
                 // the total of heads 2tq + e sits in w[0][0][e] of lane tq (g = 0)
                 const float S0 = __shfl_sync(0xffffffffu, w[0][0][0], tq);
@@ -729,7 +616,7 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 uint32_t a0, a1, a2, a3;
-                codes(mt, false, a0, a1, a2, a3);
+                codes(mt, a0, a1, a2, a3);
                 const int j = mt >> 1;
                 if ((mt & 1) == 0) make_b(j, bp, bl);
                 mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
@@ -748,7 +635,7 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
     }
 }
 
-template <int FMT, int MODE>
+template <int FMT, int MODE, bool ZT>
 __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_kernel(SplitArgs A) {
     using Cfg = KCfg<FMT, MODE>;
     constexpr int NS = Cfg::NS, STAGE = Cfg::STAGE, NU = Cfg::NU;
@@ -795,10 +682,12 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
     // prologue: fill the ring
     uint32_t phase = 0;                 // bit s = parity to wait for on stage s
     int issued = 0, consumed = 0;
+    StageMeta pend{};                   // NS == 1: the issued stage's descriptor
 #pragma unroll 1
     for (int s = 0; s < NS; ++s) {
         if (ic.valid()) {
-            next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + s * STAGE, mybar + s, mymeta + s, lane, A.fault);
+            pend = next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + s * STAGE, mybar + s,
+                                         mymeta + s, lane, A.fault);
             ++issued;
         }
     }
@@ -809,8 +698,6 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
     // per-sequence state (heads 2*tq + e of the current head group)
     int cur_b = -1, cur_vs = -1;
     uint32_t qb[8][2];                  // B fragments of q (column = head gq)
-    float *kbt = reinterpret_cast<float *>(smem + Map::KBT_OFF + warp * Map::KBT);
-    bool heads_all = false;             // all 8 heads of the head group exist
     bool head_ok[2] = {false, false};
     float m_run[2] = {-1e30f, -1e30f}, l_run[2] = {0.f, 0.f};
     float o[8][4];
@@ -856,18 +743,19 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
     while (consumed < issued) {
         // ---- wait for the stage -------------------------------------------
         const uint8_t *st = mystages + stage_i * STAGE;
-        if (!dead) {
-            if (!mbar_wait_bounded(mybar + stage_i, (phase >> stage_i) & 1)) {
-                dead = true;
-                if (lane == 0) set_status(cv.header, DKV_DEV_TIMEOUT);
-            }
+        if (!mbar_wait_bounded(mybar + stage_i, (phase >> stage_i) & 1)) {
+            dead = true;
+            if (lane == 0) set_status(cv.header, DKV_DEV_TIMEOUT);
         }
+        // a warp that gave up leaves the loop with this stage's copies (and any
+        // later ones) in flight; they are waited for below
         dead = __any_sync(0xffffffffu, dead);
+        if (dead) break;
         phase ^= 1u << stage_i;
-        const StageMeta meta = mymeta[stage_i];
+        const StageMeta meta = NS == 1 ? pend : mymeta[stage_i];
 
         // ---- sequence change: flush, load q --------------------------------
-        if (!dead && (meta.b != cur_b || meta.vs != cur_vs)) {
+        if (meta.b != cur_b || meta.vs != cur_vs) {
             if (cur_b >= 0) flush();
             cur_b = meta.b; cur_vs = meta.vs;
             const int kvh = meta.vs / A.NHG, hg = meta.vs % A.NHG;
@@ -889,8 +777,6 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
                 qb[kk][0] = pack_h2(q0, q1);
                 qb[kk][1] = pack_h2(q8, q9);
             }
-            heads_all = hg * 8 + 8 <= A.G;
-            if (Cfg::NIB && DKV_KBIAS) write_kbias(qb, gq, tq, kbt);
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 m_run[e] = -1e30f; l_run[e] = 0.f; dot_carry[e] = 0.f; e_carry[e] = 0.f;
@@ -901,7 +787,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
                 for (int j = 0; j < 4; ++j) { o[i][j] = 0.f; racc[i][j] = 0.f; }
         }
 
-        if (!dead) {
+        {
             int npos[NU];
 #pragma unroll
             for (int u = 0; u < NU; ++u) npos[u] = (meta.npos >> (8 * u)) & 0xff;
@@ -918,8 +804,8 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
-                k_side<FMT, MODE>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, qb, kbt, x[u],
-                                  dvw[u]);
+                k_side<FMT, MODE, ZT>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, qb, x[u],
+                                      dvw[u]);
             }
 
             // ================= scores, online softmax =======================
@@ -927,13 +813,6 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
             int lim[NU];
 #pragma unroll
             for (int u = 0; u < NU; ++u) lim[u] = npos[u] - 4 * gq;
-            // every slot valid: no tail masks (nibble formats; a warp-uniform test)
-            bool full = false;
-            if (DKV_FULL_FAST && Cfg::NIB) {
-                full = heads_all;
-#pragma unroll
-                for (int u = 0; u < NU; ++u) full = full && npos[u] == SEG;
-            }
             float alpha[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -953,17 +832,13 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
                     }
                 }
                 float mx = -INFINITY;
-                if (!full) {
-#pragma unroll
-                    for (int u = 0; u < NU; ++u)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            v[u][i] = (head_ok[e] && i < lim[u]) ? v[u][i] : -INFINITY;
-                }
 #pragma unroll
                 for (int u = 0; u < NU; ++u)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) mx = fmaxf(mx, v[u][i]);
+                    for (int i = 0; i < 4; ++i) {
+                        v[u][i] = (head_ok[e] && i < lim[u]) ? v[u][i] : -INFINITY;
+                        mx = fmaxf(mx, v[u][i]);
+                    }
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -1042,10 +917,10 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
         // ---- release the stage and refill it ------------------------------
         __syncwarp();
         ++consumed;
-        if (ic.valid() && !dead) {
+        if (ic.valid()) {
             if (lane == 0) fence_proxy_async();
-            next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + stage_i * STAGE, mybar + stage_i,
-                                  mymeta + stage_i, lane, A.fault);
+            pend = next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + stage_i * STAGE,
+                                         mybar + stage_i, mymeta + stage_i, lane, A.fault);
             ++issued;
         }
         stage_i = (stage_i + 1 == NS) ? 0 : stage_i + 1;
@@ -1134,7 +1009,7 @@ static size_t split_smem() {
     return (size_t)SmemMap<FMT, MODE>::BYTES;
 }
 
-template <int FMT, int MODE>
+template <int FMT, int MODE, bool ZT>
 static cudaError_t geom_for(SplitGeom *g) {
     static int cached_dev = -1, cached_ctas = 0;
     int dev;
@@ -1142,11 +1017,11 @@ static cudaError_t geom_for(SplitGeom *g) {
     if (e != cudaSuccess) return e;
     if (dev != cached_dev) {
         const size_t sm = split_smem<FMT, MODE>();
-        e = cudaFuncSetAttribute(split_kernel<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sm);
+        e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
         int per_sm = 0, nsm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_kernel<FMT, MODE>,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_kernel<FMT, MODE, ZT>,
                                                           WARPS * 32, sm);
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -1159,21 +1034,27 @@ static cudaError_t geom_for(SplitGeom *g) {
     return cudaSuccess;
 }
 
+// The kernel instance for a cache: format, mode (kf <= 32: whole groups per
+// unit; kf > 32: 32-position segments) and whether tail slots need their
+// scales zeroed (kf != 32 for the delta format).  The merge derives the warp
+// count from the same instance the split launched.
 cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g) {
     (void)batch;
     if (fmt == DKV_FMT_DELTA) {
-        return kf <= SEG ? geom_for<DKV_FMT_DELTA, SUFFIX>(g) : geom_for<DKV_FMT_DELTA, PREFIX>(g);
+        if (kf == SEG) return geom_for<DKV_FMT_DELTA, SUFFIX, false>(g);
+        return kf < SEG ? geom_for<DKV_FMT_DELTA, SUFFIX, true>(g)
+                        : geom_for<DKV_FMT_DELTA, PREFIX, true>(g);
     }
-    if (fmt == DKV_FMT_Q4_0) return geom_for<DKV_FMT_Q4_0, PLAIN>(g);
-    return geom_for<DKV_FMT_FP16, PLAIN>(g);
+    if (fmt == DKV_FMT_Q4_0) return geom_for<DKV_FMT_Q4_0, PLAIN, false>(g);
+    return geom_for<DKV_FMT_FP16, PLAIN, false>(g);
 }
 
-template <int FMT, int MODE>
+template <int FMT, int MODE, bool ZT>
 static cudaError_t launch_split_t(const SplitArgs &a, cudaStream_t st) {
     SplitGeom g;
-    cudaError_t e = geom_for<FMT, MODE>(&g);
+    cudaError_t e = geom_for<FMT, MODE, ZT>(&g);
     if (e != cudaSuccess) return e;
-    split_kernel<FMT, MODE><<<g.ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
+    split_kernel<FMT, MODE, ZT><<<g.ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
     return cudaGetLastError();
 }
 
@@ -1192,11 +1073,12 @@ cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
     a.ws = ws;
     if (cv.fmt == DKV_FMT_DELTA) {
-        return cv.kf <= SEG ? launch_split_t<DKV_FMT_DELTA, SUFFIX>(a, st)
-                            : launch_split_t<DKV_FMT_DELTA, PREFIX>(a, st);
+        if (cv.kf == SEG) return launch_split_t<DKV_FMT_DELTA, SUFFIX, false>(a, st);
+        return cv.kf < SEG ? launch_split_t<DKV_FMT_DELTA, SUFFIX, true>(a, st)
+                           : launch_split_t<DKV_FMT_DELTA, PREFIX, true>(a, st);
     }
-    if (cv.fmt == DKV_FMT_Q4_0) return launch_split_t<DKV_FMT_Q4_0, PLAIN>(a, st);
-    return launch_split_t<DKV_FMT_FP16, PLAIN>(a, st);
+    if (cv.fmt == DKV_FMT_Q4_0) return launch_split_t<DKV_FMT_Q4_0, PLAIN, false>(a, st);
+    return launch_split_t<DKV_FMT_FP16, PLAIN, false>(a, st);
 }
 
 cudaError_t launch_merge(const CacheView &cv, int Hq, float *out, const float *ws, cudaStream_t st) {

@@ -160,17 +160,6 @@ __device__ inline void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// D = A * B + C with the accumulator input C in other registers than D.
-__device__ inline void mma16816c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                 uint32_t b0, uint32_t b1, float c0, float c1, float c2, float c3) {
-    asm(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%10,%11,%12,%13};\n"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2),
-          "f"(c3));
-}
-
 // The fp16 bit pattern of 1024.0 in both halves, as a register value the
 // compiler cannot fold: OR-ing a nibble into it needs the mask as the one
 // immediate operand of a single LOP3 and this value in a register.
@@ -187,10 +176,9 @@ __device__ inline uint32_t magic_64x2() {
     return r;
 }
 
-// Biased dequantisation: one LOP3 per fp16x2 pair, no arithmetic.  The pairs
-// read 1024 + n (nibbles at bits 0-3 / 16-19, over the 1024 magic) and 64 + n
-// (bits 4-7 / 20-23, over the 64 magic); the callers remove the biases
-// 1032 = 1024 + 8 and 72 = 64 + 8 inside the tensor-core products.
+// Biased dequantisation: one LOP3 per fp16x2 pair.  The pairs read 1024 + n
+// (nibbles at bits 0-3 / 16-19, over the 1024 magic) and 64 + n (bits 4-7 /
+// 20-23, over the 64 magic); dq_word / dq_pair subtract 1032 and 72.
 __device__ inline void dq_word_biased(uint32_t w, uint32_t m1024, uint32_t m64, uint32_t &p0,
                                       uint32_t &p1, uint32_t &p2, uint32_t &p3);
 __device__ inline void dq_pair_biased(uint32_t w, uint32_t m1024, uint32_t m64, uint32_t &lo,
