@@ -252,7 +252,7 @@ class Cache:
             nb = dkv_decode_workspace_bytes(self.desc, n_q_heads)
             if nb == 0:
                 raise DkvError(DKV_ECUDA, "dkv_decode_workspace_bytes")
-            self._ws = torch.empty(nb // 4 + 64, dtype=torch.float32, device=self.device)
+            self._ws = torch.zeros(nb // 4 + 64, dtype=torch.float32, device=self.device)
             self._ws_heads = n_q_heads
         return self._ws
 

@@ -984,19 +984,40 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
     // with at least one unit per warp every range is non-empty; otherwise
     // skip the warps that own no unit (they wrote no record)
     const bool dense = T >= NW;
+    // the records are read in batches of 8 independent loads (one memory
+    // round trip per batch); the arithmetic runs over w in order, as written
+    constexpr int BATCH = 8;
+    auto has = [&](int64_t w) {
+        return w <= w1 && (dense || range_start(w, NW, T) < range_start(w + 1, NW, T));
+    };
     float M = -INFINITY;
-    for (int64_t w = w0; w <= w1; ++w) {
-        if (!dense && range_start(w, NW, T) >= range_start(w + 1, NW, T)) continue;
-        M = fmaxf(M, ws[(w + vseq) * PARTIAL_FLOATS + j]);
+    for (int64_t w = w0; w <= w1; w += BATCH) {
+        float mv[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i)
+            mv[i] = has(w + i) ? ws[(w + i + vseq) * PARTIAL_FLOATS + j] : -INFINITY;
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) M = fmaxf(M, mv[i]);
     }
     float L = 0.f, O = 0.f;
-#pragma unroll 4
-    for (int64_t w = w0; w <= w1; ++w) {
-        if (!dense && range_start(w, NW, T) >= range_start(w + 1, NW, T)) continue;
-        const float *rec = ws + (w + vseq) * PARTIAL_FLOATS;
-        const float sc = exp2f(rec[j] - M);
-        L += rec[8 + j] * sc;
-        O += rec[16 + j * 128 + c] * sc;
+    for (int64_t w = w0; w <= w1; w += BATCH) {
+        float mv[BATCH], lv[BATCH], ov[BATCH];
+        bool ok[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            ok[i] = has(w + i);
+            const float *rec = ws + (w + i + vseq) * PARTIAL_FLOATS;
+            mv[i] = ok[i] ? rec[j] : 0.f;
+            lv[i] = ok[i] ? rec[8 + j] : 0.f;
+            ov[i] = ok[i] ? rec[16 + j * 128 + c] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            if (!ok[i]) continue;
+            const float sc = exp2f(mv[i] - M);
+            L += lv[i] * sc;
+            O += ov[i] * sc;
+        }
     }
     dst[c] = O / L;
 }
