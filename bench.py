@@ -589,6 +589,29 @@ def run_ours(args, w, rank, world, local):
             extra[fmt] = {"split_us": 1e3 * t, "bytes": nb, "gbps": nb / (t * 1e-3) / 1e9,
                           "speedup_delta_vs": t / split_avg}
             del cc
+        # the same decode through a paged cache: pages of 16 groups (512 tokens)
+        # in a shuffled pool, every record reached through the block table
+        if args.fmt == "delta":
+            cp = dkv.Cache(B, Hkv, T0, "delta", kf=w.kf, device=dev, page_groups=16, page_seed=7)
+            cp.encode(Kp, Vp)
+            wsp = cp.workspace(Hq)
+            for _ in range(3):
+                cp.decode_attn(qs[0], scale, out=out)
+            torch.cuda.synchronize()
+            a, bq = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = max(5, K)
+            a.record(stream)
+            for i in range(n):
+                dkv.dkv_decode_attn_split(cp.c, qs[i % len(qs)], qcode, Hq, scale, wsp,
+                                          wsp.numel() * 4, stream)
+            bq.record(stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(bq) / n
+            nb = kv_bytes("delta", [T0] * B, Hkv, w.kf)
+            extra["delta_paged_16_groups"] = {"split_us": 1e3 * t, "bytes": nb,
+                                              "gbps": nb / (t * 1e-3) / 1e9,
+                                              "status": cp.device_status()}
+            del cp
         # reconstruction MSE on a slice (first 2 batch entries)
         nb_ = min(2, B)
         xs = {"K": Kp[:nb_].float(), "V": Vp[:nb_].float()}

@@ -21,7 +21,7 @@ LIB_PATH = _PKG / "_lib" / "libdkv.so"
 DKV_OK, DKV_EINVAL, DKV_EALIGN, DKV_ECAPACITY, DKV_EUNSUPPORTED, DKV_ECUDA, DKV_EDEVICE = range(7)
 DKV_FMT_FP16, DKV_FMT_Q4_0, DKV_FMT_DELTA = 0, 1, 2
 DKV_F32, DKV_F16, DKV_BF16 = 0, 1, 2
-DEV_BAD_SEQLEN, DEV_CAPACITY, DEV_TIMEOUT, DEV_BAD_HEADS = 0x1, 0x2, 0x4, 0x8
+DEV_BAD_SEQLEN, DEV_CAPACITY, DEV_TIMEOUT, DEV_BAD_HEADS, DEV_BAD_PAGE = 0x1, 0x2, 0x4, 0x8, 0x10
 FORMATS = {"fp16": DKV_FMT_FP16, "q4": DKV_FMT_Q4_0, "delta": DKV_FMT_DELTA}
 
 
@@ -42,7 +42,10 @@ class dkv_cache(ctypes.Structure):
                 ("seq_stride", ctypes.c_size_t), ("rec_bytes", ctypes.c_size_t),
                 ("n_groups", ctypes.c_int32), ("reserved0", ctypes.c_int32),
                 ("off_data", ctypes.c_size_t), ("off_state", ctypes.c_size_t),
-                ("off_seqlen", ctypes.c_size_t), ("off_header", ctypes.c_size_t)]
+                ("off_seqlen", ctypes.c_size_t), ("off_header", ctypes.c_size_t),
+                ("pool", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("page_bytes", ctypes.c_size_t), ("n_pages", ctypes.c_int64),
+                ("page_groups", ctypes.c_int32), ("max_pages", ctypes.c_int32)]
 
 
 _lib = None
@@ -50,7 +53,8 @@ EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode",
            "dkv_decode_workspace_bytes", "dkv_decode_attn", "dkv_decode_attn_split",
            "dkv_decode_attn_merge", "dkv_export_canonical", "dkv_dequantize",
            "dkv_get_device_status", "dkv_status_str", "dkv_decode_attn_noalloc",
-           "dkv_debug_set_fault"]
+           "dkv_debug_set_fault", "dkv_cache_meta_bytes", "dkv_page_bytes",
+           "dkv_cache_init_paged"]
 
 
 def load():
@@ -81,6 +85,9 @@ def load():
         "dkv_status_str": ([I], ctypes.c_char_p),
         "dkv_decode_attn_noalloc": ([PC, P, I, I, F, P, P], I),
         "dkv_debug_set_fault": ([I], None),
+        "dkv_cache_meta_bytes": ([PD], S),
+        "dkv_page_bytes": ([PD, I], S),
+        "dkv_cache_init_paged": ([PD, I, P, ctypes.c_int64, P, I, P, S, PC, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -137,6 +144,25 @@ def dkv_cache_init(desc: dkv_cache_desc, dev, nbytes: int, stream=None) -> dkv_c
     out = dkv_cache()
     _check(load().dkv_cache_init(ctypes.byref(desc), _ptr(dev), nbytes, ctypes.byref(out),
                                  _stream(stream)), "dkv_cache_init")
+    return out
+
+
+def dkv_cache_meta_bytes(desc: dkv_cache_desc) -> int:
+    return load().dkv_cache_meta_bytes(ctypes.byref(desc))
+
+
+def dkv_page_bytes(desc: dkv_cache_desc, page_groups: int) -> int:
+    return load().dkv_page_bytes(ctypes.byref(desc), page_groups)
+
+
+def dkv_cache_init_paged(desc: dkv_cache_desc, page_groups: int, pool, n_pages: int,
+                         block_table, max_pages: int, meta, meta_bytes: int,
+                         stream=None) -> dkv_cache:
+    out = dkv_cache()
+    _check(load().dkv_cache_init_paged(ctypes.byref(desc), page_groups, _ptr(pool), n_pages,
+                                       _ptr(block_table), max_pages, _ptr(meta), meta_bytes,
+                                       ctypes.byref(out), _stream(stream)),
+           "dkv_cache_init_paged")
     return out
 
 
@@ -222,16 +248,43 @@ class Cache:
     """A Delta-KV (or comparator) cache in torch-allocated device memory."""
 
     def __init__(self, batch, n_kv_heads, max_ctx, fmt="delta", kf=32, head_dim=128,
-                 device="cuda", stream=None):
+                 device="cuda", stream=None, page_groups=None, n_pages=None,
+                 block_table=None, page_seed=0):
+        """page_groups: a paged cache (delta format) with pages of page_groups
+        keyframe groups; the pool holds n_pages pages (default: exactly the
+        pages every sequence needs at max_ctx) and block_table ([batch,
+        max_pages] int32, default: a seeded random assignment of distinct
+        pages) maps each sequence's groups to pages."""
         import torch
         self.desc = dkv_cache_desc(batch, n_kv_heads, head_dim, kf, max_ctx,
                                    FORMATS[fmt] if isinstance(fmt, str) else fmt)
-        nbytes = dkv_cache_bytes(self.desc)
-        if nbytes == 0:
-            raise DkvError(DKV_EINVAL, "dkv_cache_bytes")
-        self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
-        base = (self.buf.data_ptr() + 255) // 256 * 256
-        self.c = dkv_cache_init(self.desc, base, nbytes, stream)
+        if page_groups:
+            mb = dkv_cache_meta_bytes(self.desc)
+            pb = dkv_page_bytes(self.desc, page_groups)
+            if mb == 0 or pb == 0:
+                raise DkvError(DKV_EINVAL, "dkv_cache_meta_bytes / dkv_page_bytes")
+            n_groups = -(-max_ctx // kf)
+            max_pages = -(-n_groups // page_groups)
+            if n_pages is None:
+                n_pages = batch * max_pages
+            if block_table is None:
+                g = torch.Generator().manual_seed(page_seed)
+                perm = torch.randperm(n_pages, generator=g)[:batch * max_pages]
+                block_table = perm.view(batch, max_pages).to(torch.int32)
+            self.block_table = block_table.to(device=device, dtype=torch.int32).contiguous()
+            self.buf = torch.empty(mb + 256, dtype=torch.uint8, device=device)
+            self.pool = torch.empty(n_pages * pb + 256, dtype=torch.uint8, device=device)
+            base = (self.buf.data_ptr() + 255) // 256 * 256
+            pool = (self.pool.data_ptr() + 255) // 256 * 256
+            self.c = dkv_cache_init_paged(self.desc, page_groups, pool, n_pages,
+                                          self.block_table, max_pages, base, mb, stream)
+        else:
+            nbytes = dkv_cache_bytes(self.desc)
+            if nbytes == 0:
+                raise DkvError(DKV_EINVAL, "dkv_cache_bytes")
+            self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+            base = (self.buf.data_ptr() + 255) // 256 * 256
+            self.c = dkv_cache_init(self.desc, base, nbytes, stream)
         self._ws = None
         self._ws_heads = None
         self.device = device

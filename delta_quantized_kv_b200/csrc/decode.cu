@@ -125,7 +125,7 @@ struct Cursor {
     int units_b;               // units per sequence of batch entry b
     int len_b;                 // tokens of batch entry b
     int seg, nseg;             // segment within the unit (kf > 32 only)
-    const uint8_t *seq;        // data of sequence (b, kv head of vs)
+    const uint8_t *seq;        // data of sequence (b, kv head of vs) (contiguous caches)
     __device__ bool valid() const { return left > 0; }
 };
 
@@ -266,10 +266,17 @@ __device__ inline StageMap stage_map(int kf, int64_t rec, int u) {
     return m;
 }
 
+// First record of the cursor's current unit (delta format).
+template <bool PAGED>
+__device__ inline const uint8_t *stage_rec(const CacheView &cv, const Cursor &c, int nhg) {
+    if (!PAGED) return c.seq + (int64_t)c.g * cv.rec_bytes;
+    return rec_ptr<true>(cv, c.b, nhg == 1 ? c.vs : c.vs / nhg, c.g);
+}
+
 // Issue the bulk copies of one stage (nu units starting at c; one lane).
-template <int FMT, int MODE>
-__device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nu, int npos_all,
-                                   uint8_t *stage, uint64_t *bar, int fault) {
+template <int FMT, int MODE, bool PAGED>
+__device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nhg, int nu,
+                                   int npos_all, uint8_t *stage, uint64_t *bar, int fault) {
     constexpr int NU = KCfg<FMT, MODE>::NU;
     const uint8_t *sb = c.seq;
     if (fault) {
@@ -279,15 +286,25 @@ __device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nu,
         return;
     }
     if (FMT == DKV_FMT_DELTA && MODE == SUFFIX) {
+        // nu consecutive records (one page holds both when paged)
+        const uint8_t *rec = stage_rec<PAGED>(cv, c, nhg);
+        if (!rec) {                      // bad block-table entry: flagged, nothing copied
+            mbar_arrive_expect_tx(bar, 0);
+            return;
+        }
         const uint32_t bytes = (uint32_t)(nu * cv.rec_bytes);
         mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(stage, sb + (int64_t)c.g * cv.rec_bytes, bytes, bar);
+        bulk_g2s(stage, rec, bytes, bar);
     } else if (FMT == DKV_FMT_DELTA) {
         const int kf = cv.kf;
         const int glen = min(kf, c.len_b - c.g * kf);
         const int a = c.seg * SEG;
         const int npos = min(SEG, glen - a);
-        const uint8_t *rec = sb + (int64_t)c.g * cv.rec_bytes;
+        const uint8_t *rec = stage_rec<PAGED>(cv, c, nhg);
+        if (!rec) {
+            mbar_arrive_expect_tx(bar, 0);
+            return;
+        }
         const uint8_t *scs = rec + KF_BYTES;
         const uint8_t *kns = scs + (int64_t)(kf - 1) * SC_BYTES;
         const uint8_t *vns = kns + (int64_t)(kf - 1) * NIB_BYTES;
@@ -326,14 +343,15 @@ __device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nu,
 // lane advances its cursor identically.
 // With one stage per warp the descriptor stays in registers (every lane
 // computes it); with more it goes to the stage's shared-memory slot.
-template <int FMT, int MODE>
+template <int FMT, int MODE, bool PAGED>
 __device__ inline StageMeta next_stage(const CacheView &cv, Cursor &c, int nvs, int nhg,
                                        uint8_t *stage, uint64_t *bar, StageMeta *meta, int lane,
                                        int fault) {
     constexpr int NU = KCfg<FMT, MODE>::NU;
     const int np0 = unit_npos(cv, c, c.g);
     int nu = 1, np1 = 0;
-    if (NU == 2 && c.left >= 2 && c.g + 1 < c.units_b) {
+    // two consecutive groups per stage, never across a page boundary
+    if (NU == 2 && c.left >= 2 && c.g + 1 < c.units_b && (!PAGED || (c.g + 1) % cv.pg != 0)) {
         nu = 2;
         np1 = unit_npos(cv, c, c.g + 1);
     }
@@ -344,7 +362,7 @@ __device__ inline StageMeta next_stage(const CacheView &cv, Cursor &c, int nvs, 
     m.flags = MODE == PREFIX ? ((c.seg == 0 ? 1 : 0) | (c.seg == c.nseg - 1 ? 2 : 0)) : 3;
     if (lane == 0) {
         if (KCfg<FMT, MODE>::NS > 1) *meta = m;
-        issue_stage<FMT, MODE>(cv, c, nu, np0 + np1, stage, bar, fault);
+        issue_stage<FMT, MODE, PAGED>(cv, c, nhg, nu, np0 + np1, stage, bar, fault);
     }
     cursor_next<MODE>(c, cv, nvs, nhg);
     if (nu == 2) cursor_next<MODE>(c, cv, nvs, nhg);
@@ -635,7 +653,7 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
     }
 }
 
-template <int FMT, int MODE, bool ZT>
+template <int FMT, int MODE, bool ZT, bool PAGED>
 __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_kernel(SplitArgs A) {
     using Cfg = KCfg<FMT, MODE>;
     constexpr int NS = Cfg::NS, STAGE = Cfg::STAGE, NU = Cfg::NU;
@@ -686,7 +704,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
 #pragma unroll 1
     for (int s = 0; s < NS; ++s) {
         if (ic.valid()) {
-            pend = next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + s * STAGE, mybar + s,
+            pend = next_stage<FMT, MODE, PAGED>(cv, ic, nvs, A.NHG, mystages + s * STAGE, mybar + s,
                                          mymeta + s, lane, A.fault);
             ++issued;
         }
@@ -919,7 +937,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
         ++consumed;
         if (ic.valid()) {
             if (lane == 0) fence_proxy_async();
-            pend = next_stage<FMT, MODE>(cv, ic, nvs, A.NHG, mystages + stage_i * STAGE,
+            pend = next_stage<FMT, MODE, PAGED>(cv, ic, nvs, A.NHG, mystages + stage_i * STAGE,
                                          mybar + stage_i, mymeta + stage_i, lane, A.fault);
             ++issued;
         }
@@ -1038,11 +1056,12 @@ static cudaError_t geom_for(SplitGeom *g) {
     if (e != cudaSuccess) return e;
     if (dev != cached_dev) {
         const size_t sm = split_smem<FMT, MODE>();
-        e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT>,
+        e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
         int per_sm = 0, nsm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_kernel<FMT, MODE, ZT>,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm,
+                                                          split_kernel<FMT, MODE, ZT, false>,
                                                           WARPS * 32, sm);
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -1070,13 +1089,34 @@ cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g) {
     return geom_for<DKV_FMT_FP16, PLAIN, false>(g);
 }
 
+// The paged instance runs on the contiguous instance's grid (the merge and the
+// workspace size follow that grid); a persistent grid is correct at any size.
 template <int FMT, int MODE, bool ZT>
 static cudaError_t launch_split_t(const SplitArgs &a, cudaStream_t st) {
     SplitGeom g;
     cudaError_t e = geom_for<FMT, MODE, ZT>(&g);
     if (e != cudaSuccess) return e;
-    split_kernel<FMT, MODE, ZT><<<g.ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
-    return cudaGetLastError();
+    if (a.cv.pg == 0) {
+        split_kernel<FMT, MODE, ZT, false><<<g.ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
+        return cudaGetLastError();
+    }
+    if constexpr (FMT == DKV_FMT_DELTA) {
+        static int paged_dev = -1;
+        int dev;
+        e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev != paged_dev) {
+            e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)split_smem<FMT, MODE>());
+            if (e != cudaSuccess) return e;
+            paged_dev = dev;
+        }
+        split_kernel<FMT, MODE, ZT, true><<<g.ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
+        return cudaGetLastError();
+    } else {
+        return cudaErrorInvalidValue;    // only the delta format is paged
+    }
 }
 
 cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq,

@@ -34,7 +34,9 @@ dkv_status check_desc(const dkv_cache_desc *d) {
     return DKV_OK;
 }
 
-Layout make_layout(const dkv_cache_desc *d) {
+// paged: no data area (the records live in the page pool); the metadata
+// starts at the buffer's beginning
+Layout make_layout(const dkv_cache_desc *d, bool paged = false) {
     Layout L{};
     const size_t cap = (size_t)d->max_ctx;
     if (d->fmt == DKV_FMT_DELTA) {
@@ -52,21 +54,36 @@ Layout make_layout(const dkv_cache_desc *d) {
     }
     const size_t nseq = (size_t)d->batch * d->n_kv_heads;
     L.off_data = 0;
-    L.off_state = align_up(nseq * L.seq_stride + 4096, kAlign);
+    L.off_state = paged ? 0 : align_up(nseq * L.seq_stride + 4096, kAlign);
     L.off_seqlen = align_up(L.off_state + 2 * nseq * 2 * dkv::D * sizeof(float), kAlign);
     L.off_header = align_up(L.off_seqlen + (size_t)d->batch * sizeof(int32_t), kAlign);
     L.total = align_up(L.off_header + 16, kAlign);
     return L;
 }
 
+size_t page_bytes_of(const dkv_cache_desc *d, int32_t pg) {
+    return align_up((size_t)d->n_kv_heads * (size_t)pg * (size_t)dkv::delta_rec_bytes(d->kf),
+                    kAlign);
+}
+
 dkv_status check_cache(const dkv_cache *c) {
     if (!c || !c->base) return DKV_EINVAL;
     dkv_status s = check_desc(&c->desc);
     if (s != DKV_OK) return s;
-    Layout L = make_layout(&c->desc);
+    const bool paged = c->page_groups != 0;
+    Layout L = make_layout(&c->desc, paged);
     if (c->bytes < L.total || c->seq_stride != L.seq_stride || c->off_header != L.off_header)
         return DKV_EINVAL;
     if ((reinterpret_cast<uintptr_t>(c->base) & (kAlign - 1)) != 0) return DKV_EALIGN;
+    if (paged) {
+        if (c->desc.fmt != DKV_FMT_DELTA || c->page_groups < 1 || !c->pool || !c->block_table ||
+            c->n_pages < 1 || c->page_bytes != page_bytes_of(&c->desc, c->page_groups) ||
+            (int64_t)c->max_pages * c->page_groups < L.n_groups)
+            return DKV_EINVAL;
+        if ((reinterpret_cast<uintptr_t>(c->pool) & (kAlign - 1)) != 0 ||
+            (reinterpret_cast<uintptr_t>(c->block_table) & 3) != 0)
+            return DKV_EALIGN;
+    }
     return DKV_OK;
 }
 
@@ -82,6 +99,12 @@ CacheView view_of(const dkv_cache *c) {
     v.B = c->desc.batch;
     v.Hkv = c->desc.n_kv_heads;
     v.kf = c->desc.fmt == DKV_FMT_DELTA ? c->desc.kf : 1;
+    v.pool = static_cast<uint8_t *>(c->pool);
+    v.bt = c->block_table;
+    v.page_bytes = (int64_t)c->page_bytes;
+    v.n_pages = c->n_pages;
+    v.pg = c->page_groups;
+    v.maxp = c->max_pages;
     v.cap = c->desc.max_ctx;
     v.fmt = c->desc.fmt;
     v.n_groups = c->n_groups;
@@ -153,6 +176,55 @@ dkv_status dkv_cache_init(const dkv_cache_desc *desc, void *dev, size_t bytes, d
     out->off_seqlen = L.off_seqlen;
     out->off_header = L.off_header;
     return cuda_status(cudaMemsetAsync(dev, 0, L.total, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dkv_cache_meta_bytes(const dkv_cache_desc *desc) {
+    if (check_desc(desc) != DKV_OK || desc->fmt != DKV_FMT_DELTA) return 0;
+    return make_layout(desc, true).total;
+}
+
+size_t dkv_page_bytes(const dkv_cache_desc *desc, int32_t page_groups) {
+    if (check_desc(desc) != DKV_OK || desc->fmt != DKV_FMT_DELTA || page_groups < 1) return 0;
+    return page_bytes_of(desc, page_groups);
+}
+
+dkv_status dkv_cache_init_paged(const dkv_cache_desc *desc, int32_t page_groups, void *pool,
+                                int64_t n_pages, const int32_t *block_table, int32_t max_pages,
+                                void *meta, size_t meta_bytes, dkv_cache *out, void *stream) {
+    dkv_status s = check_desc(desc);
+    if (s != DKV_OK) return s;
+    if (desc->fmt != DKV_FMT_DELTA) return DKV_EUNSUPPORTED;
+    if (!pool || !block_table || !meta || !out || page_groups < 1 || n_pages < 1 ||
+        max_pages < 1)
+        return DKV_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(pool) & (kAlign - 1)) != 0 ||
+        (reinterpret_cast<uintptr_t>(meta) & (kAlign - 1)) != 0 ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3) != 0)
+        return DKV_EALIGN;
+    Layout L = make_layout(desc, true);
+    if ((int64_t)max_pages * page_groups < L.n_groups) return DKV_EINVAL;
+    if (meta_bytes < L.total) return DKV_ECAPACITY;
+    std::memset(out, 0, sizeof(*out));
+    out->desc = *desc;
+    out->base = meta;
+    out->bytes = meta_bytes;
+    out->seq_stride = L.seq_stride;
+    out->rec_bytes = L.rec_bytes;
+    out->n_groups = L.n_groups;
+    out->off_data = 0;
+    out->off_state = L.off_state;
+    out->off_seqlen = L.off_seqlen;
+    out->off_header = L.off_header;
+    out->pool = pool;
+    out->block_table = block_table;
+    out->page_bytes = page_bytes_of(desc, page_groups);
+    out->n_pages = n_pages;
+    out->page_groups = page_groups;
+    out->max_pages = max_pages;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(meta, 0, L.total, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(pool, 0, (size_t)n_pages * out->page_bytes, st);
+    return cuda_status(e);
 }
 
 dkv_status dkv_encode(dkv_cache *cache, const void *K, const void *V, int32_t dtype,

@@ -83,10 +83,33 @@ struct CacheView {
     int64_t seq_stride;
     int64_t rec_bytes;
     int32_t B, Hkv, kf, cap, fmt, n_groups;
+    // paged (delta format): pg = groups per page (0: contiguous)
+    uint8_t *pool;
+    const int32_t *bt;     // [B][maxp] page indices
+    int64_t page_bytes, n_pages;
+    int32_t pg, maxp;
 };
 
 __device__ inline void set_status(int32_t *header, int bits) {
     atomicOr(reinterpret_cast<int *>(header), bits);
+}
+
+// Record g (delta format) of sequence (b, kvh): contiguous, or through the
+// block table (PAGED); nullptr (and DKV_DEV_BAD_PAGE) for an entry outside the
+// pool.
+template <bool PAGED>
+__device__ inline uint8_t *rec_ptr(const CacheView &cv, int b, int kvh, int g) {
+    if (!PAGED)
+        return cv.data + ((int64_t)b * cv.Hkv + kvh) * cv.seq_stride + (int64_t)g * cv.rec_bytes;
+    const int page = cv.bt[(int64_t)b * cv.maxp + g / cv.pg];
+    if (page < 0 || page >= cv.n_pages) {
+        set_status(cv.header, DKV_DEV_BAD_PAGE);
+        return nullptr;
+    }
+    return cv.pool + (int64_t)page * cv.page_bytes + ((int64_t)kvh * cv.pg + g % cv.pg) * cv.rec_bytes;
+}
+__device__ inline uint8_t *rec_ptr(const CacheView &cv, int b, int kvh, int g) {
+    return cv.pg ? rec_ptr<true>(cv, b, kvh, g) : rec_ptr<false>(cv, b, kvh, g);
 }
 
 // ---------------------------------------------------------------------------

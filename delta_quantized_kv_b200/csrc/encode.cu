@@ -125,8 +125,12 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
             const int kf = cv.kf;
             const int g = start / kf + blockIdx.x;
             const int p0 = max(start, g * kf), p1 = min(start + n, (g + 1) * kf);
-            if (p0 < p1) {
-                uint8_t *rec = sb + (int64_t)g * cv.rec_bytes;
+            uint8_t *rec = p0 < p1 ? rec_ptr(cv, b, kvh, g) : nullptr;
+            if (p0 < p1 && !rec) {
+                // bad block-table entry (flagged by rec_ptr): nothing written;
+                // the state carries over
+                if (p1 == start + n) state_new[c] = (p0 % kf) ? state_old[c] : 0.0f;
+            } else if (p0 < p1) {
                 uint8_t *sc_base = rec + KF_BYTES;
                 uint8_t *nib_base = rec + KF_BYTES + (int64_t)(kf - 1) * SC_BYTES +
                                     (int64_t)t * (kf - 1) * NIB_BYTES;
@@ -277,7 +281,8 @@ __global__ void __launch_bounds__(128) readback_kernel(ExportArgs a) {
                 cv.state[((((int64_t)parity * cv.B + b) * cv.Hkv + kvh) * 2 + t) * D + c];
         }
         if (g * kf >= len) return;
-        const uint8_t *rec = sb + (int64_t)g * cv.rec_bytes;
+        const uint8_t *rec = rec_ptr(cv, b, kvh, g);
+        if (!rec) return;
         const uint8_t *scb = rec + KF_BYTES;
         const uint8_t *nib = rec + KF_BYTES + (int64_t)(kf - 1) * SC_BYTES +
                              (int64_t)t * (kf - 1) * NIB_BYTES;

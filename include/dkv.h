@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define DKV_ABI_VERSION 1
+#define DKV_ABI_VERSION 2
 
 typedef enum {
     DKV_OK = 0,
@@ -71,6 +71,7 @@ typedef enum { DKV_F32 = 0, DKV_F16 = 1, DKV_BF16 = 2 } dkv_dtype;
 #define DKV_DEV_CAPACITY     0x2   /* an append would pass max_ctx (skipped) */
 #define DKV_DEV_TIMEOUT      0x4   /* a bounded pipeline wait ran out */
 #define DKV_DEV_BAD_HEADS    0x8   /* n_q_heads not a multiple of n_kv_heads */
+#define DKV_DEV_BAD_PAGE     0x10  /* a block-table entry outside the page pool (skipped) */
 
 typedef struct {
     int32_t batch;         /* B >= 1 (<= 1024) */
@@ -82,19 +83,32 @@ typedef struct {
 } dkv_cache_desc;
 
 /* POD view of a cache laid out in caller-owned device memory.  Filled by
- * dkv_cache_init; all offsets are bytes from `base`. */
+ * dkv_cache_init (contiguous) or dkv_cache_init_paged; all offsets are bytes
+ * from `base`. */
 typedef struct {
     dkv_cache_desc desc;
     void *base;
     size_t bytes;
-    size_t seq_stride;     /* bytes of one (batch, kv-head) sequence's data */
+    size_t seq_stride;     /* contiguous: bytes of one (batch, kv-head) sequence's data */
     size_t rec_bytes;      /* DELTA: bytes of one keyframe group record */
     int32_t n_groups;      /* DELTA: groups per sequence at capacity */
     int32_t reserved0;
-    size_t off_data;       /* compressed data, B*Hkv*seq_stride bytes */
+    size_t off_data;       /* contiguous: compressed data, B*Hkv*seq_stride bytes */
     size_t off_state;      /* fp32 reconstruction state [2][B][Hkv][2][D] */
     size_t off_seqlen;     /* int32 seq_len[B] */
     size_t off_header;     /* int32 {status, counter, parity, reserved} */
+    /* paged (DELTA only; page_groups == 0 for a contiguous cache): the records
+     * live in a pool of pages; page i holds, for every kv head h, the records
+     * of page_groups consecutive keyframe groups of one sequence, at
+     * pool + i*page_bytes + (h*page_groups + g % page_groups)*rec_bytes, and
+     * block_table[b*max_pages + g / page_groups] names the page of group g of
+     * batch entry b. */
+    void *pool;
+    const int32_t *block_table;  /* device int32 [B][max_pages], caller-owned */
+    size_t page_bytes;
+    int64_t n_pages;
+    int32_t page_groups;
+    int32_t max_pages;
 } dkv_cache;
 
 /* ABI version of the loaded library (DKV_ABI_VERSION). */
@@ -108,6 +122,31 @@ size_t dkv_cache_bytes(const dkv_cache_desc *desc);
  * with cudaMemsetAsync on `stream` (every seq_len becomes 0).  Fills *out. */
 dkv_status dkv_cache_init(const dkv_cache_desc *desc, void *dev, size_t bytes,
                           dkv_cache *out, void *stream);
+
+/* Paged cache (NEXT row: a paged, group-aligned cache for ragged serving;
+ * the "decoupled memory management" of page "DeltaKV ... Sparse-vLLM",
+ * section "B. Sparse-vLLM", without the learned compressor).
+ * dkv_cache_meta_bytes: bytes of the small metadata buffer a paged cache
+ * needs (reconstruction state, lengths, header); dkv_page_bytes: bytes of one
+ * page of page_groups keyframe groups (all kv heads), a multiple of 256.
+ * Both return 0 for an invalid descriptor (or a format other than
+ * DKV_FMT_DELTA, or page_groups < 1). */
+size_t dkv_cache_meta_bytes(const dkv_cache_desc *desc);
+size_t dkv_page_bytes(const dkv_cache_desc *desc, int32_t page_groups);
+
+/* Lay out a paged cache: metadata in `meta` (>= dkv_cache_meta_bytes,
+ * 256-byte aligned), records in `pool` (n_pages pages of dkv_page_bytes,
+ * 256-byte aligned), pages named by `block_table` (device int32
+ * [B][max_pages], 4-byte aligned, max_pages >= the pages max_ctx needs).
+ * Zeroes the metadata and the pool with cudaMemsetAsync on `stream`.  The
+ * block table stays caller-owned: entries may change between calls (a page
+ * per page_groups*kf tokens of one sequence, never shared by two sequences);
+ * a kernel that meets an entry outside [0, n_pages) sets DKV_DEV_BAD_PAGE and
+ * skips that group.  DKV_FMT_DELTA only (DKV_EUNSUPPORTED otherwise).  Every
+ * other call takes the resulting cache as it takes a contiguous one. */
+dkv_status dkv_cache_init_paged(const dkv_cache_desc *desc, int32_t page_groups, void *pool,
+                                int64_t n_pages, const int32_t *block_table, int32_t max_pages,
+                                void *meta, size_t meta_bytes, dkv_cache *out, void *stream);
 
 /* Encode whole sequences, replacing the cache contents.
  * K, V: [B][Hkv][T][D] contiguous device arrays of `dtype`.

@@ -40,7 +40,9 @@ def test_exports_every_declared_symbol(dkv):
 
 
 def test_abi_version_and_status_strings(dkv):
-    assert dkv.dkv_abi_version() == 1
+    hdr = (ROOT / "include" / "dkv.h").read_text()
+    want = int(re.search(r"#define DKV_ABI_VERSION (\d+)", hdr).group(1))
+    assert dkv.dkv_abi_version() == want
     for s in range(7):
         assert dkv.status_str(s) and dkv.status_str(s) != "unknown status"
     assert dkv.status_str(99) == "unknown status"
@@ -178,3 +180,33 @@ def test_work_split_covers_every_unit_once_and_slots_are_unique():
                 assert slot not in slots, (slot, slots.get(slot), (w, s))
                 slots[slot] = (w, s)
                 assert slot < NW + nseq
+
+
+def test_paged_sizes_and_argument_checks(dkv):
+    """Paged cache (delta format): metadata and page sizes follow the record
+    layout, and bad arguments are rejected on the host before any launch."""
+    import ctypes
+    d = _desc(dkv, B=4, H=8, kf=32, cap=4096)
+    rec = 512 + 31 * 144
+    assert dkv.dkv_page_bytes(d, 16) == -(-8 * 16 * rec // 256) * 256
+    assert dkv.dkv_page_bytes(d, 0) == 0
+    meta = dkv.dkv_cache_meta_bytes(d)
+    # fp32 state [2][B][Hkv][2][128], seq_len[B], header: no data area
+    assert 2 * 4 * 8 * 2 * 128 * 4 < meta < 2 * 4 * 8 * 2 * 128 * 4 + 4096
+    assert dkv.dkv_cache_meta_bytes(_desc(dkv, fmt=1)) == 0          # Q4_0 is not paged
+    lib = dkv.load()
+    out = dkv.dkv_cache()
+    A = 1 << 20                                                          # 256-aligned fake addresses
+    # too few block-table columns for max_ctx (4096 / 32 = 128 groups, 16 per page -> 8)
+    assert lib.dkv_cache_init_paged(ctypes.byref(d), 16, A, 64, A, 7, A, meta, ctypes.byref(out),
+                                    None) == dkv.DKV_EINVAL
+    # misaligned pool, meta too small, page_groups < 1, comparator format
+    assert lib.dkv_cache_init_paged(ctypes.byref(d), 16, A + 16, 64, A, 8, A, meta,
+                                    ctypes.byref(out), None) == dkv.DKV_EALIGN
+    assert lib.dkv_cache_init_paged(ctypes.byref(d), 16, A, 64, A, 8, A, meta - 1,
+                                    ctypes.byref(out), None) == dkv.DKV_ECAPACITY
+    assert lib.dkv_cache_init_paged(ctypes.byref(d), 0, A, 64, A, 8, A, meta, ctypes.byref(out),
+                                    None) == dkv.DKV_EINVAL
+    dq = _desc(dkv, B=4, H=8, cap=4096, fmt=1)
+    assert lib.dkv_cache_init_paged(ctypes.byref(dq), 16, A, 64, A, 8, A, meta,
+                                    ctypes.byref(out), None) == dkv.DKV_EUNSUPPORTED
