@@ -126,6 +126,9 @@ struct Cursor {
     int len_b;                 // tokens of batch entry b
     int seg, nseg;             // segment within the unit (kf > 32 only)
     const uint8_t *seq;        // data of sequence (b, kv head of vs) (contiguous caches)
+    // paged caches, issuing lane only: the page last looked up
+    int pb, pv, pidx;          // its batch entry, sequence and block-table column
+    const uint8_t *pbase;      // its records of kv head vs / nhg (null: entry was bad)
     __device__ bool valid() const { return left > 0; }
 };
 
@@ -186,6 +189,7 @@ __device__ inline void cursor_seek(Cursor &c, const CacheView &cv, int nvs, int 
     c.seg = 0;
     c.nseg = nseg_of<MODE>(cv, c.len_b, c.g);
     c.seq = seq_ptr(cv, c.b, c.vs, nhg);
+    c.pb = -1;
 }
 
 template <int MODE>
@@ -266,16 +270,25 @@ __device__ inline StageMap stage_map(int kf, int64_t rec, int u) {
     return m;
 }
 
-// First record of the cursor's current unit (delta format).
+// First record of the cursor's current unit (delta format).  Paged: the
+// block table is read once per page (the issuing lane keeps the page's base).
 template <bool PAGED>
-__device__ inline const uint8_t *stage_rec(const CacheView &cv, const Cursor &c, int nhg) {
+__device__ inline const uint8_t *stage_rec(const CacheView &cv, Cursor &c, int nhg) {
     if (!PAGED) return c.seq + (int64_t)c.g * cv.rec_bytes;
-    return rec_ptr<true>(cv, c.b, nhg == 1 ? c.vs : c.vs / nhg, c.g);
+    const int pidx = c.g / cv.pg;
+    if (c.pb != c.b || c.pv != c.vs || c.pidx != pidx) {
+        const int kvh = nhg == 1 ? c.vs : c.vs / nhg;
+        c.pbase = rec_ptr<true>(cv, c.b, kvh, pidx * cv.pg);
+        c.pb = c.b;
+        c.pv = c.vs;
+        c.pidx = pidx;
+    }
+    return c.pbase ? c.pbase + (int64_t)(c.g - pidx * cv.pg) * cv.rec_bytes : nullptr;
 }
 
 // Issue the bulk copies of one stage (nu units starting at c; one lane).
 template <int FMT, int MODE, bool PAGED>
-__device__ inline void issue_stage(const CacheView &cv, const Cursor &c, int nhg, int nu,
+__device__ inline void issue_stage(const CacheView &cv, Cursor &c, int nhg, int nu,
                                    int npos_all, uint8_t *stage, uint64_t *bar, int fault) {
     constexpr int NU = KCfg<FMT, MODE>::NU;
     const uint8_t *sb = c.seq;

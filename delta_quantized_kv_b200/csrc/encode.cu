@@ -9,7 +9,8 @@
 // the reconstruction (closed loop, section "컨텍스트 길이에 따른 안정성").
 // Each quantiser step is one IEEE fp32 operation in a fixed order (__fsub_rn,
 // __fdiv_rn, __fadd_rn, __fmul_rn), so codes and scales are bit-exact with any
-// other implementation that takes the same steps in the same order.
+// other implementation that takes the same steps in the same order (m / -8 is
+// taken as m * -0.125: the same real value, rounded once, so the same bits).
 #include <cstdint>
 
 #include "dkv_common.cuh"
@@ -30,7 +31,7 @@ __device__ inline int quant_lane(float v, __half *d16_out) {
     uint32_t mx = __reduce_max_sync(0xffffffffu, a);
     uint32_t ball = __ballot_sync(0xffffffffu, a == mx);
     float m = __shfl_sync(0xffffffffu, v, __ffs(ball) - 1);  // lowest index on ties
-    float d32 = __fdiv_rn(m, -8.0f);
+    float d32 = __fmul_rn(m, -0.125f);   // = m / -8 exactly: one rounding of the same real value
     __half d16 = __float2half_rn(d32);
     float d = __half2float(d16);
     *d16_out = d16;
