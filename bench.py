@@ -612,6 +612,28 @@ def run_ours(args, w, rank, world, local):
                                               "gbps": nb / (t * 1e-3) / 1e9,
                                               "status": cp.device_status()}
             del cp
+        # multi-query decode: 2 queries per sequence (speculative decoding), G = 8,
+        # so 16 virtual heads per kv head in two groups of 8 (the cache is read
+        # once per group)
+        if args.fmt == "delta":
+            nq = 2
+            gq = torch.Generator(device=dev).manual_seed(5)
+            Q2 = torch.randn((B, nq, Hq, D), generator=gq, device=dev).to(w.q_dtype)
+            out2 = torch.empty((B, nq, Hq, D), dtype=torch.float32, device=dev)
+            for _ in range(3):
+                cache.decode_attn_mq(Q2, scale, out=out2)
+            torch.cuda.synchronize()
+            a, bq = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = max(5, K)
+            a.record(stream)
+            for i in range(n):
+                cache.decode_attn_mq(Q2, scale, out=out2)
+            bq.record(stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(bq) / n
+            nb = kv_bytes("delta", [T0 + n_app + n_e2e] * B, Hkv, w.kf)
+            extra["delta_2_queries"] = {"decode_attn_us": 1e3 * t, "bytes": nb,
+                                        "gbps": nb / (t * 1e-3) / 1e9}
         # reconstruction MSE on a slice (first 2 batch entries)
         nb_ = min(2, B)
         xs = {"K": Kp[:nb_].float(), "V": Vp[:nb_].float()}

@@ -54,7 +54,7 @@ EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode",
            "dkv_decode_attn_merge", "dkv_export_canonical", "dkv_dequantize",
            "dkv_get_device_status", "dkv_status_str", "dkv_decode_attn_noalloc",
            "dkv_debug_set_fault", "dkv_cache_meta_bytes", "dkv_page_bytes",
-           "dkv_cache_init_paged"]
+           "dkv_cache_init_paged", "dkv_decode_workspace_bytes_mq", "dkv_decode_attn_mq"]
 
 
 def load():
@@ -88,6 +88,8 @@ def load():
         "dkv_cache_meta_bytes": ([PD], S),
         "dkv_page_bytes": ([PD, I], S),
         "dkv_cache_init_paged": ([PD, I, P, ctypes.c_int64, P, I, P, S, PC, P], I),
+        "dkv_decode_workspace_bytes_mq": ([PD, I, I], S),
+        "dkv_decode_attn_mq": ([PC, P, I, I, I, F, P, P, S, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -189,6 +191,17 @@ def dkv_decode_attn(cache: dkv_cache, Q, q_dtype, n_q_heads, softmax_scale, out,
     _check(load().dkv_decode_attn(ctypes.byref(cache), _ptr(Q), q_dtype, n_q_heads,
                                   softmax_scale, _ptr(out), _ptr(workspace), ws_bytes,
                                   _stream(stream)), "dkv_decode_attn")
+
+
+def dkv_decode_workspace_bytes_mq(desc: dkv_cache_desc, n_q_heads: int, n_queries: int) -> int:
+    return load().dkv_decode_workspace_bytes_mq(ctypes.byref(desc), n_q_heads, n_queries)
+
+
+def dkv_decode_attn_mq(cache: dkv_cache, Q, q_dtype, n_q_heads, n_queries, softmax_scale, out,
+                       workspace, ws_bytes, stream=None) -> None:
+    _check(load().dkv_decode_attn_mq(ctypes.byref(cache), _ptr(Q), q_dtype, n_q_heads, n_queries,
+                                     softmax_scale, _ptr(out), _ptr(workspace), ws_bytes,
+                                     _stream(stream)), "dkv_decode_attn_mq")
 
 
 def dkv_decode_attn_split(cache: dkv_cache, Q, q_dtype, n_q_heads, softmax_scale, workspace,
@@ -317,6 +330,25 @@ class Cache:
         ws = self.workspace(Hq)
         dkv_decode_attn(self.c, Q, _dtype_code(Q.dtype), Hq, softmax_scale, out, ws,
                         ws.numel() * 4, stream)
+        return out
+
+    def decode_attn_mq(self, Q, softmax_scale, out=None, stream=None):
+        """Q: [B, n_queries, Hq, D]; query t attends causally (see
+        dkv_decode_attn_mq).  Returns fp32 [B, n_queries, Hq, D]."""
+        import torch
+        B, nq, Hq, Dh = Q.shape
+        if out is None:
+            out = torch.empty((B, nq, Hq, Dh), dtype=torch.float32, device=Q.device)
+        key = ("mq", Hq, nq)
+        ws = getattr(self, "_ws_mq", {}).get(key)
+        if ws is None:
+            nb = dkv_decode_workspace_bytes_mq(self.desc, Hq, nq)
+            if nb == 0:
+                raise DkvError(DKV_EINVAL, "dkv_decode_workspace_bytes_mq")
+            ws = torch.zeros(nb // 4 + 64, dtype=torch.float32, device=self.device)
+            self._ws_mq = {key: ws}
+        dkv_decode_attn_mq(self.c, Q.contiguous(), _dtype_code(Q.dtype), Hq, nq, softmax_scale,
+                           out, ws, ws.numel() * 4, stream)
         return out
 
     def seq_lens(self):

@@ -82,10 +82,10 @@ template <int FMT, int MODE> struct SmemMap {
     static constexpr int NS = KCfg<FMT, MODE>::NS, STAGE = KCfg<FMT, MODE>::STAGE;
     static constexpr int BAR_OFF = 0;
     static constexpr int META_OFF = ((BAR_OFF + 8 * WARPS * NS) + 15) / 16 * 16;
-    static constexpr int STAGE_OFF = ((META_OFF + 16 * WARPS * NS) + 127) / 128 * 128;
+    static constexpr int STAGE_OFF = ((META_OFF + 32 * WARPS * NS) + 127) / 128 * 128;
     static constexpr int BYTES = STAGE_OFF + WARPS * NS * STAGE;
     static_assert(META_OFF >= BAR_OFF + 8 * WARPS * NS, "barriers overlap descriptors");
-    static_assert(STAGE_OFF >= META_OFF + 16 * WARPS * NS, "descriptors overlap stages");
+    static_assert(STAGE_OFF >= META_OFF + 32 * WARPS * NS, "descriptors overlap stages");
     static_assert(STAGE % 128 == 0, "stages must stay 128-byte aligned");
     static_assert(BYTES <= 227 * 1024, "shared memory per CTA");
 };
@@ -95,6 +95,7 @@ struct SplitArgs {
     const void *Q;
     int q_dtype;
     int Hq, G, NHG;            // query heads, heads per kv head, head groups of 8
+    int nq;                    // queries per sequence (the newest nq tokens' own, causal)
     float scale_log2;          // softmax_scale * log2(e), > 0
     float *ws;                 // partial records
     int fault;                 // test support: 1 = arm the copy barriers but issue no copy
@@ -218,7 +219,10 @@ struct StageMeta {
     int b, vs;                 // batch entry, sequence within it
     int npos;                  // valid positions: unit 0 in bits 0-7, unit 1 in bits 8-15
     int flags;                 // bit 0: first segment of a group; bit 1: last segment
+    int pos0;                  // position of unit 0's first slot in its sequence
+    int pad[3];
 };
+static_assert(sizeof(StageMeta) == 32, "stage descriptors are 32 bytes");
 
 // Positions of the current unit of c.
 __device__ inline int unit_npos(const CacheView &cv, const Cursor &c, int g) {
@@ -373,6 +377,7 @@ __device__ inline StageMeta next_stage(const CacheView &cv, Cursor &c, int nvs, 
     m.vs = c.vs;
     m.npos = np0 | (np1 << 8);
     m.flags = MODE == PREFIX ? ((c.seg == 0 ? 1 : 0) | (c.seg == c.nseg - 1 ? 2 : 0)) : 3;
+    m.pos0 = FMT == DKV_FMT_DELTA ? c.g * cv.kf + c.seg * SEG : c.g * SEG;
     if (lane == 0) {
         if (KCfg<FMT, MODE>::NS > 1) *meta = m;
         issue_stage<FMT, MODE, PAGED>(cv, c, nhg, nu, np0 + np1, stage, bar, fault);
@@ -729,7 +734,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
     // per-sequence state (heads 2*tq + e of the current head group)
     int cur_b = -1, cur_vs = -1;
     uint32_t qb[8][2];                  // B fragments of q (column = head gq)
-    bool head_ok[2] = {false, false};
+    int lp[2] = {0, 0};                 // positions heads 2tq + e may see (causal queries)
     float m_run[2] = {-1e30f, -1e30f}, l_run[2] = {0.f, 0.f};
     float o[8][4];
     float racc[8][4];                   // PREFIX: sum of dequantised deltas of the group
@@ -789,12 +794,22 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
         if (meta.b != cur_b || meta.vs != cur_vs) {
             if (cur_b >= 0) flush();
             cur_b = meta.b; cur_vs = meta.vs;
+            // virtual heads of a kv head: query t of the sequence, head h of the
+            // GQA group -> v = t * G + h, 8 per head group; query t sees the
+            // positions before len - (nq - 1 - t)
             const int kvh = meta.vs / A.NHG, hg = meta.vs % A.NHG;
-            const int hl = hg * 8 + gq;                  // head of this thread's q column
-            const bool qok = hl < A.G;
-            head_ok[0] = hg * 8 + 2 * tq < A.G;
-            head_ok[1] = hg * 8 + 2 * tq + 1 < A.G;
-            const int64_t qrow = ((int64_t)meta.b * A.Hq + (int64_t)kvh * A.G + (qok ? hl : 0)) * D;
+            const int Gv = A.nq * A.G;
+            const int vq = hg * 8 + gq;                  // virtual head of this thread's q column
+            const bool qok = vq < Gv;
+            const int qt = qok ? vq / A.G : 0, hl = qok ? vq % A.G : 0;
+            const int len_b = clamp_len(cv, meta.b);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int ve = hg * 8 + 2 * tq + e;
+                lp[e] = ve < Gv ? len_b - (A.nq - 1 - ve / A.G) : 0;   // absent head: none
+            }
+            const int64_t qrow =
+                (((int64_t)meta.b * A.nq + qt) * A.Hq + (int64_t)kvh * A.G + hl) * D;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int c = 16 * kk + 2 * tq;
@@ -840,10 +855,15 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
             }
 
             // ================= scores, online softmax =======================
-            // valid slots of this thread: positions 4g + i with i < lim[u]
-            int lim[NU];
+            // valid slots of this thread per head: positions 4g + i with i < lim[u][e]
+            // (the unit's end, and for causal queries the head's own limit)
+            int lim[NU][2];
 #pragma unroll
-            for (int u = 0; u < NU; ++u) lim[u] = npos[u] - 4 * gq;
+            for (int u = 0; u < NU; ++u) {
+                const int us = meta.pos0 + u * (FMT == DKV_FMT_DELTA ? cv.kf : SEG);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) lim[u][e] = min(npos[u], lp[e] - us) - 4 * gq;
+            }
             float alpha[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -867,7 +887,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
                 for (int u = 0; u < NU; ++u)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        v[u][i] = (head_ok[e] && i < lim[u]) ? v[u][i] : -INFINITY;
+                        v[u][i] = i < lim[u][e] ? v[u][i] : -INFINITY;
                         mx = fmaxf(mx, v[u][i]);
                     }
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
@@ -974,18 +994,20 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
 // ---------------------------------------------------------------------------
 // merge: grid (Hq, B), 128 threads (one per channel)
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G, int NHG,
+// merge: grid (nq * Hq, B), 128 threads (one per channel); block x is query
+// t = x / Hq, head h = x % Hq, i.e. virtual head t * G + h % G of kv head h / G
+__global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G, int NHG, int nq,
                                                     int64_t NW, const float *ws, float *out) {
-    const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
+    const int t = blockIdx.x / Hq, h = blockIdx.x % Hq, b = blockIdx.y, c = threadIdx.x;
     const int nvs = cv.Hkv * NHG;
     const int len = clamp_len(cv, b);
     const int ub = units_of(cv.fmt, cv.kf, len);
-    float *dst = out + ((int64_t)b * Hq + h) * D;
+    float *dst = out + (((int64_t)b * nq + t) * Hq + h) * D;
     if (ub == 0) {                      // uniform over the block
         dst[c] = 0.f;
         return;
     }
-    const int kvh = h / G, hl = h % G, hg = hl >> 3, j = hl & 7;
+    const int kvh = h / G, vh = t * G + h % G, hg = vh >> 3, j = vh & 7;
     const int vsl = kvh * NHG + hg;
     // the warps whose unit ranges touch this sequence: found once per block
     __shared__ int64_t sh_w0, sh_w1, sh_total;
@@ -1050,7 +1072,7 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
             O += ov[i] * sc;
         }
     }
-    dst[c] = O / L;
+    dst[c] = L > 0.f ? O / L : 0.f;     // a causal query with no position gets 0
 }
 
 // ---------------------------------------------------------------------------
@@ -1132,7 +1154,7 @@ static cudaError_t launch_split_t(const SplitArgs &a, cudaStream_t st) {
     }
 }
 
-cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq,
+cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq, int nq,
                          float softmax_scale, float *ws, int64_t ws_floats, int fault,
                          cudaStream_t st) {
     (void)ws_floats;
@@ -1143,7 +1165,8 @@ cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq
     a.q_dtype = q_dtype;
     a.Hq = Hq;
     a.G = Hq / cv.Hkv;
-    a.NHG = (a.G + 7) / 8;
+    a.nq = nq;
+    a.NHG = (nq * a.G + 7) / 8;
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
     a.ws = ws;
     if (cv.fmt == DKV_FMT_DELTA) {
@@ -1155,14 +1178,16 @@ cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq
     return launch_split_t<DKV_FMT_FP16, PLAIN, false>(a, st);
 }
 
-cudaError_t launch_merge(const CacheView &cv, int Hq, float *out, const float *ws, cudaStream_t st) {
+cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const float *ws,
+                         cudaStream_t st) {
     SplitGeom g;
     cudaError_t e = split_geometry(cv.fmt, cv.kf, cv.B, &g);
     if (e != cudaSuccess) return e;
     const int G = Hq / cv.Hkv;
-    const int NHG = (G + 7) / 8;
-    dim3 grid(Hq, cv.B);
-    merge_kernel<<<grid, 128, 0, st>>>(cv, Hq, G, NHG, (int64_t)g.ctas * g.warps_per_cta, ws, out);
+    const int NHG = (nq * G + 7) / 8;
+    dim3 grid(nq * Hq, cv.B);
+    merge_kernel<<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, (int64_t)g.ctas * g.warps_per_cta, ws,
+                                       out);
     return cudaGetLastError();
 }
 

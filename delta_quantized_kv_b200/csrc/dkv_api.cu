@@ -117,28 +117,32 @@ int g_debug_fault = 0;   // dkv_debug_set_fault
 
 inline bool valid_dtype(int32_t t) { return t == DKV_F32 || t == DKV_F16 || t == DKV_BF16; }
 
-int64_t workspace_floats(const dkv_cache_desc *d, int32_t Hq, bool *ok) {
+constexpr int32_t kMaxQueries = 256;
+
+int64_t workspace_floats(const dkv_cache_desc *d, int32_t Hq, int32_t nq, bool *ok) {
     *ok = false;
     if (check_desc(d) != DKV_OK || Hq < 1 || Hq % d->n_kv_heads != 0) return 0;
+    if (nq < 1 || nq > kMaxQueries) return 0;
     dkv::SplitGeom g;
     if (dkv::split_geometry(d->fmt, d->kf, d->batch, &g) != cudaSuccess) return 0;
     const int G = Hq / d->n_kv_heads;
-    const int64_t nhg = (G + 7) / 8;
+    const int64_t nhg = ((int64_t)nq * G + 7) / 8;
     const int64_t slots = (int64_t)g.ctas * g.warps_per_cta + (int64_t)d->batch * d->n_kv_heads * nhg;
     *ok = true;
     return slots * dkv::PARTIAL_FLOATS;
 }
 
 dkv_status check_decode(const dkv_cache *cache, const void *Q, int32_t q_dtype, int32_t Hq,
-                        void *ws, size_t ws_bytes, int64_t *need_floats) {
+                        int32_t nq, void *ws, size_t ws_bytes, int64_t *need_floats) {
     dkv_status s = check_cache(cache);
     if (s != DKV_OK) return s;
     if (!ws || (Q == nullptr && q_dtype >= 0)) return DKV_EINVAL;
     if (q_dtype >= 0 && !valid_dtype(q_dtype)) return DKV_EINVAL;
     if (Hq < 1 || Hq % cache->desc.n_kv_heads != 0) return DKV_EINVAL;
+    if (nq < 1 || nq > kMaxQueries) return DKV_EINVAL;
     if ((Q && !aligned16(Q)) || !aligned16(ws)) return DKV_EALIGN;
     bool ok;
-    int64_t need = workspace_floats(&cache->desc, Hq, &ok);
+    int64_t need = workspace_floats(&cache->desc, Hq, nq, &ok);
     if (!ok) return DKV_ECUDA;
     if (ws_bytes < (size_t)need * sizeof(float)) return DKV_ECAPACITY;
     *need_floats = need;
@@ -253,8 +257,13 @@ dkv_status dkv_append(dkv_cache *cache, const void *K_new, const void *V_new, in
 }
 
 size_t dkv_decode_workspace_bytes(const dkv_cache_desc *desc, int32_t n_q_heads) {
+    return dkv_decode_workspace_bytes_mq(desc, n_q_heads, 1);
+}
+
+size_t dkv_decode_workspace_bytes_mq(const dkv_cache_desc *desc, int32_t n_q_heads,
+                                     int32_t n_queries) {
     bool ok;
-    int64_t f = workspace_floats(desc, n_q_heads, &ok);
+    int64_t f = workspace_floats(desc, n_q_heads, n_queries, &ok);
     return ok ? (size_t)f * sizeof(float) : 0;
 }
 
@@ -264,10 +273,10 @@ dkv_status dkv_decode_attn_split(const dkv_cache *cache, const void *Q, int32_t 
     int64_t need;
     if (!Q) return DKV_EINVAL;
     if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return DKV_EINVAL;  // finite, > 0
-    dkv_status s = check_decode(cache, Q, q_dtype, n_q_heads, workspace, ws_bytes, &need);
+    dkv_status s = check_decode(cache, Q, q_dtype, n_q_heads, 1, workspace, ws_bytes, &need);
     if (s != DKV_OK) return s;
     CacheView v = view_of(cache);
-    return cuda_status(dkv::launch_split(v, Q, q_dtype, n_q_heads, softmax_scale,
+    return cuda_status(dkv::launch_split(v, Q, q_dtype, n_q_heads, 1, softmax_scale,
                                          static_cast<float *>(workspace), need, g_debug_fault,
                                          static_cast<cudaStream_t>(stream)));
 }
@@ -276,11 +285,11 @@ dkv_status dkv_decode_attn_merge(const dkv_cache *cache, int32_t n_q_heads, floa
                                  void *workspace, size_t ws_bytes, void *stream) {
     int64_t need;
     if (!out) return DKV_EINVAL;
-    dkv_status s = check_decode(cache, nullptr, -1, n_q_heads, workspace, ws_bytes, &need);
+    dkv_status s = check_decode(cache, nullptr, -1, n_q_heads, 1, workspace, ws_bytes, &need);
     if (s != DKV_OK) return s;
     if (!aligned16(out)) return DKV_EALIGN;
     CacheView v = view_of(cache);
-    return cuda_status(dkv::launch_merge(v, n_q_heads, out, static_cast<const float *>(workspace),
+    return cuda_status(dkv::launch_merge(v, n_q_heads, 1, out, static_cast<const float *>(workspace),
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -293,6 +302,25 @@ dkv_status dkv_decode_attn(const dkv_cache *cache, const void *Q, int32_t q_dtyp
                                          ws_bytes, stream);
     if (s != DKV_OK) return s;
     return dkv_decode_attn_merge(cache, n_q_heads, out, workspace, ws_bytes, stream);
+}
+
+dkv_status dkv_decode_attn_mq(const dkv_cache *cache, const void *Q, int32_t q_dtype,
+                              int32_t n_q_heads, int32_t n_queries, float softmax_scale,
+                              float *out, void *workspace, size_t ws_bytes, void *stream) {
+    if (!out || !Q) return DKV_EINVAL;
+    if (!aligned16(out)) return DKV_EALIGN;
+    if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return DKV_EINVAL;  // finite, > 0
+    int64_t need;
+    dkv_status s = check_decode(cache, Q, q_dtype, n_q_heads, n_queries, workspace, ws_bytes,
+                                &need);
+    if (s != DKV_OK) return s;
+    CacheView v = view_of(cache);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *ws = static_cast<float *>(workspace);
+    cudaError_t e = dkv::launch_split(v, Q, q_dtype, n_q_heads, n_queries, softmax_scale, ws,
+                                      need, g_debug_fault, st);
+    if (e == cudaSuccess) e = dkv::launch_merge(v, n_q_heads, n_queries, out, ws, st);
+    return cuda_status(e);
 }
 
 dkv_status dkv_export_canonical(const dkv_cache *cache, uint8_t *codes, uint16_t *scales,

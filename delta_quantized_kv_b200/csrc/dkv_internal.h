@@ -25,10 +25,12 @@ cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g);
 // Floats per partial record: m[8], l[8], o[8][128].
 constexpr int PARTIAL_FLOATS = 8 + 8 + 8 * 128;
 
-cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq,
+// nq queries per sequence: query t attends to the positions before
+// seq_len - (nq - 1 - t); Q and out are [B][nq][Hq][D].
+cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq, int nq,
                          float softmax_scale, float *ws, int64_t ws_floats, int fault,
                          cudaStream_t st);
-cudaError_t launch_merge(const CacheView &cv, int Hq, float *out, const float *ws,
+cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const float *ws,
                          cudaStream_t st);
 
 }  // namespace dkv

@@ -191,6 +191,23 @@ dkv_status dkv_decode_attn_split(const dkv_cache *cache, const void *Q, int32_t 
 dkv_status dkv_decode_attn_merge(const dkv_cache *cache, int32_t n_q_heads, float *out,
                                  void *workspace, size_t ws_bytes, void *stream);
 
+/* Multi-query decode (NEXT row: several new tokens per sequence, as in
+ * speculative decoding).  The n_queries newest tokens of every sequence have
+ * been appended (dkv_append with n_new = n_queries); query t (0 <= t <
+ * n_queries) is token seq_len - n_queries + t's own query and attends to the
+ * positions before seq_len - (n_queries - 1 - t), i.e. causally.
+ * Q: [B][n_queries][n_q_heads][D] device array of q_dtype; out: the same
+ * shape in fp32.  A query with no position gets zeros.  The queries of one kv
+ * head are packed with its GQA heads into groups of 8 for the tensor cores
+ * (n_queries * G <= 8 reads the cache once; each further group of 8 reads it
+ * again).  1 <= n_queries <= 256; with n_queries = 1 this is dkv_decode_attn.
+ * Workspace: dkv_decode_workspace_bytes_mq. */
+size_t dkv_decode_workspace_bytes_mq(const dkv_cache_desc *desc, int32_t n_q_heads,
+                                     int32_t n_queries);
+dkv_status dkv_decode_attn_mq(const dkv_cache *cache, const void *Q, int32_t q_dtype,
+                              int32_t n_q_heads, int32_t n_queries, float softmax_scale,
+                              float *out, void *workspace, size_t ws_bytes, void *stream);
+
 /* Size of the library-owned scratch array used by dkv_decode_attn_noalloc. */
 #define DKV_NOALLOC_SCRATCH_BYTES (16u << 20)
 
