@@ -671,7 +671,9 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
     }
 }
 
-template <int FMT, int MODE, bool ZT, bool PAGED>
+// MQ: several causal queries per sequence (virtual heads with their own
+// position limits); the one-query instance keeps the plain tail mask.
+template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ>
 __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_kernel(SplitArgs A) {
     using Cfg = KCfg<FMT, MODE>;
     constexpr int NS = Cfg::NS, STAGE = Cfg::STAGE, NU = Cfg::NU;
@@ -860,9 +862,15 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
             int lim[NU][2];
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
-                const int us = meta.pos0 + u * (FMT == DKV_FMT_DELTA ? cv.kf : SEG);
+                if (MQ) {
+                    const int us = meta.pos0 + u * (FMT == DKV_FMT_DELTA ? cv.kf : SEG);
 #pragma unroll
-                for (int e = 0; e < 2; ++e) lim[u][e] = min(npos[u], lp[e] - us) - 4 * gq;
+                    for (int e = 0; e < 2; ++e) lim[u][e] = min(npos[u], lp[e] - us) - 4 * gq;
+                } else {
+                    // one query: lp[e] is the length (or 0 for an absent head)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) lim[u][e] = lp[e] > 0 ? npos[u] - 4 * gq : 0;
+                }
             }
             float alpha[2];
 #pragma unroll
@@ -1091,12 +1099,12 @@ static cudaError_t geom_for(SplitGeom *g) {
     if (e != cudaSuccess) return e;
     if (dev != cached_dev) {
         const size_t sm = split_smem<FMT, MODE>();
-        e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, false>,
+        e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, false, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
         int per_sm = 0, nsm = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm,
-                                                          split_kernel<FMT, MODE, ZT, false>,
+                                                          split_kernel<FMT, MODE, ZT, false, false>,
                                                           WARPS * 32, sm);
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -1124,33 +1132,41 @@ cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g) {
     return geom_for<DKV_FMT_FP16, PLAIN, false>(g);
 }
 
-// The paged instance runs on the contiguous instance's grid (the merge and the
-// workspace size follow that grid); a persistent grid is correct at any size.
+// Every instance runs on the contiguous one-query instance's grid (the merge
+// and the workspace size follow that grid); a persistent grid is correct at
+// any size.
+template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ>
+static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
+    if (PAGED || MQ) {
+        static int set_dev = -1;                 // one flag per instance
+        int dev;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev != set_dev) {
+            e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, PAGED, MQ>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)split_smem<FMT, MODE>());
+            if (e != cudaSuccess) return e;
+            set_dev = dev;
+        }
+    }
+    split_kernel<FMT, MODE, ZT, PAGED, MQ><<<ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
+    return cudaGetLastError();
+}
+
 template <int FMT, int MODE, bool ZT>
 static cudaError_t launch_split_t(const SplitArgs &a, cudaStream_t st) {
     SplitGeom g;
     cudaError_t e = geom_for<FMT, MODE, ZT>(&g);
     if (e != cudaSuccess) return e;
-    if (a.cv.pg == 0) {
-        split_kernel<FMT, MODE, ZT, false><<<g.ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
-        return cudaGetLastError();
-    }
-    if constexpr (FMT == DKV_FMT_DELTA) {
-        static int paged_dev = -1;
-        int dev;
-        e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) return e;
-        if (dev != paged_dev) {
-            e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)split_smem<FMT, MODE>());
-            if (e != cudaSuccess) return e;
-            paged_dev = dev;
-        }
-        split_kernel<FMT, MODE, ZT, true><<<g.ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
-        return cudaGetLastError();
+    const bool paged = a.cv.pg != 0, mq = a.nq > 1;
+    if (!paged && !mq) return launch_inst<FMT, MODE, ZT, false, false>(a, g.ctas, st);
+    if constexpr (FMT == DKV_FMT_DELTA) {        // only the delta format pages / takes queries
+        if (paged && mq) return launch_inst<FMT, MODE, ZT, true, true>(a, g.ctas, st);
+        if (paged) return launch_inst<FMT, MODE, ZT, true, false>(a, g.ctas, st);
+        return launch_inst<FMT, MODE, ZT, false, true>(a, g.ctas, st);
     } else {
-        return cudaErrorInvalidValue;    // only the delta format is paged
+        return cudaErrorInvalidValue;
     }
 }
 

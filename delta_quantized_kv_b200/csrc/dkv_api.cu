@@ -314,6 +314,7 @@ dkv_status dkv_decode_attn_mq(const dkv_cache *cache, const void *Q, int32_t q_d
     dkv_status s = check_decode(cache, Q, q_dtype, n_q_heads, n_queries, workspace, ws_bytes,
                                 &need);
     if (s != DKV_OK) return s;
+    if (n_queries > 1 && cache->desc.fmt != DKV_FMT_DELTA) return DKV_EUNSUPPORTED;
     CacheView v = view_of(cache);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float *ws = static_cast<float *>(workspace);

@@ -201,6 +201,7 @@ dkv_status dkv_decode_attn_merge(const dkv_cache *cache, int32_t n_q_heads, floa
  * head are packed with its GQA heads into groups of 8 for the tensor cores
  * (n_queries * G <= 8 reads the cache once; each further group of 8 reads it
  * again).  1 <= n_queries <= 256; with n_queries = 1 this is dkv_decode_attn.
+ * n_queries > 1 is for DKV_FMT_DELTA caches (DKV_EUNSUPPORTED otherwise).
  * Workspace: dkv_decode_workspace_bytes_mq. */
 size_t dkv_decode_workspace_bytes_mq(const dkv_cache_desc *desc, int32_t n_q_heads,
                                      int32_t n_queries);
