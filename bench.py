@@ -404,18 +404,22 @@ def run_ours(args, w, rank, world, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     W, K = args.warmup, args.steps
-    n_eag = W + K                        # appended tokens, per-kernel timed loop
-    n_app = 2 * (W + K)                  # ... plus the graph-launched timed loop
-    n_e2e = W + K                        # appended tokens, end-to-end loop
+    fused = args.fmt == "delta"          # the delta cache can also append inside the decode
+    # appended tokens per sequence: [0, R) eager per-kernel loop of the timed
+    # step, [R, 2R) eager loop of the fused call, [2R, 3R) the graph-timed
+    # steps, [3R, 4R) graph-timed fused calls, [4R, 5R) end to end
+    R = W + K
+    O_EAG, O_SEP, O_GRAPH, O_GSEP, O_E2E = 0, R, 2 * R, 3 * R, 4 * R
+    n_tok = 5 * R
     T0 = w.T
-    cap = T0 + n_app + n_e2e + 8
+    cap = T0 + n_tok + 8
     B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
     scale = 1.0 / math.sqrt(D)
 
     # ---- inputs (generated on the device, then only the cache stays) -------
     torch.manual_seed(1234 + rank)
     N_BATCHED = 256                      # one append call of 256 tokens per sequence
-    n_gen = max(n_app + n_e2e, N_BATCHED)
+    n_gen = max(n_tok, N_BATCHED)
     K_all = torch.empty((B, Hkv, T0 + n_gen, D), dtype=w.kv_dtype, device=dev)
     V_all = torch.empty_like(K_all)
     for b in range(B):
@@ -423,11 +427,12 @@ def run_ours(args, w, rank, world, local):
     Kp, Vp = K_all[:, :, :T0].contiguous(), V_all[:, :, :T0].contiguous()
     K256 = K_all[:, :, T0:T0 + N_BATCHED].contiguous()
     V256 = V_all[:, :, T0:T0 + N_BATCHED].contiguous()
-    app_k = [K_all[:, :, T0 + i:T0 + i + 1].contiguous() for i in range(n_app + n_e2e)]
-    app_v = [V_all[:, :, T0 + i:T0 + i + 1].contiguous() for i in range(n_app + n_e2e)]
+    app_k = [K_all[:, :, T0 + i:T0 + i + 1].contiguous() for i in range(n_tok)]
+    app_v = [V_all[:, :, T0 + i:T0 + i + 1].contiguous() for i in range(n_tok)]
     del K_all, V_all
-    qs = [S.gen_q(w, device=dev, step=i) for i in range(n_app + n_e2e)]
+    qs = [S.gen_q(w, device=dev, step=i) for i in range(n_tok)]
     in_elem = torch.finfo(w.kv_dtype).bits // 8
+    kvcode = dkv._dtype_code(w.kv_dtype)
 
     res = {}
     # ---- encode throughput (prefill of the whole context) --------------------
@@ -449,36 +454,57 @@ def run_ours(args, w, rank, world, local):
     qcode = dkv._dtype_code(w.q_dtype)
     wsb = ws.numel() * 4
 
-    def step(i, st):
-        cache.append(app_k[i], app_v[i], stream=st)
-        dkv.dkv_decode_attn_split(cache.c, qs[i], qcode, Hq, scale, ws, wsb, st)
-        dkv.dkv_decode_attn_merge(cache.c, Hq, out, ws, wsb, st)
+    # The timed step, as launches: the separate append, split and merge (the
+    # faster form of the step on B200); beside it the fused append + decode
+    # (a split kernel that first appends the token, then the merge that
+    # publishes the lengths).
+    def launches_fused(i, st):
+        return [lambda: dkv.dkv_append_decode_attn_split(cache.c, app_k[i], app_v[i], kvcode, 1,
+                                                        qs[i], qcode, Hq, scale, ws, wsb, st),
+                lambda: dkv.dkv_append_decode_attn_merge(cache.c, 1, Hq, out, ws, wsb, st)]
 
-    # ---- per-kernel times (eager launches, events between the kernels) --------
-    for i in range(W):
-        step(i, stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    with ClockSampler(local) as clk_eager:
+    def launches_sep(i, st):
+        return [lambda: cache.append(app_k[i], app_v[i], stream=st),
+                lambda: dkv.dkv_decode_attn_split(cache.c, qs[i], qcode, Hq, scale, ws, wsb, st),
+                lambda: dkv.dkv_decode_attn_merge(cache.c, Hq, out, ws, wsb, st)]
+
+    launches = launches_sep
+
+    def eager_loop(mk, off):
+        """W untimed steps, then K steps with an event between launches;
+        returns per-launch times [K][n_launches] in ms."""
+        for i in range(W):
+            for f in mk(off + i, stream):
+                f()
         torch.cuda.synchronize()
+        barrier(world)
+        n_l = len(mk(0, stream))
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_l + 1)] for _ in range(K)]
         for k in range(K):
-            i = W + k
             e = evs[k]
             e[0].record(stream)
-            cache.append(app_k[i], app_v[i])
-            e[1].record(stream)
-            dkv.dkv_decode_attn_split(cache.c, qs[i], qcode, Hq, scale, ws, wsb, stream)
-            e[2].record(stream)
-            dkv.dkv_decode_attn_merge(cache.c, Hq, out, ws, wsb, stream)
-            e[3].record(stream)
+            for j, f in enumerate(mk(off + W + k, stream)):
+                f()
+                e[j + 1].record(stream)
         torch.cuda.synchronize()
-    split_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    app_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    merge_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    eager_lens = [T0 + W + k + 1 for k in range(K)]
-    split_avg = sum(split_ms) / K
+        return [[e[j].elapsed_time(e[j + 1]) for j in range(n_l)] for e in evs]
+
+    # ---- per-kernel times of the timed step (eager launches) -----------------
+    with ClockSampler(local) as clk_eager:
+        torch.cuda.synchronize()
+        t_main = eager_loop(launches, O_EAG)
+    eager_lens = [T0 + O_EAG + W + k + 1 for k in range(K)]       # lengths decoded
+    split_avg = sum(t[1] for t in t_main) / K                     # the split kernel
     split_bytes_avg = sum(kv_bytes(args.fmt, [L] * B, Hkv, w.kf) for L in eager_lens) / K
+    app_ms = [t[0] for t in t_main]
+    split_plain = split_avg
+    kernels_us = {"append": 1e3 * sum(app_ms) / K, "split": 1e3 * split_avg,
+                  "merge": 1e3 * sum(t[2] for t in t_main) / K}
+    if fused:
+        # the fused call, for comparison (same cache, the next tokens)
+        t_fz = eager_loop(launches_fused, O_SEP)
+        kernels_us["fused_split"] = 1e3 * sum(t[0] for t in t_fz) / K
+        kernels_us["fused_merge"] = 1e3 * sum(t[1] for t in t_fz) / K
     app_bytes_avg = sum(append_bytes(args.fmt, [L - 1] * B, 1, Hkv, w.kf, in_elem)
                         for L in eager_lens) / K
 
@@ -501,43 +527,51 @@ def run_ours(args, w, rank, world, local):
                      "gbps_256_tokens": append_bytes(args.fmt, [T0] * B, N_BATCHED, Hkv, w.kf,
                                                      in_elem) / (batched_ms * 1e-3) / 1e9}
 
-    # ---- the timed steps: each step's three launches (append, split, merge)
-    # captured once as a CUDA graph, then replayed back to back -----------------
-    graphs = []
-    for i in range(n_eag, n_app):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step(i, torch.cuda.current_stream())
-        graphs.append(g)
-    for k in range(W):
-        graphs[k].replay()
-    torch.cuda.synchronize()
-    barrier(world)
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    lens = []
-    with ClockSampler(local) as clk:
+    # ---- the timed steps: each step's launches captured once as a CUDA graph,
+    # then replayed back to back -------------------------------------------------
+    def graph_run(mk, off, sampler):
+        graphs = []
+        for i in range(off, off + R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for f in mk(i, torch.cuda.current_stream()):
+                    f()
+            graphs.append(g)
+        for k in range(W):
+            graphs[k].replay()
         torch.cuda.synchronize()
         barrier(world)
-        e_start.record(stream)
-        for k in range(K):
-            graphs[W + k].replay()
-            lens.append(T0 + n_eag + W + k + 1)
-        e_end.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    del graphs
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        lens_ = []
+        with sampler:
+            torch.cuda.synchronize()
+            barrier(world)
+            e0.record(stream)
+            for k in range(K):
+                graphs[W + k].replay()
+                lens_.append(T0 + off + W + k + 1)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        del graphs
+        return max_over_ranks(e0.elapsed_time(e1), world, dev), lens_
+
+    clk = ClockSampler(local)
+    total_ms, lens = graph_run(launches, O_GRAPH, clk)
+    fused_step_ms = None
+    if fused:
+        fused_step_ms, _ = graph_run(launches_fused, O_GSEP, ClockSampler(local))
+        fused_step_ms /= K
     status = cache.device_status()
-    total_ms = e_start.elapsed_time(e_end)
-    total_ms = max_over_ranks(total_ms, world, dev)
     bytes_steps = sum(kv_bytes(args.fmt, [L] * B, Hkv, w.kf) for L in lens)
     units_steps = sum(L * B * Hkv for L in lens)
     value = world * bytes_steps / (total_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
 
     # ---- end to end through the public API with host buffers ------------------
-    pin_k = [t.cpu().pin_memory() for t in app_k[n_app:]]
-    pin_v = [t.cpu().pin_memory() for t in app_v[n_app:]]
-    pin_q = [t.cpu().pin_memory() for t in qs[n_app:]]
+    pin_k = [t.cpu().pin_memory() for t in app_k[O_E2E:]]
+    pin_v = [t.cpu().pin_memory() for t in app_v[O_E2E:]]
+    pin_q = [t.cpu().pin_memory() for t in qs[O_E2E:]]
     dk = torch.empty_like(app_k[0]); dv = torch.empty_like(app_v[0]); dq = torch.empty_like(qs[0])
     host_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
     h2d = pin_k[0].numel() * pin_k[0].element_size() * 2 + pin_q[0].numel() * pin_q[0].element_size()
@@ -560,7 +594,7 @@ def run_ours(args, w, rank, world, local):
     t0e.record(stream)
     for k in range(K):
         e2e_step(W + k)
-        lens2.append(T0 + n_app + W + k + 1)
+        lens2.append(T0 + O_E2E + W + k + 1)
     t1e.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(t0e.elapsed_time(t1e), world, dev)
@@ -587,7 +621,7 @@ def run_ours(args, w, rank, world, local):
             t = a.elapsed_time(bq) / n
             nb = kv_bytes(fmt, [T0] * B, Hkv, w.kf)
             extra[fmt] = {"split_us": 1e3 * t, "bytes": nb, "gbps": nb / (t * 1e-3) / 1e9,
-                          "speedup_delta_vs": t / split_avg}
+                          "speedup_delta_vs": t / split_plain}
             del cc
         # the same decode through a paged cache: pages of 16 groups (512 tokens)
         # in a shuffled pool, every record reached through the block table
@@ -631,7 +665,7 @@ def run_ours(args, w, rank, world, local):
             bq.record(stream)
             torch.cuda.synchronize()
             t = a.elapsed_time(bq) / n
-            nb = kv_bytes("delta", [T0 + n_app + n_e2e] * B, Hkv, w.kf)
+            nb = kv_bytes("delta", [T0 + n_tok] * B, Hkv, w.kf)
             extra["delta_2_queries"] = {"decode_attn_us": 1e3 * t, "bytes": nb,
                                         "gbps": nb / (t * 1e-3) / 1e9}
         # reconstruction MSE on a slice (first 2 batch entries)
@@ -691,8 +725,8 @@ def run_ours(args, w, rank, world, local):
                      "algorithmic_bytes": split_bytes_avg,
                      "kernel": "split_kernel (decode split)",
                      "peak_kind": f"{peak_kind} (copy bandwidth, MEASURED_PEAKS hbm_gbs)"},
-        "kernels_us": {"append": 1e3 * sum(app_ms) / K, "split": 1e3 * split_avg,
-                       "merge": 1e3 * sum(merge_ms) / K},
+        "kernels_us": kernels_us,
+        "step_fused_call_us": None if fused_step_ms is None else 1e3 * fused_step_ms,
         "encode": res["encode"],
         "append": res["append"],
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,

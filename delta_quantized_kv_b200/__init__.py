@@ -54,7 +54,9 @@ EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode",
            "dkv_decode_attn_merge", "dkv_export_canonical", "dkv_dequantize",
            "dkv_get_device_status", "dkv_status_str", "dkv_decode_attn_noalloc",
            "dkv_debug_set_fault", "dkv_cache_meta_bytes", "dkv_page_bytes",
-           "dkv_cache_init_paged", "dkv_decode_workspace_bytes_mq", "dkv_decode_attn_mq"]
+           "dkv_cache_init_paged", "dkv_decode_workspace_bytes_mq", "dkv_decode_attn_mq",
+           "dkv_append_decode_attn", "dkv_append_decode_attn_split",
+           "dkv_append_decode_attn_merge"]
 
 
 def load():
@@ -90,6 +92,9 @@ def load():
         "dkv_cache_init_paged": ([PD, I, P, ctypes.c_int64, P, I, P, S, PC, P], I),
         "dkv_decode_workspace_bytes_mq": ([PD, I, I], S),
         "dkv_decode_attn_mq": ([PC, P, I, I, I, F, P, P, S, P], I),
+        "dkv_append_decode_attn": ([PC, P, P, I, I, P, I, I, F, P, P, S, P], I),
+        "dkv_append_decode_attn_split": ([PC, P, P, I, I, P, I, I, F, P, S, P], I),
+        "dkv_append_decode_attn_merge": ([PC, I, I, P, P, S, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -202,6 +207,31 @@ def dkv_decode_attn_mq(cache: dkv_cache, Q, q_dtype, n_q_heads, n_queries, softm
     _check(load().dkv_decode_attn_mq(ctypes.byref(cache), _ptr(Q), q_dtype, n_q_heads, n_queries,
                                      softmax_scale, _ptr(out), _ptr(workspace), ws_bytes,
                                      _stream(stream)), "dkv_decode_attn_mq")
+
+
+def dkv_append_decode_attn(cache: dkv_cache, K_new, V_new, kv_dtype, n_new, Q, q_dtype,
+                           n_q_heads, softmax_scale, out, workspace, ws_bytes,
+                           stream=None) -> None:
+    _check(load().dkv_append_decode_attn(ctypes.byref(cache), _ptr(K_new), _ptr(V_new), kv_dtype,
+                                         n_new, _ptr(Q), q_dtype, n_q_heads, softmax_scale,
+                                         _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "dkv_append_decode_attn")
+
+
+def dkv_append_decode_attn_split(cache: dkv_cache, K_new, V_new, kv_dtype, n_new, Q, q_dtype,
+                                 n_q_heads, softmax_scale, workspace, ws_bytes,
+                                 stream=None) -> None:
+    _check(load().dkv_append_decode_attn_split(ctypes.byref(cache), _ptr(K_new), _ptr(V_new),
+                                               kv_dtype, n_new, _ptr(Q), q_dtype, n_q_heads,
+                                               softmax_scale, _ptr(workspace), ws_bytes,
+                                               _stream(stream)), "dkv_append_decode_attn_split")
+
+
+def dkv_append_decode_attn_merge(cache: dkv_cache, n_new, n_q_heads, out, workspace, ws_bytes,
+                                 stream=None) -> None:
+    _check(load().dkv_append_decode_attn_merge(ctypes.byref(cache), n_new, n_q_heads, _ptr(out),
+                                               _ptr(workspace), ws_bytes, _stream(stream)),
+           "dkv_append_decode_attn_merge")
 
 
 def dkv_decode_attn_split(cache: dkv_cache, Q, q_dtype, n_q_heads, softmax_scale, workspace,
@@ -332,6 +362,18 @@ class Cache:
                         ws.numel() * 4, stream)
         return out
 
+    def workspace_mq(self, n_q_heads, n_queries):
+        import torch
+        key = ("mq", n_q_heads, n_queries)
+        ws = getattr(self, "_ws_mq", {}).get(key)
+        if ws is None:
+            nb = dkv_decode_workspace_bytes_mq(self.desc, n_q_heads, n_queries)
+            if nb == 0:
+                raise DkvError(DKV_EINVAL, "dkv_decode_workspace_bytes_mq")
+            ws = torch.zeros(nb // 4 + 64, dtype=torch.float32, device=self.device)
+            self._ws_mq = {key: ws}
+        return ws
+
     def decode_attn_mq(self, Q, softmax_scale, out=None, stream=None):
         """Q: [B, n_queries, Hq, D]; query t attends causally (see
         dkv_decode_attn_mq).  Returns fp32 [B, n_queries, Hq, D]."""
@@ -339,16 +381,28 @@ class Cache:
         B, nq, Hq, Dh = Q.shape
         if out is None:
             out = torch.empty((B, nq, Hq, Dh), dtype=torch.float32, device=Q.device)
-        key = ("mq", Hq, nq)
-        ws = getattr(self, "_ws_mq", {}).get(key)
-        if ws is None:
-            nb = dkv_decode_workspace_bytes_mq(self.desc, Hq, nq)
-            if nb == 0:
-                raise DkvError(DKV_EINVAL, "dkv_decode_workspace_bytes_mq")
-            ws = torch.zeros(nb // 4 + 64, dtype=torch.float32, device=self.device)
-            self._ws_mq = {key: ws}
+        ws = self.workspace_mq(Hq, nq)
         dkv_decode_attn_mq(self.c, Q.contiguous(), _dtype_code(Q.dtype), Hq, nq, softmax_scale,
                            out, ws, ws.numel() * 4, stream)
+        return out
+
+    def append_decode_attn(self, K_new, V_new, Q, softmax_scale, out=None, stream=None):
+        """Fused append + decode (dkv_append_decode_attn): K_new, V_new
+        [B, Hkv, n_new, D]; Q [B, Hq, D] (n_new = 1) or [B, n_new, Hq, D].
+        Returns fp32 of Q's shape."""
+        import torch
+        n_new = K_new.shape[2]
+        Hq = Q.shape[-2]
+        if Q.dim() == 3 and n_new != 1:
+            raise ValueError("Q of shape [B, Hq, D] takes one new token per sequence")
+        if Q.dim() == 4 and Q.shape[1] != n_new:
+            raise ValueError("Q must hold one query per new token")
+        if out is None:
+            out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+        ws = self.workspace_mq(Hq, n_new)
+        dkv_append_decode_attn(self.c, K_new, V_new, _dtype_code(K_new.dtype), n_new,
+                               Q.contiguous(), _dtype_code(Q.dtype), Hq, softmax_scale, out, ws,
+                               ws.numel() * 4, stream)
         return out
 
     def seq_lens(self):

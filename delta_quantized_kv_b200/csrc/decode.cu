@@ -90,16 +90,6 @@ template <int FMT, int MODE> struct SmemMap {
     static_assert(BYTES <= 227 * 1024, "shared memory per CTA");
 };
 
-struct SplitArgs {
-    CacheView cv;
-    const void *Q;
-    int q_dtype;
-    int Hq, G, NHG;            // query heads, heads per kv head, head groups of 8
-    int nq;                    // queries per sequence (the newest nq tokens' own, causal)
-    float scale_log2;          // softmax_scale * log2(e), > 0
-    float *ws;                 // partial records
-    int fault;                 // test support: 1 = arm the copy barriers but issue no copy
-};
 
 __host__ __device__ inline int units_of(int fmt, int kf, int len) {
     if (len <= 0) return 0;
@@ -114,9 +104,34 @@ __host__ __device__ inline int64_t warp_of(int64_t x, int64_t NW, int64_t T) {
     return ((x + 1) * NW - 1) / T;
 }
 
+struct SplitArgs {
+    CacheView cv;
+    const void *Q;
+    int q_dtype;
+    int Hq, G, NHG;            // query heads, heads per kv head, head groups of 8
+    int nq;                    // queries per sequence (the newest nq tokens' own, causal)
+    float scale_log2;          // softmax_scale * log2(e), > 0
+    float *ws;                 // partial records
+    int fault;                 // test support: 1 = arm the copy barriers but issue no copy
+    // fused append (cv.len_add = n > 0): the n new tokens of each sequence,
+    // [B][Hkv][n][D] of kv_dtype
+    const void *Kn, *Vn;
+    int kv_dtype;
+};
+
+// Stored length of batch entry b, and whether the entry takes the call's new
+// tokens (fused append): its length is valid and the tokens fit.
+__device__ inline bool takes_append(const CacheView &cv, int b, int &l) {
+    l = cv.seqlen[b];
+    return l >= 0 && l <= cv.cap && l + cv.len_add <= cv.cap;
+}
+
+// Length decoded for batch entry b: 0 for an invalid stored length; with a
+// fused append, the stored length plus the new tokens when they fit.
 __device__ inline int clamp_len(const CacheView &cv, int b) {
     int l = cv.seqlen[b];
-    return (l < 0 || l > cv.cap) ? 0 : l;
+    if (l < 0 || l > cv.cap) return 0;
+    return l + cv.len_add <= cv.cap ? l + cv.len_add : l;
 }
 
 // Iterates the (unit, segment) stage items of one warp's range in order.
@@ -211,6 +226,12 @@ __device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs, int 
         c.seq = seq_ptr(cv, c.b, c.vs, nhg);
     }
     if (MODE == PREFIX) c.nseg = nseg_of<MODE>(cv, c.len_b, c.g);
+}
+
+// Fused append: the lengths the split kernel decoded, int32[B], after the
+// partial records of the workspace (NW warp slots + one per sequence).
+__host__ __device__ inline int32_t *merge_lengths(float *ws, int64_t NW, int64_t nseq) {
+    return reinterpret_cast<int32_t *>(ws + (NW + nseq) * PARTIAL_FLOATS);
 }
 
 // What the consumer needs to know about a stage, written next to the stage by
@@ -671,10 +692,177 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
     }
 }
 
+// ---------------------------------------------------------------------------
+// Fused append (delta format).  The n new tokens of sequence (b, kv head) are
+// quantised inside the split kernel by the warps whose unit ranges hold the
+// groups they land in, before those warps copy any record: each such warp runs
+// the closed loop of the method (page "...Delta-KV", section "핵심 아이디어":
+// keyframe at p mod kf == 0, else a Q4_0 delta from the reconstruction of
+// p - 1) over the new tokens from the stored reconstruction, and stores the
+// fields of the positions in its own groups.  Every quantiser step is the
+// encoder's, in the same order, so the stored fields are the ones the
+// separate append would write.  A warp of another head group of the same kv
+// head (multi-query, more than 8 virtual heads) stores the same bytes again;
+// each warp reads the records only after its own stores.  The reconstruction
+// after the last token goes to the other state slot, which the merge makes
+// current.
+// ---------------------------------------------------------------------------
+// Input element c of row `row` of an n-token K_new / V_new array.
+__device__ inline float load_new(const void *src, int dtype, int64_t row, int c) {
+    const int64_t i = row * D + c;
+    if (dtype == DKV_F16) return __half2float(__ldg(static_cast<const __half *>(src) + i));
+    if (dtype == DKV_BF16)
+        return __bfloat162float(__ldg(static_cast<const __nv_bfloat16 *>(src) + i));
+    return __ldg(static_cast<const float *>(src) + i);
+}
+
+template <bool PAGED>
+__device__ __noinline__ void append_tokens(const SplitArgs &A, int b, int kvh, int L0, int g_lo,
+                                           int g_hi, bool write_state) {
+    const CacheView &cv = A.cv;
+    const int lane = threadIdx.x & 31, kf = cv.kf, n = cv.len_add;
+    const int64_t sb = ((int64_t)b * cv.Hkv + kvh) * 2 * D;          // (b, kvh) in a slot
+    const int64_t slot = (int64_t)cv.B * cv.Hkv * 2 * D;
+    const int64_t row0 = ((int64_t)b * cv.Hkv + kvh) * n;
+    // one round trip: the slot word, both state slots and the first token
+    const int parity = cv.header[2] & 1;
+    const bool cont = (L0 % kf) != 0;            // the first token continues a group
+    float s0[2][4], s1[2][4], x[2][4];
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t e = sb + t * D + 32 * j + lane;
+            s0[t][j] = cont ? __ldg(cv.state + e) : 0.f;
+            s1[t][j] = cont ? __ldg(cv.state + slot + e) : 0.f;
+            x[t][j] = load_new(t ? A.Vn : A.Kn, A.kv_dtype, row0, 32 * j + lane);
+        }
+    float xh[2][4];                     // reconstruction of channels 32 j + lane, K and V
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xh[t][j] = parity ? s1[t][j] : s0[t][j];
+    float *st_new = cv.state + (parity ^ 1) * slot + sb;
+    // this lane's nibble word: K word `lane` (lanes 0-15) or V word lane - 16
+    const int wt = lane >> 4, ww = lane & 15;
+#pragma unroll 1
+    for (int i = 0; i < n; ++i) {
+        const int p = L0 + i, g = p / kf, di = p - g * kf;   // di 0: keyframe; else delta di - 1
+        if (g > g_hi) break;
+        uint8_t *rec = g >= g_lo ? rec_ptr<PAGED>(cv, b, kvh, g) : nullptr;
+        if (di == 0) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const __half h = __float2half_rn(x[t][j]);
+                    xh[t][j] = __half2float(h);
+                    const int ch = 32 * j + lane;
+                    if (rec)
+                        reinterpret_cast<__half *>(rec + t * 256)[t == 0 ? k_half_idx(ch)
+                                                                         : v_half_idx(ch)] = h;
+                }
+        } else {
+            // the eight blocks (K and V, 4 each) are independent chains
+            uint32_t codes = 0;         // code of channel 32 j + lane of tensor t at bit 16 t + 4 j
+            __half d16[2][4];
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int code = quant_lane(__fsub_rn(x[t][j], xh[t][j]), &d16[t][j]);
+                    codes |= (uint32_t)code << (16 * t + 4 * j);
+                    xh[t][j] = __fadd_rn(xh[t][j],
+                                         __fmul_rn((float)(code - 8), __half2float(d16[t][j])));
+                }
+            if (rec) {
+                // gather the 8 codes of this lane's word from the lanes holding them
+                uint32_t word = 0;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int ch = nib_channel(wt, ww, k);
+                    const uint32_t v = __shfl_sync(0xffffffffu, codes, ch & 31);
+                    word |= ((v >> (16 * wt + 4 * (ch >> 5))) & 15u) << (4 * k);
+                }
+                uint8_t *nib = rec + KF_BYTES + (int64_t)(kf - 1) * SC_BYTES +
+                               ((int64_t)wt * (kf - 1) + (di - 1)) * NIB_BYTES;
+                reinterpret_cast<uint32_t *>(nib)[ww] = word;
+                if (lane < 2) {
+                    uint2 v;
+                    v.x = (uint32_t)__half_as_ushort(d16[lane][0]) |
+                          ((uint32_t)__half_as_ushort(d16[lane][1]) << 16);
+                    v.y = (uint32_t)__half_as_ushort(d16[lane][2]) |
+                          ((uint32_t)__half_as_ushort(d16[lane][3]) << 16);
+                    *reinterpret_cast<uint2 *>(rec + KF_BYTES + (int64_t)(di - 1) * SC_BYTES +
+                                               lane * 8) = v;
+                }
+            }
+        }
+        if (i + 1 < n) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    x[t][j] = load_new(t ? A.Vn : A.Kn, A.kv_dtype, row0 + i + 1, 32 * j + lane);
+        }
+    }
+    if (write_state) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) st_new[t * D + 32 * j + lane] = xh[t][j];
+    }
+}
+
+// The new tokens that land in units [lo, hi) of a warp's range (offsets from
+// the range's first unit, which is group g0 of sequence vs of batch entry b,
+// a sequence of ub units): walk the sequences those units belong to and
+// quantise, for each, the new tokens of the groups held there.  The owner of a
+// sequence's last group (head group 0) writes the state.  Returns whether this
+// warp stored anything.
+template <bool PAGED>
+__device__ __noinline__ bool append_range(const SplitArgs &A, int nvs, int b, int vs, int g0,
+                                          int ub, int64_t lo, int64_t hi) {
+    const CacheView &cv = A.cv;
+    bool wrote = false;
+    int64_t off = 0;                    // offset of group g0 of (b, vs) in the range
+#pragma unroll 1
+    while (off < hi) {
+        const int64_t seg = ub - g0;    // units of this sequence from g0 on
+        if (off + seg > lo) {
+            const int ga = g0 + (int)max((int64_t)0, lo - off);
+            const int gb = g0 + (int)(min(hi, off + seg) - off) - 1;
+            int L;
+            if (takes_append(cv, b, L)) {
+                const int first = max(ga, L / cv.kf);
+                if (first <= gb) {
+                    append_tokens<PAGED>(A, b, A.NHG == 1 ? vs : vs / A.NHG, L, first, gb,
+                                         gb == ub - 1 && vs % A.NHG == 0);
+                    wrote = true;
+                }
+            }
+        }
+        off += seg;
+        if (off >= hi) break;
+        g0 = 0;
+        if (++vs == nvs) {
+            vs = 0;
+            do {
+                if (++b >= cv.B) return wrote;
+                ub = units_of(cv.fmt, cv.kf, clamp_len(cv, b));
+            } while (ub == 0);
+        }
+    }
+    return wrote;
+}
+
 // MQ: several causal queries per sequence (virtual heads with their own
-// position limits); the one-query instance keeps the plain tail mask.
-template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ>
-__global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_kernel(SplitArgs A) {
+// position limits); the one-query instance keeps the plain tail mask.  APP:
+// the fused append (the kernel parameters stay in the constant bank while the
+// append functions take their address).
+template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP>
+__global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB))
+    split_kernel(const __grid_constant__ SplitArgs A) {
     using Cfg = KCfg<FMT, MODE>;
     constexpr int NS = Cfg::NS, STAGE = Cfg::STAGE, NU = Cfg::NU;
     using Map = SmemMap<FMT, MODE>;
@@ -704,10 +892,32 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
     int bdummy;
     int64_t base_dummy;
     const int64_t total = locate(cv, nvs, -1, bdummy, base_dummy);
-    if (gw == 0 && lane == 0) {
-        for (int b = 0; b < cv.B; ++b) {
-            const int l = cv.seqlen[b];
-            if (l < 0 || l > cv.cap) set_status(cv.header, DKV_DEV_BAD_SEQLEN);
+    if constexpr (APP) {
+        if (gw == 0) {
+            // the lengths this call decodes, for the merge (which publishes
+            // the new ones); an entry that takes no tokens keeps its
+            // reconstruction: carry it into the slot the merge makes current
+            int32_t *lenv = merge_lengths(A.ws, NW, cv.B * nvs);
+            for (int b = lane; b < cv.B; b += 32) lenv[b] = clamp_len(cv, b);
+            const int parity = cv.header[2] & 1;
+            const int64_t per_b = (int64_t)cv.Hkv * 2 * D;
+            for (int b = 0; b < cv.B; ++b) {
+                int l;
+                if (takes_append(cv, b, l)) continue;
+                if (lane == 0)
+                    set_status(cv.header, (l < 0 || l > cv.cap) ? DKV_DEV_BAD_SEQLEN
+                                                                : DKV_DEV_CAPACITY);
+                const float *so = cv.state + ((int64_t)parity * cv.B + b) * per_b;
+                float *sn = cv.state + ((int64_t)(parity ^ 1) * cv.B + b) * per_b;
+                for (int64_t k = lane; k < per_b; k += 32) sn[k] = so[k];
+            }
+        }
+    } else {
+        if (gw == 0 && lane == 0) {
+            for (int b = 0; b < cv.B; ++b) {
+                const int l = cv.seqlen[b];
+                if (l < 0 || l > cv.cap) set_status(cv.header, DKV_DEV_BAD_SEQLEN);
+            }
         }
     }
     if (total == 0) return;
@@ -716,6 +926,18 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
 
     Cursor ic;
     cursor_seek<MODE>(ic, cv, nvs, A.NHG, r0, r1 - r0);
+    // fused append: tokens landing in the units the first NS stages can hold
+    // are stored before those copies are issued; the rest after, while the
+    // first copies are in flight (each warp copies a record only after its
+    // own stores and a proxy fence)
+    const int ab = ic.b, avs = ic.vs, ag = ic.g, aub = ic.units_b;
+    constexpr int64_t PRE = (int64_t)NS * NU;
+    if constexpr (APP) {
+        if (append_range<PAGED>(A, nvs, ab, avs, ag, aub, 0, min(PRE, r1 - r0))) {
+            fence_proxy_async_global();
+            __syncwarp();
+        }
+    }
 
     // prologue: fill the ring
     uint32_t phase = 0;                 // bit s = parity to wait for on stage s
@@ -727,6 +949,13 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
             pend = next_stage<FMT, MODE, PAGED>(cv, ic, nvs, A.NHG, mystages + s * STAGE, mybar + s,
                                          mymeta + s, lane, A.fault);
             ++issued;
+        }
+    }
+    if constexpr (APP) {
+        if (r1 - r0 > PRE &&
+            append_range<PAGED>(A, nvs, ab, avs, ag, aub, PRE, r1 - r0)) {
+            fence_proxy_async_global();
+            __syncwarp();
         }
     }
 
@@ -1004,11 +1233,21 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB)) split_ker
 // ---------------------------------------------------------------------------
 // merge: grid (nq * Hq, B), 128 threads (one per channel); block x is query
 // t = x / Hq, head h = x % Hq, i.e. virtual head t * G + h % G of kv head h / G
-__global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G, int NHG, int nq,
-                                                    int64_t NW, const float *ws, float *out) {
+// Length decoded for batch entry b: from the stored lengths, or (fused
+// append) from the copy the split kernel left in the workspace.
+template <bool FIN>
+__device__ inline int merge_len(const CacheView &cv, const int32_t *lenv, int b) {
+    if constexpr (FIN) return lenv[b];
+    else return clamp_len(cv, b);
+}
+
+template <bool FIN>
+__device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, int nq, int64_t NW,
+                                  const float *ws, float *out) {
     const int t = blockIdx.x / Hq, h = blockIdx.x % Hq, b = blockIdx.y, c = threadIdx.x;
     const int nvs = cv.Hkv * NHG;
-    const int len = clamp_len(cv, b);
+    const int32_t *lenv = FIN ? merge_lengths(const_cast<float *>(ws), NW, cv.B * nvs) : nullptr;
+    const int len = merge_len<FIN>(cv, lenv, b);
     const int ub = units_of(cv.fmt, cv.kf, len);
     float *dst = out + (((int64_t)b * nq + t) * Hq + h) * D;
     if (ub == 0) {                      // uniform over the block
@@ -1020,17 +1259,20 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
     // the warps whose unit ranges touch this sequence: found once per block
     __shared__ int64_t sh_w0, sh_w1, sh_total;
     if (threadIdx.x < 32) {
-        int bb;
-        int64_t bdummy;
-        const int64_t total = locate(cv, nvs, -1, bb, bdummy);
-        // units of the batch entries before b
-        int64_t mine = 0;
-        for (int b0 = 0; b0 < b; b0 += 32) {
+        // units of all batch entries, and of those before b
+        int64_t total = 0, mine = 0;
+        for (int b0 = 0; b0 < cv.B; b0 += 32) {
             const int xb = b0 + (int)threadIdx.x;
-            int64_t u = xb < b ? (int64_t)nvs * units_of(cv.fmt, cv.kf, clamp_len(cv, xb)) : 0;
+            int64_t u = xb < cv.B ? (int64_t)nvs * units_of(cv.fmt, cv.kf,
+                                                            merge_len<FIN>(cv, lenv, xb)) : 0;
+            int64_t ub4 = xb < b ? u : 0;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
-            mine += u;
+            for (int o = 16; o > 0; o >>= 1) {
+                u += __shfl_xor_sync(0xffffffffu, u, o);
+                ub4 += __shfl_xor_sync(0xffffffffu, ub4, o);
+            }
+            total += u;
+            mine += ub4;
         }
         if (threadIdx.x == 0) {
             const int64_t xs = mine + (int64_t)vsl * ub, xe = xs + ub;
@@ -1083,6 +1325,22 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
     dst[c] = L > 0.f ? O / L : 0.f;     // a causal query with no position gets 0
 }
 
+template <bool FIN>
+__global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G, int NHG, int nq,
+                                                    int64_t NW, const float *ws, float *out) {
+    merge_body<FIN>(cv, Hq, G, NHG, nq, NW, ws, out);
+    if constexpr (FIN) {
+        // fused append: publish batch entry b's new length (no other block of
+        // this launch reads it) and make the state slot the split kernel
+        // wrote current
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
+            int l;
+            if (takes_append(cv, blockIdx.y, l)) cv.seqlen[blockIdx.y] = l + cv.len_add;
+            if (blockIdx.y == 0) cv.header[2] ^= 1;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -1099,12 +1357,12 @@ static cudaError_t geom_for(SplitGeom *g) {
     if (e != cudaSuccess) return e;
     if (dev != cached_dev) {
         const size_t sm = split_smem<FMT, MODE>();
-        e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, false, false>,
+        e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, false, false, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
         int per_sm = 0, nsm = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm,
-                                                          split_kernel<FMT, MODE, ZT, false, false>,
+                                                          split_kernel<FMT, MODE, ZT, false, false, false>,
                                                           WARPS * 32, sm);
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -1135,36 +1393,43 @@ cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g) {
 // Every instance runs on the contiguous one-query instance's grid (the merge
 // and the workspace size follow that grid); a persistent grid is correct at
 // any size.
-template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ>
+template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP>
 static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
-    if (PAGED || MQ) {
+    if (PAGED || MQ || APP) {
         static int set_dev = -1;                 // one flag per instance
         int dev;
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
         if (dev != set_dev) {
-            e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, PAGED, MQ>,
+            e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, PAGED, MQ, APP>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)split_smem<FMT, MODE>());
             if (e != cudaSuccess) return e;
             set_dev = dev;
         }
     }
-    split_kernel<FMT, MODE, ZT, PAGED, MQ><<<ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
+    split_kernel<FMT, MODE, ZT, PAGED, MQ, APP><<<ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
     return cudaGetLastError();
 }
 
 template <int FMT, int MODE, bool ZT>
-static cudaError_t launch_split_t(const SplitArgs &a, cudaStream_t st) {
+static cudaError_t launch_split_t(const SplitArgs &a_in, cudaStream_t st) {
     SplitGeom g;
     cudaError_t e = geom_for<FMT, MODE, ZT>(&g);
     if (e != cudaSuccess) return e;
-    const bool paged = a.cv.pg != 0, mq = a.nq > 1;
-    if (!paged && !mq) return launch_inst<FMT, MODE, ZT, false, false>(a, g.ctas, st);
+    const SplitArgs &a = a_in;
+    const bool paged = a.cv.pg != 0, mq = a.nq > 1, app = a.cv.len_add > 0;
+    if (!paged && !mq && !app) return launch_inst<FMT, MODE, ZT, false, false, false>(a, g.ctas, st);
     if constexpr (FMT == DKV_FMT_DELTA) {        // only the delta format pages / takes queries
-        if (paged && mq) return launch_inst<FMT, MODE, ZT, true, true>(a, g.ctas, st);
-        if (paged) return launch_inst<FMT, MODE, ZT, true, false>(a, g.ctas, st);
-        return launch_inst<FMT, MODE, ZT, false, true>(a, g.ctas, st);
+        if (app) {
+            if (paged && mq) return launch_inst<FMT, MODE, ZT, true, true, true>(a, g.ctas, st);
+            if (paged) return launch_inst<FMT, MODE, ZT, true, false, true>(a, g.ctas, st);
+            if (mq) return launch_inst<FMT, MODE, ZT, false, true, true>(a, g.ctas, st);
+            return launch_inst<FMT, MODE, ZT, false, false, true>(a, g.ctas, st);
+        }
+        if (paged && mq) return launch_inst<FMT, MODE, ZT, true, true, false>(a, g.ctas, st);
+        if (paged) return launch_inst<FMT, MODE, ZT, true, false, false>(a, g.ctas, st);
+        return launch_inst<FMT, MODE, ZT, false, true, false>(a, g.ctas, st);
     } else {
         return cudaErrorInvalidValue;
     }
@@ -1172,10 +1437,13 @@ static cudaError_t launch_split_t(const SplitArgs &a, cudaStream_t st) {
 
 cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq, int nq,
                          float softmax_scale, float *ws, int64_t ws_floats, int fault,
-                         cudaStream_t st) {
+                         cudaStream_t st, const void *K_new, const void *V_new, int kv_dtype) {
     (void)ws_floats;
     SplitArgs a;
     a.fault = fault;
+    a.Kn = K_new;
+    a.Vn = V_new;
+    a.kv_dtype = kv_dtype;
     a.cv = cv;
     a.Q = Q;
     a.q_dtype = q_dtype;
@@ -1202,8 +1470,11 @@ cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const 
     const int G = Hq / cv.Hkv;
     const int NHG = (nq * G + 7) / 8;
     dim3 grid(nq * Hq, cv.B);
-    merge_kernel<<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, (int64_t)g.ctas * g.warps_per_cta, ws,
-                                       out);
+    const int64_t NW = (int64_t)g.ctas * g.warps_per_cta;
+    if (cv.len_add > 0)
+        merge_kernel<true><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+    else
+        merge_kernel<false><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
     return cudaGetLastError();
 }
 

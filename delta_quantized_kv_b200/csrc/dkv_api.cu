@@ -108,6 +108,7 @@ CacheView view_of(const dkv_cache *c) {
     v.cap = c->desc.max_ctx;
     v.fmt = c->desc.fmt;
     v.n_groups = c->n_groups;
+    v.len_add = 0;
     return v;
 }
 
@@ -129,7 +130,8 @@ int64_t workspace_floats(const dkv_cache_desc *d, int32_t Hq, int32_t nq, bool *
     const int64_t nhg = ((int64_t)nq * G + 7) / 8;
     const int64_t slots = (int64_t)g.ctas * g.warps_per_cta + (int64_t)d->batch * d->n_kv_heads * nhg;
     *ok = true;
-    return slots * dkv::PARTIAL_FLOATS;
+    // + the decoded lengths of a fused append + decode, int32[B]
+    return slots * dkv::PARTIAL_FLOATS + ((int64_t)d->batch + 3) / 4 * 4;
 }
 
 dkv_status check_decode(const dkv_cache *cache, const void *Q, int32_t q_dtype, int32_t Hq,
@@ -322,6 +324,60 @@ dkv_status dkv_decode_attn_mq(const dkv_cache *cache, const void *Q, int32_t q_d
                                       need, g_debug_fault, st);
     if (e == cudaSuccess) e = dkv::launch_merge(v, n_q_heads, n_queries, out, ws, st);
     return cuda_status(e);
+}
+
+dkv_status dkv_append_decode_attn_split(dkv_cache *cache, const void *K_new, const void *V_new,
+                                        int32_t kv_dtype, int32_t n_new, const void *Q,
+                                        int32_t q_dtype, int32_t n_q_heads, float softmax_scale,
+                                        void *workspace, size_t ws_bytes, void *stream) {
+    if (!Q || !K_new || !V_new || !valid_dtype(kv_dtype)) return DKV_EINVAL;
+    if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return DKV_EINVAL;  // finite, > 0
+    if (!aligned16(K_new) || !aligned16(V_new)) return DKV_EALIGN;
+    dkv_status s = check_cache(cache);
+    if (s != DKV_OK) return s;
+    if (cache->desc.fmt != DKV_FMT_DELTA) return DKV_EUNSUPPORTED;
+    int64_t need;
+    s = check_decode(cache, Q, q_dtype, n_q_heads, n_new, workspace, ws_bytes, &need);
+    if (s != DKV_OK) return s;
+    if (n_new > cache->desc.max_ctx) return DKV_ECAPACITY;
+    CacheView v = view_of(cache);
+    v.len_add = n_new;
+    return cuda_status(dkv::launch_split(v, Q, q_dtype, n_q_heads, n_new, softmax_scale,
+                                         static_cast<float *>(workspace), need, g_debug_fault,
+                                         static_cast<cudaStream_t>(stream), K_new, V_new,
+                                         kv_dtype));
+}
+
+dkv_status dkv_append_decode_attn_merge(dkv_cache *cache, int32_t n_new, int32_t n_q_heads,
+                                        float *out, void *workspace, size_t ws_bytes,
+                                        void *stream) {
+    if (!out) return DKV_EINVAL;
+    if (!aligned16(out)) return DKV_EALIGN;
+    dkv_status s = check_cache(cache);
+    if (s != DKV_OK) return s;
+    if (cache->desc.fmt != DKV_FMT_DELTA) return DKV_EUNSUPPORTED;
+    int64_t need;
+    s = check_decode(cache, nullptr, -1, n_q_heads, n_new, workspace, ws_bytes, &need);
+    if (s != DKV_OK) return s;
+    if (n_new > cache->desc.max_ctx) return DKV_ECAPACITY;
+    CacheView v = view_of(cache);
+    v.len_add = n_new;
+    return cuda_status(dkv::launch_merge(v, n_q_heads, n_new, out,
+                                         static_cast<const float *>(workspace),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+dkv_status dkv_append_decode_attn(dkv_cache *cache, const void *K_new, const void *V_new,
+                                  int32_t kv_dtype, int32_t n_new, const void *Q,
+                                  int32_t q_dtype, int32_t n_q_heads, float softmax_scale,
+                                  float *out, void *workspace, size_t ws_bytes, void *stream) {
+    if (!out) return DKV_EINVAL;
+    if (!aligned16(out)) return DKV_EALIGN;
+    dkv_status s = dkv_append_decode_attn_split(cache, K_new, V_new, kv_dtype, n_new, Q, q_dtype,
+                                                n_q_heads, softmax_scale, workspace, ws_bytes,
+                                                stream);
+    if (s != DKV_OK) return s;
+    return dkv_append_decode_attn_merge(cache, n_new, n_q_heads, out, workspace, ws_bytes, stream);
 }
 
 dkv_status dkv_export_canonical(const dkv_cache *cache, uint8_t *codes, uint16_t *scales,

@@ -74,6 +74,17 @@ __host__ __device__ inline int v_half_idx(int c) {
     return g * 16 + 2 * mt + e;
 }
 
+// Channel held by nibble i (0..7) of word w (0..15) of one position's nibble
+// row of tensor t: the inverse of k_nib_pos (K) / v_nib_pos (V).
+__host__ __device__ inline int nib_channel(int t, int w, int i) {
+    if (t == 0) {
+        const int tt = w >> 2, j = w & 3, h = i >> 2, s2 = (i >> 1) & 1, e = i & 1;
+        return 32 * j + 16 * s2 + 8 * e + 2 * tt + h;
+    }
+    const int g = w >> 1, u = w & 1, mt = 4 * u + (i >> 1);
+    return 16 * mt + g + 8 * (i & 1);
+}
+
 // Device-side cache view passed by value to kernels.
 struct CacheView {
     uint8_t *data;
@@ -88,6 +99,9 @@ struct CacheView {
     const int32_t *bt;     // [B][maxp] page indices
     int64_t page_bytes, n_pages;
     int32_t pg, maxp;
+    // fused append + decode: tokens each sequence takes in this call (0:
+    // none); a sequence whose tokens fit is decoded at its stored length + this
+    int32_t len_add;
 };
 
 __device__ inline void set_status(int32_t *header, int bits) {
@@ -127,6 +141,10 @@ __device__ inline void fence_mbar_init() {
 }
 __device__ inline void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+// orders this thread's generic-proxy global stores before later bulk copies
+__device__ inline void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;\n" ::: "memory");
 }
 __device__ inline void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
@@ -258,6 +276,33 @@ __device__ inline void dq_pair(uint32_t w, uint32_t m1024, uint32_t m64, uint32_
     dq_pair_biased(w, m1024, m64, lo, hi);
     lo = hsub2_1032(lo);
     hi = hsub2_72(hi);
+}
+
+// ---------------------------------------------------------------------------
+// The quantiser, shared by the encoder and the fused append of the decode
+// ---------------------------------------------------------------------------
+__device__ inline float load_in(const void *p, int dtype, int64_t i) {
+    if (dtype == DKV_F32) return static_cast<const float *>(p)[i];
+    if (dtype == DKV_F16) return __half2float(static_cast<const __half *>(p)[i]);
+    return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
+// The Q4_0 block rule for the 32 lanes of one warp (lane = element).
+// Returns the code; *d16 receives the block scale (same value in every lane).
+__device__ inline int quant_lane(float v, __half *d16_out) {
+    uint32_t a = __float_as_uint(v) & 0x7fffffffu;
+    uint32_t mx = __reduce_max_sync(0xffffffffu, a);
+    uint32_t ball = __ballot_sync(0xffffffffu, a == mx);
+    float m = __shfl_sync(0xffffffffu, v, __ffs(ball) - 1);  // lowest index on ties
+    float d32 = __fmul_rn(m, -0.125f);   // = m / -8 exactly: one rounding of the same real value
+    __half d16 = __float2half_rn(d32);
+    float d = __half2float(d16);
+    *d16_out = d16;
+    if (d == 0.0f) return 8;
+    float q = __fdiv_rn(v, d);
+    float u = __fadd_rn(q, 8.5f);
+    int c = (int)truncf(u);
+    return min(15, max(0, c));
 }
 
 }  // namespace dkv

@@ -26,10 +26,13 @@ cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g);
 constexpr int PARTIAL_FLOATS = 8 + 8 + 8 * 128;
 
 // nq queries per sequence: query t attends to the positions before
-// seq_len - (nq - 1 - t); Q and out are [B][nq][Hq][D].
+// seq_len - (nq - 1 - t); Q and out are [B][nq][Hq][D].  With cv.len_add = n
+// > 0 (delta format) the split kernel first appends the n new tokens K_new,
+// V_new ([B][Hkv][n][D] of kv_dtype) and the merge publishes the new lengths.
 cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq, int nq,
                          float softmax_scale, float *ws, int64_t ws_floats, int fault,
-                         cudaStream_t st);
+                         cudaStream_t st, const void *K_new = nullptr,
+                         const void *V_new = nullptr, int kv_dtype = 0);
 cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const float *ws,
                          cudaStream_t st);
 

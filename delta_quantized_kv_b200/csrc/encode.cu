@@ -18,30 +18,6 @@
 
 namespace dkv {
 
-__device__ inline float load_in(const void *p, int dtype, int64_t i) {
-    if (dtype == DKV_F32) return static_cast<const float *>(p)[i];
-    if (dtype == DKV_F16) return __half2float(static_cast<const __half *>(p)[i]);
-    return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
-}
-
-// The Q4_0 block rule for the 32 lanes of one warp (lane = element).
-// Returns the code; *d16 receives the block scale (same value in every lane).
-__device__ inline int quant_lane(float v, __half *d16_out) {
-    uint32_t a = __float_as_uint(v) & 0x7fffffffu;
-    uint32_t mx = __reduce_max_sync(0xffffffffu, a);
-    uint32_t ball = __ballot_sync(0xffffffffu, a == mx);
-    float m = __shfl_sync(0xffffffffu, v, __ffs(ball) - 1);  // lowest index on ties
-    float d32 = __fmul_rn(m, -0.125f);   // = m / -8 exactly: one rounding of the same real value
-    __half d16 = __float2half_rn(d32);
-    float d = __half2float(d16);
-    *d16_out = d16;
-    if (d == 0.0f) return 8;
-    float q = __fdiv_rn(v, d);
-    float u = __fadd_rn(q, 8.5f);
-    int c = (int)truncf(u);
-    return min(15, max(0, c));
-}
-
 struct EncodeArgs {
     CacheView cv;
     const void *K;
@@ -79,17 +55,7 @@ __device__ inline void pack_nibbles(const uint8_t (*codes)[D], int cnt, int t, u
         int s = idx >> 4, w = idx & 15;
         uint32_t word = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            int c;
-            if (t == 0) {
-                int tt = w >> 2, j = w & 3, h = i >> 2, s2 = (i >> 1) & 1, e = i & 1;
-                c = 32 * j + 16 * s2 + 8 * e + 2 * tt + h;
-            } else {
-                int g = w >> 1, u = w & 1, mt = 4 * u + (i >> 1);
-                c = 16 * mt + g + 8 * (i & 1);
-            }
-            word |= (uint32_t)(codes[s][c] & 15) << (4 * i);
-        }
+        for (int i = 0; i < 8; ++i) word |= (uint32_t)(codes[s][nib_channel(t, w, i)] & 15) << (4 * i);
         reinterpret_cast<uint32_t *>(dst + (int64_t)s * NIB_BYTES)[w] = word;
     }
 }

@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define DKV_ABI_VERSION 2
+#define DKV_ABI_VERSION 3
 
 typedef enum {
     DKV_OK = 0,
@@ -191,8 +191,8 @@ dkv_status dkv_decode_attn_split(const dkv_cache *cache, const void *Q, int32_t 
 dkv_status dkv_decode_attn_merge(const dkv_cache *cache, int32_t n_q_heads, float *out,
                                  void *workspace, size_t ws_bytes, void *stream);
 
-/* Multi-query decode (NEXT row: several new tokens per sequence, as in
- * speculative decoding).  The n_queries newest tokens of every sequence have
+/* Multi-query decode (several new tokens per sequence, as in speculative
+ * decoding).  The n_queries newest tokens of every sequence have
  * been appended (dkv_append with n_new = n_queries); query t (0 <= t <
  * n_queries) is token seq_len - n_queries + t's own query and attends to the
  * positions before seq_len - (n_queries - 1 - t), i.e. causally.
@@ -208,6 +208,40 @@ size_t dkv_decode_workspace_bytes_mq(const dkv_cache_desc *desc, int32_t n_q_hea
 dkv_status dkv_decode_attn_mq(const dkv_cache *cache, const void *Q, int32_t q_dtype,
                               int32_t n_q_heads, int32_t n_queries, float softmax_scale,
                               float *out, void *workspace, size_t ws_bytes, void *stream);
+
+/* Fused append + decode (DKV_FMT_DELTA): one call that appends n_new tokens
+ * to every sequence, exactly as dkv_append would, and runs the decode step
+ * over the grown cache with the new tokens' own n_new queries, exactly as
+ * dkv_decode_attn_mq with n_queries = n_new would (dkv_decode_attn for
+ * n_new = 1).  The quantiser runs inside the decode's split kernel: the warps
+ * that stream the groups the new tokens land in first quantise those tokens
+ * (the same steps, in the same order, as the encoder: the stored codes, scales,
+ * keyframes and reconstruction state are bit-identical to dkv_append's), so
+ * the step takes two launches instead of three, and the merge publishes the
+ * new lengths.
+ * K_new, V_new: [B][Hkv][n_new][D] contiguous device arrays of kv_dtype (as
+ * for dkv_append); Q: [B][n_new][n_q_heads][D] of q_dtype (for n_new = 1 that
+ * is [B][n_q_heads][D]); out: the same shape as Q in fp32; workspace: >=
+ * dkv_decode_workspace_bytes_mq(desc, n_q_heads, n_new).  A batch entry whose
+ * tokens do not fit (seq_len + n_new > max_ctx) takes none, sets
+ * DKV_DEV_CAPACITY and is decoded at its stored length; an invalid stored
+ * length sets DKV_DEV_BAD_SEQLEN and decodes as empty.  1 <= n_new <= 256.
+ * Other formats: DKV_EUNSUPPORTED.  A bad block-table entry (paged cache) sets
+ * DKV_DEV_BAD_PAGE; the tokens of that page are then not stored.
+ * The _split and _merge halves are the two launches, exposed so each can be
+ * timed alone; they must run back to back on one stream with the same
+ * arguments, with no other call on the cache between them. */
+dkv_status dkv_append_decode_attn(dkv_cache *cache, const void *K_new, const void *V_new,
+                                  int32_t kv_dtype, int32_t n_new, const void *Q,
+                                  int32_t q_dtype, int32_t n_q_heads, float softmax_scale,
+                                  float *out, void *workspace, size_t ws_bytes, void *stream);
+dkv_status dkv_append_decode_attn_split(dkv_cache *cache, const void *K_new, const void *V_new,
+                                        int32_t kv_dtype, int32_t n_new, const void *Q,
+                                        int32_t q_dtype, int32_t n_q_heads, float softmax_scale,
+                                        void *workspace, size_t ws_bytes, void *stream);
+dkv_status dkv_append_decode_attn_merge(dkv_cache *cache, int32_t n_new, int32_t n_q_heads,
+                                        float *out, void *workspace, size_t ws_bytes,
+                                        void *stream);
 
 /* Size of the library-owned scratch array used by dkv_decode_attn_noalloc. */
 #define DKV_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -107,6 +107,8 @@ def test_calls_on_an_invalid_cache_are_rejected(dkv):
     assert lib.dkv_append(ctypes.byref(c), 16, 16, 1, 1, None) == dkv.DKV_EINVAL
     assert lib.dkv_decode_attn(ctypes.byref(c), 16, 1, 8, 1.0, 16, 16, 1 << 20, None) == dkv.DKV_EINVAL
     assert lib.dkv_dequantize(ctypes.byref(c), 16, None) == dkv.DKV_EINVAL
+    assert lib.dkv_append_decode_attn(ctypes.byref(c), 16, 16, 1, 1, 16, 1, 8, 1.0, 16, 16,
+                                      1 << 20, None) == dkv.DKV_EINVAL
     w = ctypes.c_int32(0)
     assert lib.dkv_get_device_status(ctypes.byref(c), ctypes.byref(w), None) == dkv.DKV_EINVAL
 
@@ -136,6 +138,25 @@ def test_bad_dtype_and_sizes_rejected_on_host(dkv):
     # n_q_heads not a multiple of n_kv_heads
     assert lib.dkv_decode_attn(ctypes.byref(c), 1 << 12, 1, 3, 1.0, 1 << 12, 1 << 12, 1 << 30,
                                None) == dkv.DKV_EINVAL
+    # fused append + decode: K/V dtype, alignment, token count, heads, scale
+    fused = lambda kvd=1, k=1 << 12, n=1, hq=4, s=1.0: lib.dkv_append_decode_attn(
+        ctypes.byref(c), k, 1 << 12, kvd, n, 1 << 12, 1, hq, s, 1 << 12, 1 << 12, 1 << 30, None)
+    assert fused(kvd=9) == dkv.DKV_EINVAL
+    assert fused(k=(1 << 12) + 2) == dkv.DKV_EALIGN
+    assert fused(n=0) == dkv.DKV_EINVAL
+    assert fused(n=257) == dkv.DKV_EINVAL
+    assert fused(hq=3) == dkv.DKV_EINVAL
+    assert fused(s=0.0) == dkv.DKV_EINVAL
+    assert lib.dkv_append_decode_attn_merge(ctypes.byref(c), 1, 4, (1 << 12) + 4, 1 << 12,
+                                            1 << 30, None) == dkv.DKV_EALIGN
+    # only the delta format appends inside the decode (a well-formed Q4_0 view)
+    c.desc.fmt = 1
+    c.seq_stride, c.rec_bytes, c.n_groups = 100 * 144, 0, 0
+    c.off_state = up(4 * c.seq_stride + 4096)
+    c.off_seqlen = up(c.off_state + 2 * 4 * 2 * 128 * 4)
+    c.off_header = up(c.off_seqlen + 8)
+    c.bytes = dkv.dkv_cache_bytes(c.desc)
+    assert fused() == dkv.DKV_EUNSUPPORTED
 
 
 # ---- the decode work split (restated from the kernel's range arithmetic) ----
