@@ -231,3 +231,101 @@ def test_paged_sizes_and_argument_checks(dkv):
     dq = _desc(dkv, B=4, H=8, cap=4096, fmt=1)
     assert lib.dkv_cache_init_paged(ctypes.byref(dq), 16, A, 64, A, 8, A, meta,
                                     ctypes.byref(out), None) == dkv.DKV_EUNSUPPORTED
+
+
+# ---- fused append: which warp stores which new token (restated walk) -------
+def _append_walk(units_of_seq, nvs, r0, r1, lens, n, kf, cap, pre, nhg):
+    """The groups (b, vs, g) a warp with range [r0, r1) stores new tokens of, in
+    its two phases (units [0, pre) of the range before its first copies, the
+    rest after), and the (b, kv head) states it writes."""
+    stores, states = [], []
+    # locate the range's first unit
+    x, b = 0, 0
+    while b < len(lens) and x + nvs * units_of_seq[b] <= r0:
+        x += nvs * units_of_seq[b]
+        b += 1
+    r = r0 - x
+    vs, g0, ub = r // units_of_seq[b], r % units_of_seq[b], units_of_seq[b]
+    for lo, hi in ((0, min(pre, r1 - r0)), (pre, r1 - r0)):
+        if lo >= hi:
+            continue
+        bb, vv, gg, uu, off = b, vs, g0, ub, 0
+        while off < hi:
+            seg = uu - gg
+            if off + seg > lo:
+                ga = gg + max(0, lo - off)
+                gb = gg + min(hi, off + seg) - off - 1
+                L = lens[bb]
+                if 0 <= L <= cap and L + n <= cap:
+                    first = max(ga, L // kf)
+                    for g in range(first, gb + 1):
+                        stores.append((bb, vv, g))
+                    if first <= gb and gb == uu - 1 and vv % nhg == 0:
+                        states.append((bb, vv // nhg))
+            off += seg
+            if off >= hi:
+                break
+            gg = 0
+            vv += 1
+            if vv == nvs:
+                vv = 0
+                while True:
+                    bb += 1
+                    if bb >= len(lens):
+                        break
+                    uu = units_of_seq[bb]
+                    if uu:
+                        break
+                if bb >= len(lens):
+                    break
+    return stores, states
+
+
+def test_fused_append_walk_stores_every_new_group_once_per_owner():
+    """Every group holding new tokens is stored by the warp that owns it (so
+    that warp's own copy reads it after its own stores), no warp stores a group
+    it does not own, and each (batch entry, kv head) that takes tokens has
+    exactly one state writer."""
+    rng = random.Random(11)
+    for _ in range(300):
+        B, Hkv, nhg = rng.randint(1, 5), rng.randint(1, 3), rng.choice([1, 1, 2, 3])
+        kf, n = rng.choice([1, 3, 16, 32, 64]), rng.choice([1, 1, 2, 5])
+        cap = rng.choice([40, 100, 300])
+        lens = [rng.choice([0, 1, 31, 32, 33, 64, cap - n, cap - n + 1, cap, -1, cap + 1])
+                for _ in range(B)]
+        nvs = Hkv * nhg
+        dec = [(L + n if 0 <= L <= cap and L + n <= cap else (L if 0 <= L <= cap else 0))
+               for L in lens]
+        units = [-(-d // kf) if d > 0 else 0 for d in dec]
+        T = sum(nvs * u for u in units)
+        if T == 0:
+            continue
+        NW = rng.choice([1, 2, 7, 64, 300])
+        pre = rng.choice([1, 2])
+        owner = {}
+        x = 0
+        for b in range(B):
+            for vs in range(nvs):
+                for g in range(units[b]):
+                    owner[(b, vs, g)] = ((x + 1) * NW - 1) // T
+                    x += 1
+        stored, writers = {}, {}
+        for w in range(NW):
+            r0, r1 = (w * T) // NW, ((w + 1) * T) // NW
+            if r0 >= r1:
+                continue
+            st, sw = _append_walk(units, nvs, r0, r1, lens, n, kf, cap, pre, nhg)
+            for key in st:
+                assert owner[key] == w, (key, w)
+                stored[key] = stored.get(key, 0) + 1
+            for key in sw:
+                writers[key] = writers.get(key, 0) + 1
+        for b, L in enumerate(lens):
+            takes = 0 <= L <= cap and L + n <= cap
+            for vs in range(nvs):
+                new_groups = range(L // kf, units[b]) if takes else range(0)
+                for g in new_groups:
+                    assert stored.get((b, vs, g)) == 1, (b, vs, g, lens, n, kf)
+            for kvh in range(Hkv):
+                assert writers.get((b, kvh), 0) == (1 if takes else 0), (b, kvh, lens)
+        assert all(k[2] >= max(0, lens[k[0]]) // kf for k in stored)
