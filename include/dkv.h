@@ -123,8 +123,8 @@ size_t dkv_cache_bytes(const dkv_cache_desc *desc);
 dkv_status dkv_cache_init(const dkv_cache_desc *desc, void *dev, size_t bytes,
                           dkv_cache *out, void *stream);
 
-/* Paged cache (NEXT row: a paged, group-aligned cache for ragged serving;
- * the "decoupled memory management" of page "DeltaKV ... Sparse-vLLM",
+/* Paged cache (a paged, group-aligned cache for ragged serving; the
+ * "decoupled memory management" of page "DeltaKV ... Sparse-vLLM",
  * section "B. Sparse-vLLM", without the learned compressor).
  * dkv_cache_meta_bytes: bytes of the small metadata buffer a paged cache
  * needs (reconstruction state, lengths, header); dkv_page_bytes: bytes of one
@@ -209,8 +209,11 @@ dkv_status dkv_decode_attn_mq(const dkv_cache *cache, const void *Q, int32_t q_d
                               int32_t n_q_heads, int32_t n_queries, float softmax_scale,
                               float *out, void *workspace, size_t ws_bytes, void *stream);
 
-/* Fused append + decode (DKV_FMT_DELTA): one call that appends n_new tokens
- * to every sequence, exactly as dkv_append would, and runs the decode step
+/* Fused append + decode (DKV_FMT_DELTA): the append of page "...Delta-KV",
+ * section "핵심 아이디어", and the decode step of page "KV 캐시 벡터 양자화와
+ * 주의 보존 변환", section "KV 캐시가 왜 병목인가", in one call.  The call
+ * appends n_new tokens to every sequence, exactly as dkv_append would, and
+ * runs the decode step
  * over the grown cache with the new tokens' own n_new queries, exactly as
  * dkv_decode_attn_mq with n_queries = n_new would (dkv_decode_attn for
  * n_new = 1).  The quantiser runs inside the decode's split kernel: the warps
