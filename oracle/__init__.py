@@ -15,7 +15,11 @@ it (see the C source header for the citations):
 * ``delta_append``     -- the same loop continued from a saved state;
 * ``delta_decode``     -- reconstruction from the stored codes alone;
 * ``q4_encode`` / ``f16_encode`` -- the two comparator caches;
-* ``attn``             -- one decode step of softmax attention, binary64.
+* ``attn``             -- one decode step of softmax attention, binary64;
+* ``lr_encode``        -- long-range reference encoding: fp16 references at a
+                          fixed stride, each other token the Q4_0 residual
+                          against the mean of its most similar references
+                          (the training-free part of DeltaKV).
 
 Every function is pinned by tests under ``tests/test_oracle_*.py`` against
 closed forms, invariants, brute force and library routines (numpy float16
@@ -67,8 +71,9 @@ def _load():
         lib.or_q4_encode.argtypes = [i, i, P, P, P, P]
         lib.or_f16_encode.argtypes = [i, i, P, P, P]
         lib.or_attn.argtypes = [i, i, i, P, P, P, ctypes.c_double, P]
+        lib.or_lr_encode.argtypes = [i, i, i, i, P, P, P, P, P, P]
         for f in ("or_quant_block", "or_delta_encode_range", "or_delta_decode",
-                  "or_q4_encode", "or_f16_encode", "or_attn"):
+                  "or_q4_encode", "or_f16_encode", "or_attn", "or_lr_encode"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -193,6 +198,24 @@ def f16_encode(x):
     xhat = np.zeros((T, D), dtype=np.float32)
     lib.or_f16_encode(T, D, _p(x), _p(bits), _p(xhat))
     return bits, xhat
+
+
+def lr_encode(x, s: int, m: int) -> dict:
+    """Long-range reference encoding of one [T, D] sequence (stride s, the m
+    most similar references; see ``or_lr_encode`` in the C source) ->
+    dict(ref[T, m] int32, kfr[ceil(T/s), D] fp16 bits, scales[T, D/32] fp16
+    bits, codes[T, D], xhat[T, D] binary32)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    T, D = x.shape
+    assert D % BLOCK == 0 and s >= 1 and m >= 1
+    ng = max(1, (T + s - 1) // s)
+    out = {"ref": np.zeros((T, m), np.int32), "kfr": np.zeros((ng, D), np.uint16),
+           "scales": np.zeros((T, D // BLOCK), np.uint16), "codes": np.zeros((T, D), np.uint8),
+           "xhat": np.zeros((T, D), np.float32)}
+    lib.or_lr_encode(T, D, s, m, _p(x), _p(out["ref"]), _p(out["kfr"]), _p(out["scales"]),
+                     _p(out["codes"]), _p(out["xhat"]))
+    return out
 
 
 # --------------------------------------------------------------------------

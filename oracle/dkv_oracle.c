@@ -276,3 +276,109 @@ void or_attn(int T, int D, int G, const double *q, const float *khat,
     }
     free(s);
 }
+
+/* ---------------------------------------------------------------------------
+ * Long-range reference encoder (the training-free part of DeltaKV), one
+ * sequence of one tensor.  Source: the gist.science summary of DeltaKV
+ * (arXiv 2602.08005):
+ *   section "2. 핵심 관찰": similar tokens are spread far apart over the
+ *     context (long-range inter-token similarity);
+ *   section "A. DeltaKV 프레임워크": "Strided Reference Selection" (the
+ *     reference set is the tokens at a fixed stride), "Residual Encoding"
+ *     (subtract the mean of the most similar reference tokens; encode the
+ *     residual), "Reconstruction" (add that mean back);
+ *   section "4. 주요 기여 및 결과", "양자화 친화성": the residuals sit near
+ *     zero and take 4-bit quantisation.
+ * The learned compressor is replaced by the Q4_0 block rule.
+ * Readings where the page is silent:
+ *   - the references are the positions r with r mod s == 0, stored as fp16;
+ *   - token p (not a reference) chooses among the references before it, r < p;
+ *   - "most similar" is the smallest squared Euclidean distance to the stored
+ *     reference, summed over channels c = 0 .. D-1 in binary64, in that order
+ *     (each difference, square and sum one binary64 operation); ties go to
+ *     the smaller position;
+ *   - the m most similar are used (all of them when fewer exist); their mean
+ *     is the binary32 sum in ascending position, divided (binary32) by their
+ *     count;
+ *   - the residual x_p - mean (binary32) is quantised with the Q4_0 block
+ *     rule and x^_p = mean + (code - 8) * d.
+ * Outputs, indexed by position p in [0, T):
+ *   ref    [T][m]   reference numbers r / s of the chosen references in
+ *                   ascending order; -1 for unused slots and reference tokens
+ *   kfr    [ng][D]  fp16 bits of reference g (position g * s), ng = ceil(T/s)
+ *   scales [T][D/32], codes [T][D]  (zero on reference rows)
+ *   xhat   [T][D]   reconstruction
+ * ------------------------------------------------------------------------- */
+void or_lr_encode(int T, int D, int s, int m, const float *x, int32_t *ref, uint16_t *kfr,
+                  uint16_t *scales, uint8_t *codes, float *xhat)
+{
+    const int nb = D / OR_BLOCK;
+    const int ng = (T + s - 1) / s;
+    float *kv = (float *)malloc(sizeof(float) * (size_t)(ng > 0 ? ng : 1) * D);
+    double *dist = (double *)malloc(sizeof(double) * (size_t)(ng > 0 ? ng : 1));
+    int *sel = (int *)malloc(sizeof(int) * (size_t)m);
+    float *mean = (float *)malloc(sizeof(float) * (size_t)D);
+    float res[OR_BLOCK];
+    for (int p = 0; p < T; ++p) {
+        const float *xp = x + (size_t)p * D;
+        for (int k = 0; k < m; ++k) ref[(size_t)p * m + k] = -1;
+        memset(scales + (size_t)p * nb, 0, sizeof(uint16_t) * (size_t)nb);
+        memset(codes + (size_t)p * D, 0, (size_t)D);
+        if (p % s == 0) {                    /* a reference token: fp16 */
+            const int g = p / s;
+            for (int c = 0; c < D; ++c) {
+                uint16_t h = or_f32_to_f16(xp[c]);
+                kfr[(size_t)g * D + c] = h;
+                kv[(size_t)g * D + c] = or_f16_to_f32(h);
+                xhat[(size_t)p * D + c] = kv[(size_t)g * D + c];
+            }
+            continue;
+        }
+        const int nc = (p - 1) / s + 1;      /* references 0, s, 2s, ... below p */
+        for (int g = 0; g < nc; ++g) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c) {
+                double diff = (double)xp[c] - (double)kv[(size_t)g * D + c];
+                double sq = diff * diff;
+                acc = acc + sq;
+            }
+            dist[g] = acc;
+        }
+        const int me = nc < m ? nc : m;
+        for (int k = 0; k < me; ++k) {       /* k-th smallest, smaller position first */
+            int best = -1;
+            for (int g = 0; g < nc; ++g) {
+                int used = 0;
+                for (int j = 0; j < k; ++j) used |= (sel[j] == g);
+                if (used) continue;
+                if (best < 0 || dist[g] < dist[best]) best = g;
+            }
+            sel[k] = best;
+        }
+        for (int i = 1; i < me; ++i)         /* ascending position */
+            for (int j = i; j > 0 && sel[j - 1] > sel[j]; --j) {
+                int t = sel[j]; sel[j] = sel[j - 1]; sel[j - 1] = t;
+            }
+        for (int k = 0; k < me; ++k) ref[(size_t)p * m + k] = sel[k];
+        for (int c = 0; c < D; ++c) {
+            float acc = 0.0f;
+            for (int k = 0; k < me; ++k) acc = acc + kv[(size_t)sel[k] * D + c];
+            mean[c] = acc / (float)me;
+        }
+        for (int b = 0; b < nb; ++b) {
+            for (int i = 0; i < OR_BLOCK; ++i)
+                res[i] = xp[b * OR_BLOCK + i] - mean[b * OR_BLOCK + i];
+            uint16_t d16;
+            uint8_t *cb = codes + (size_t)p * D + b * OR_BLOCK;
+            or_quant_block(res, &d16, cb);
+            scales[(size_t)p * nb + b] = d16;
+            for (int i = 0; i < OR_BLOCK; ++i)
+                xhat[(size_t)p * D + b * OR_BLOCK + i] =
+                    mean[b * OR_BLOCK + i] + or_dequant(cb[i], d16);
+        }
+    }
+    free(kv);
+    free(dist);
+    free(sel);
+    free(mean);
+}
