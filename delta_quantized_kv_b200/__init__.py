@@ -56,7 +56,7 @@ EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode",
            "dkv_debug_set_fault", "dkv_cache_meta_bytes", "dkv_page_bytes",
            "dkv_cache_init_paged", "dkv_decode_workspace_bytes_mq", "dkv_decode_attn_mq",
            "dkv_append_decode_attn", "dkv_append_decode_attn_split",
-           "dkv_append_decode_attn_merge"]
+           "dkv_append_decode_attn_merge", "dkv_lr_encode"]
 
 
 def load():
@@ -95,6 +95,7 @@ def load():
         "dkv_append_decode_attn": ([PC, P, P, I, I, P, I, I, F, P, P, S, P], I),
         "dkv_append_decode_attn_split": ([PC, P, P, I, I, P, I, I, F, P, S, P], I),
         "dkv_append_decode_attn_merge": ([PC, I, I, P, P, S, P], I),
+        "dkv_lr_encode": ([P, I, I, I, I, I, P, P, P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -232,6 +233,27 @@ def dkv_append_decode_attn_merge(cache: dkv_cache, n_new, n_q_heads, out, worksp
     _check(load().dkv_append_decode_attn_merge(ctypes.byref(cache), n_new, n_q_heads, _ptr(out),
                                                _ptr(workspace), ws_bytes, _stream(stream)),
            "dkv_append_decode_attn_merge")
+
+
+def lr_encode(X, stride: int, n_refs: int, stream=None) -> dict:
+    """Long-range reference encoding (dkv_lr_encode) of X [n_seq, T, 128] on
+    the GPU -> dict of device tensors ref, ref_values, scales, codes, xhat in
+    the canonical layouts."""
+    import torch
+    n_seq, T, Dh = X.shape
+    ng = -(-T // stride)
+    dev = X.device
+    out = {"ref": torch.empty((n_seq, T, n_refs), dtype=torch.int32, device=dev),
+           "ref_values": torch.empty((n_seq, ng, Dh), dtype=torch.int16, device=dev),
+           "scales": torch.empty((n_seq, T, Dh // 32), dtype=torch.int16, device=dev),
+           "codes": torch.empty((n_seq, T, Dh), dtype=torch.uint8, device=dev),
+           "xhat": torch.empty((n_seq, T, Dh), dtype=torch.float32, device=dev)}
+    X = X.contiguous()
+    _check(load().dkv_lr_encode(_ptr(X), _dtype_code(X.dtype), n_seq, T, stride, n_refs,
+                                _ptr(out["ref"]), _ptr(out["ref_values"]), _ptr(out["scales"]),
+                                _ptr(out["codes"]), _ptr(out["xhat"]), _stream(stream)),
+           "dkv_lr_encode")
+    return out
 
 
 def dkv_decode_attn_split(cache: dkv_cache, Q, q_dtype, n_q_heads, softmax_scale, workspace,

@@ -13,7 +13,7 @@ from pathlib import Path
 PKG = Path(__file__).resolve().parent
 CSRC = PKG / "csrc"
 OUT = PKG / "_lib" / "libdkv.so"
-SOURCES = ["dkv_api.cu", "encode.cu", "decode.cu", "noalloc.cu"]
+SOURCES = ["dkv_api.cu", "encode.cu", "decode.cu", "noalloc.cu", "lr_encode.cu"]
 HEADERS = ["dkv_common.cuh", "dkv_internal.h"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared"]

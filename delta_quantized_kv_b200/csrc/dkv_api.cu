@@ -380,6 +380,21 @@ dkv_status dkv_append_decode_attn(dkv_cache *cache, const void *K_new, const voi
     return dkv_append_decode_attn_merge(cache, n_new, n_q_heads, out, workspace, ws_bytes, stream);
 }
 
+dkv_status dkv_lr_encode(const void *X, int32_t dtype, int32_t n_seq, int32_t T, int32_t stride,
+                         int32_t n_refs, int32_t *ref, uint16_t *ref_values, uint16_t *scales,
+                         uint8_t *codes, float *xhat, void *stream) {
+    if (!X || !ref || !ref_values || !scales || !codes || !valid_dtype(dtype)) return DKV_EINVAL;
+    if (n_seq < 1 || n_seq > 65535 || T < 1 || stride < 1 || n_refs < 1 || n_refs > 8)
+        return DKV_EINVAL;
+    if ((int64_t)n_seq * T > ((int64_t)1 << 31)) return DKV_ECAPACITY;
+    if (!aligned16(X) || !aligned16(ref) || !aligned16(ref_values) || !aligned16(scales) ||
+        !aligned16(codes) || (xhat && !aligned16(xhat)))
+        return DKV_EALIGN;
+    return cuda_status(dkv::launch_lr_encode(X, dtype, n_seq, T, stride, n_refs, ref, ref_values,
+                                             scales, codes, xhat,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 dkv_status dkv_export_canonical(const dkv_cache *cache, uint8_t *codes, uint16_t *scales,
                                 uint16_t *keyframes, float *state, void *stream) {
     dkv_status s = check_cache(cache);

@@ -36,4 +36,10 @@ cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq
 cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const float *ws,
                          cudaStream_t st);
 
+// Long-range reference encoding of n_seq sequences [n_seq][T][D] (layouts
+// of dkv_lr_encode).
+cudaError_t launch_lr_encode(const void *X, int dtype, int n_seq, int T, int s, int m,
+                             int32_t *ref, uint16_t *kfr, uint16_t *scales, uint8_t *codes,
+                             float *xhat, cudaStream_t st);
+
 }  // namespace dkv

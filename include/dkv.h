@@ -246,6 +246,31 @@ dkv_status dkv_append_decode_attn_merge(dkv_cache *cache, int32_t n_new, int32_t
                                         float *out, void *workspace, size_t ws_bytes,
                                         void *stream);
 
+/* Long-range reference encoding: the training-free part of DeltaKV (page
+ * "DeltaKV" summary, section 2: similar tokens lie far apart in the context;
+ * section A: "Strided Reference Selection", "Residual Encoding",
+ * "Reconstruction"; section 4, "양자화 친화성": the residuals take 4-bit
+ * quantisation), with the learned compressor replaced by the Q4_0 block rule.
+ * Every stride-th token (p mod stride == 0) is a reference, stored as fp16.
+ * Every other token p takes the n_refs references r < p nearest to it
+ * (squared Euclidean distance to the stored reference, binary64, channels in
+ * order; ties to the smaller position; all of them when fewer exist), and
+ * stores its residual against their mean (binary32 sum in ascending position
+ * divided by their count) with the Q4_0 block rule; x^ = mean + (code - 8) d.
+ * n_seq independent sequences.  X: [n_seq][T][128] device array of dtype.
+ * Outputs (device, caller-owned, canonical layouts):
+ *   ref        int32  [n_seq][T][n_refs]   chosen reference numbers r / stride,
+ *                                          ascending; -1 unused / reference rows
+ *   ref_values uint16 [n_seq][ceil(T/stride)][128]  fp16 bits of the references
+ *   scales     uint16 [n_seq][T][4]         fp16 bits (0 on reference rows)
+ *   codes      uint8  [n_seq][T][128]       0..15 (0 on reference rows)
+ *   xhat       float  [n_seq][T][128]       reconstruction (NULL: not written)
+ * 1 <= n_refs <= 8, stride >= 1.  Encoding only: there is no decode over this
+ * format yet. */
+dkv_status dkv_lr_encode(const void *X, int32_t dtype, int32_t n_seq, int32_t T, int32_t stride,
+                         int32_t n_refs, int32_t *ref, uint16_t *ref_values, uint16_t *scales,
+                         uint8_t *codes, float *xhat, void *stream);
+
 /* Size of the library-owned scratch array used by dkv_decode_attn_noalloc. */
 #define DKV_NOALLOC_SCRATCH_BYTES (16u << 20)
 
