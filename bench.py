@@ -387,6 +387,40 @@ def quality_report(dev, max_batch: int = 2):
     return rep
 
 
+LR_CASES = [("batched_decode", "repeat", 2048), ("llama3_8b_layer", None, 4096)]
+
+
+def lr_quality(dev, lr_encode, recon):
+    """Long-range reference encoding (the training-free part of DeltaKV) next
+    to the delta and Q4_0 caches on the same tokens: relative reconstruction
+    MSE of K and V for the first batch entry of each case (stride = kf, 1 and
+    4 references).  `lr_encode(X, stride, n_refs)` returns the reconstruction
+    of X [n_seq, T, 128]; `recon(fmt, K, V, kf)` the cache's reconstruction
+    of K, V [Hkv, T, 128] as two tensors.  The encoder costs O(T^2 / stride),
+    so the cases are short."""
+    import torch
+    import synthetic as S
+    out = {}
+    for name, gen, T in LR_CASES:
+        w = S.WORKLOADS[name].with_(B=1, T=T)
+        if gen:
+            w = w.with_(gen=gen)
+        K, V = S.gen_kv_one(w, 0, T, device=dev)
+        X = torch.cat([K, V]).contiguous()
+        x = X.float()
+        sig = (x ** 2).sum().item()
+        row = {}
+        for n_refs in (1, 4):
+            xh = lr_encode(X, w.kf, n_refs)
+            row[f"lr_{n_refs}_ref"] = ((xh - x) ** 2).sum().item() / sig
+        for fmt in ("delta", "q4"):
+            kh, vh = recon(fmt, K, V, w.kf)
+            row[fmt] = (((kh - K.float()) ** 2).sum().item() +
+                        ((vh - V.float()) ** 2).sum().item()) / sig
+        out[name + (f"_{gen}" if gen else "") + f"_T{T}_stride{w.kf}"] = row
+    return out
+
+
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
@@ -685,6 +719,19 @@ def run_ours(args, w, rank, world, local):
 
     if rank == 0 and args.comparators:
         res["quality"] = quality_report(dev)
+
+        def _recon(fmt, K, V, kf):
+            cc = dkv.Cache(1, K.shape[0], K.shape[1], fmt, kf=kf, device=dev)
+            cc.encode(K[None].contiguous(), V[None].contiguous())
+            xh = cc.dequantize()[0]
+            T_ = K.shape[1]
+            return xh[:, 0, :T_], xh[:, 1, :T_]
+
+        try:
+            res["quality"]["long_range_refs"] = lr_quality(
+                dev, lambda X, s, m: dkv.lr_encode(X, s, m)["xhat"], _recon)
+        except Exception as e:          # a reported extra: never costs the bench line
+            res["quality"]["long_range_refs"] = {"error": repr(e)[:200]}
     if rank != 0:
         return
     cpu = None

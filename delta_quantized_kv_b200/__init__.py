@@ -240,7 +240,11 @@ def lr_encode(X, stride: int, n_refs: int, stream=None) -> dict:
     the GPU -> dict of device tensors ref, ref_values, scales, codes, xhat in
     the canonical layouts."""
     import torch
+    if X.dim() != 3 or X.shape[2] != 128:
+        raise ValueError("lr_encode takes X of shape [n_seq, T, 128]")
     n_seq, T, Dh = X.shape
+    if stride < 1 or not 1 <= n_refs <= 8:
+        raise DkvError(DKV_EINVAL, "dkv_lr_encode")
     ng = -(-T // stride)
     dev = X.device
     out = {"ref": torch.empty((n_seq, T, n_refs), dtype=torch.int32, device=dev),

@@ -159,6 +159,29 @@ def test_bad_dtype_and_sizes_rejected_on_host(dkv):
     assert fused() == dkv.DKV_EUNSUPPORTED
 
 
+def test_lr_encode_rejects_bad_arguments_on_host(dkv):
+    """dkv_lr_encode validates before any launch: pointers, dtype, sizes,
+    stride, reference count (1..8) and 16-byte alignment."""
+    lib = dkv.load()
+    A = 1 << 20
+
+    def call(X=A, dt=1, n=2, T=64, s=8, m=2, ref=A, kv=A, sc=A, co=A, xh=A):
+        return lib.dkv_lr_encode(X, dt, n, T, s, m, ref, kv, sc, co, xh, None)
+    assert call(X=None) == dkv.DKV_EINVAL
+    assert call(co=None) == dkv.DKV_EINVAL
+    assert call(dt=7) == dkv.DKV_EINVAL
+    assert call(n=0) == dkv.DKV_EINVAL
+    assert call(T=0) == dkv.DKV_EINVAL
+    assert call(s=0) == dkv.DKV_EINVAL
+    assert call(m=0) == dkv.DKV_EINVAL
+    assert call(m=9) == dkv.DKV_EINVAL
+    assert call(n=65536) == dkv.DKV_EINVAL
+    assert call(n=60000, T=60000) == dkv.DKV_ECAPACITY
+    assert call(X=A + 2) == dkv.DKV_EALIGN
+    assert call(sc=A + 8) == dkv.DKV_EALIGN
+    assert call(xh=A + 4) == dkv.DKV_EALIGN
+
+
 # ---- the decode work split (restated from the kernel's range arithmetic) ----
 def _start(w, NW, T):
     return (w * T) // NW
