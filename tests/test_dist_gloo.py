@@ -74,3 +74,35 @@ def test_kv_bytes_model():
     assert bench.kv_bytes("fp16", [32768] * 16, 8, 32) == 2_147_483_648
     # a partial last group still pays a whole keyframe
     assert bench.kv_bytes("delta", [33], 1, 32) == 2 * 512 + 31 * 144
+
+
+def test_long_range_quality_report_logic():
+    """bench.lr_quality's bookkeeping (cases, keys, ratios), driven on the CPU
+    by the oracle in place of the GPU encoder and caches: the long-range
+    encoding must beat plain Q4_0 on the window-repeat generator, where far
+    repeats are what the strided references exploit."""
+    import numpy as np
+    import torch
+    import bench
+    import oracle
+
+    def enc(X, s, m):
+        return torch.stack([torch.from_numpy(oracle.lr_encode(X[i].float().numpy(), s, m)["xhat"])
+                            for i in range(X.shape[0])])
+
+    def recon(fmt, K, V, kf):
+        f = lambda A: torch.stack([torch.from_numpy(
+            oracle.encode_cache(fmt, A[i].float().numpy(), kf)["xhat"]) for i in range(A.shape[0])])
+        return f(K), f(V)
+
+    saved = bench.LR_CASES
+    bench.LR_CASES = [("batched_decode", "repeat", 256)]
+    try:
+        rep = bench.lr_quality("cpu", enc, recon)
+    finally:
+        bench.LR_CASES = saved
+    (key, row), = rep.items()
+    assert key == "batched_decode_repeat_T256_stride32"
+    assert set(row) == {"lr_1_ref", "lr_4_ref", "delta", "q4"}
+    assert all(np.isfinite(v) and v >= 0 for v in row.values())
+    assert row["lr_1_ref"] < 0.1 * row["q4"]
