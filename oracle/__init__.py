@@ -242,12 +242,15 @@ def attn(q, khat, vhat, scale: float) -> np.ndarray:
 # --------------------------------------------------------------------------
 # whole-cache helpers used by the parity tests and the CPU baseline
 # --------------------------------------------------------------------------
-def encode_cache(fmt: str, x, kf: int = 32):
-    """Encode one [T, D] tensor in format ``fmt`` ('delta', 'q4', 'fp16').
+def encode_cache(fmt: str, x, kf: int = 32, n_refs: int = 1):
+    """Encode one [T, D] tensor in format ``fmt`` ('delta', 'q4', 'fp16', or
+    'lr': long-range references at stride kf, the n_refs nearest).
 
     Returns a dict with the reconstruction ``xhat`` and the stored fields.
     """
     x = np.asarray(x, dtype=np.float32)
+    if fmt == "lr":
+        return lr_encode(x, kf, n_refs)
     if fmt == "delta":
         s = delta_encode(x, kf)
         return {"xhat": s.xhat, "kfr": s.kfr, "scales": s.scales, "codes": s.codes,

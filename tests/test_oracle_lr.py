@@ -94,3 +94,15 @@ def test_reconstruction_error_within_the_block_step(orc):
     ref_rows = np.arange(90) % 16 == 0
     lim = np.where(o["codes"] == 15, np.abs(d), np.abs(d) / 2) * (1 + 1e-6) + 1e-7
     assert (err[~ref_rows] <= lim[~ref_rows]).all()
+
+
+def test_attention_over_stride_one_is_the_fp16_cache(orc):
+    """A decode step over the long-range format with stride 1 (every token a
+    fp16 reference) is the decode step over the fp16 cache."""
+    rs = np.random.RandomState(12)
+    K = rs.randn(2, 2, 40, 64).astype(np.float32)
+    V = rs.randn(2, 2, 40, 64).astype(np.float32)
+    q = rs.randn(2, 4, 64)
+    a = orc.decode_attention("lr", q, K, V, kf=1, scale=0.125)
+    b = orc.decode_attention("fp16", q, K, V, kf=1, scale=0.125)
+    assert np.array_equal(a, b)
