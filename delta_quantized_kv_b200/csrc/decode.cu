@@ -36,7 +36,9 @@
 // state per sequence it touches, and writes one partial (max, sum, output)
 // record per such sequence.  The merge kernel combines the partial records
 // with a log-sum-exp.
+#include <atomic>
 #include <cstdint>
+#include <mutex>
 
 #include "dkv_common.cuh"
 #include "dkv_internal.h"
@@ -1349,28 +1351,44 @@ static size_t split_smem() {
     return (size_t)SmemMap<FMT, MODE>::BYTES;
 }
 
+// Per-device host state of the launches (the persistent grid of an instance,
+// whether an instance's shared-memory attribute is set), shared by every host
+// thread: read lock-free once published, computed under a mutex.
+constexpr int kMaxDevices = 64;
+static std::mutex g_launch_mu;
+
+static cudaError_t current_device(int *dev) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return e;
+    return (*dev < 0 || *dev >= kMaxDevices) ? cudaErrorInvalidDevice : cudaSuccess;
+}
+
 template <int FMT, int MODE, bool ZT>
 static cudaError_t geom_for(SplitGeom *g) {
-    static int cached_dev = -1, cached_ctas = 0;
+    static std::atomic<int> ctas_of[kMaxDevices];      // 0: not computed yet
     int dev;
-    cudaError_t e = cudaGetDevice(&dev);
+    cudaError_t e = current_device(&dev);
     if (e != cudaSuccess) return e;
-    if (dev != cached_dev) {
-        const size_t sm = split_smem<FMT, MODE>();
-        e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, false, false, false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
-        int per_sm = 0, nsm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm,
-                                                          split_kernel<FMT, MODE, ZT, false, false, false>,
-                                                          WARPS * 32, sm);
-        if (e != cudaSuccess) return e;
-        e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-        cached_ctas = (per_sm < 1 ? 1 : per_sm) * nsm;
-        cached_dev = dev;
+    int ctas = ctas_of[dev].load(std::memory_order_acquire);
+    if (ctas == 0) {
+        std::lock_guard<std::mutex> lock(g_launch_mu);
+        ctas = ctas_of[dev].load(std::memory_order_relaxed);
+        if (ctas == 0) {
+            const size_t sm = split_smem<FMT, MODE>();
+            e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, false, false, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            if (e != cudaSuccess) return e;
+            int per_sm = 0, nsm = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm, split_kernel<FMT, MODE, ZT, false, false, false>, WARPS * 32, sm);
+            if (e != cudaSuccess) return e;
+            e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            ctas = (per_sm < 1 ? 1 : per_sm) * nsm;
+            ctas_of[dev].store(ctas, std::memory_order_release);
+        }
     }
-    g->ctas = cached_ctas;
+    g->ctas = ctas;
     g->warps_per_cta = WARPS;
     return cudaSuccess;
 }
@@ -1396,16 +1414,19 @@ cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g) {
 template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP>
 static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
     if (PAGED || MQ || APP) {
-        static int set_dev = -1;                 // one flag per instance
+        static std::atomic<bool> set_on[kMaxDevices];   // per instance and device
         int dev;
-        cudaError_t e = cudaGetDevice(&dev);
+        cudaError_t e = current_device(&dev);
         if (e != cudaSuccess) return e;
-        if (dev != set_dev) {
-            e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, PAGED, MQ, APP>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)split_smem<FMT, MODE>());
-            if (e != cudaSuccess) return e;
-            set_dev = dev;
+        if (!set_on[dev].load(std::memory_order_acquire)) {
+            std::lock_guard<std::mutex> lock(g_launch_mu);
+            if (!set_on[dev].load(std::memory_order_relaxed)) {
+                e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, PAGED, MQ, APP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)split_smem<FMT, MODE>());
+                if (e != cudaSuccess) return e;
+                set_on[dev].store(true, std::memory_order_release);
+            }
         }
     }
     split_kernel<FMT, MODE, ZT, PAGED, MQ, APP><<<ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);

@@ -153,6 +153,8 @@ dkv_status check_decode(const dkv_cache *cache, const void *Q, int32_t q_dtype, 
 
 }  // namespace
 
+dkv_status dkv::validate_cache(const dkv_cache *c) { return check_cache(c); }
+
 extern "C" {
 
 int32_t dkv_abi_version(void) { return DKV_ABI_VERSION; }

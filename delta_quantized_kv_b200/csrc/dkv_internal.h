@@ -5,7 +5,13 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "../../include/dkv.h"
+
 namespace dkv {
+
+// The host-side checks every entry point runs on a cache view before any
+// launch: DKV_OK, or the status those entry points return for it.
+dkv_status validate_cache(const dkv_cache *c);
 
 struct CacheView;
 

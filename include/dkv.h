@@ -282,10 +282,15 @@ dkv_status dkv_lr_encode(const void *X, int32_t dtype, int32_t n_seq, int32_t T,
  * workspace.  The partial records go to a fixed 16 MiB array that the library
  * itself holds on every GPU that loads it, until the process exits.  The
  * first call on a device looks up that array's address (make it before any
- * stream capture).  Returns DKV_ECAPACITY when the step needs more than
- * DKV_NOALLOC_SCRATCH_BYTES of records (see dkv_decode_workspace_bytes).  All
- * calls share the array: calls that overlap on the GPU race and must be
- * serialised by the caller.  Allocates and frees nothing. */
+ * stream capture); the lookup is repeated only when the device's context has
+ * changed since (cudaDeviceReset loads the library's device code anew, so
+ * the array may move), which again must not happen under capture.  The cache
+ * is validated first, with the statuses of dkv_decode_attn (DKV_EINVAL,
+ * DKV_EALIGN, DKV_EUNSUPPORTED); then DKV_ECAPACITY when the step needs more
+ * than DKV_NOALLOC_SCRATCH_BYTES of records (see dkv_decode_workspace_bytes);
+ * DKV_ECUDA only for a failed device query or launch.  All calls share the
+ * array: calls that overlap on the GPU race and must be serialised by the
+ * caller.  Allocates and frees nothing. */
 dkv_status dkv_decode_attn_noalloc(const dkv_cache *cache, const void *Q, int32_t q_dtype,
                                    int32_t n_q_heads, float softmax_scale, float *out,
                                    void *stream);

@@ -113,6 +113,28 @@ def test_calls_on_an_invalid_cache_are_rejected(dkv):
     assert lib.dkv_get_device_status(ctypes.byref(c), ctypes.byref(w), None) == dkv.DKV_EINVAL
 
 
+def test_noalloc_gives_invalid_caches_the_statuses_of_dkv_decode_attn(dkv):
+    """The no-workspace decode validates the cache before it sizes the step,
+    so a bad descriptor gets the same status as from dkv_decode_attn (and
+    nothing touches the GPU)."""
+    lib = dkv.load()
+    for field, val, want in [("kf", 0, dkv.DKV_EINVAL), ("head_dim", 64, dkv.DKV_EUNSUPPORTED),
+                             ("fmt", 9, dkv.DKV_EINVAL), ("batch", 0, dkv.DKV_EINVAL),
+                             ("max_ctx", 0, dkv.DKV_EINVAL)]:
+        c = dkv.dkv_cache()
+        c.desc = _desc(dkv, B=2, H=2, cap=100)
+        setattr(c.desc, field, val)
+        c.base = 1 << 20
+        c.bytes = 1 << 30
+        got = lib.dkv_decode_attn_noalloc(ctypes.byref(c), 1 << 12, 1, 8, 1.0, 1 << 12, None)
+        ref = lib.dkv_decode_attn(ctypes.byref(c), 1 << 12, 1, 8, 1.0, 1 << 12, 1 << 12,
+                                  1 << 30, None)
+        assert got == ref == want, (field, got, ref, want)
+    c = dkv.dkv_cache()                                   # base == NULL
+    assert lib.dkv_decode_attn_noalloc(ctypes.byref(c), 1 << 12, 1, 8, 1.0, 1 << 12,
+                                       None) == dkv.DKV_EINVAL
+
+
 def test_bad_dtype_and_sizes_rejected_on_host(dkv):
     """A well-formed view whose arguments are wrong: nothing is launched."""
     lib = dkv.load()

@@ -1,9 +1,11 @@
 """dkv_decode_attn_noalloc: the decode step for callers that cannot allocate
 device memory when they decode (graph capture, engines that pre-plan every
-allocation).  Called through the C ABI, its output must match the regular
-dkv_decode_attn (which takes a caller-allocated workspace) within the
-attention tolerance, on two calls in a row (the second call reuses the
-library's scratch array with different queries).
+allocation).  Called through the C ABI, its output must equal the regular
+dkv_decode_attn (which takes a caller-allocated workspace) bit for bit: both
+run the same kernels on the same grid, only the scratch address differs.
+Checked on two calls in a row, after a differently shaped call has left its
+partial records in the library's shared scratch array (a stale record read by
+mistake would show).
 
 The file name sorts last so that a run stopping at the first failure has
 already run every other test."""
@@ -13,15 +15,28 @@ import pytest
 import torch
 
 import synthetic as S
-from _parity import ATTN_TOL, row_rel_err
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+def _stale_call(dkv):
+    """A decode through the no-workspace entry point on another shape, so the
+    shared array holds records that are not the next call's."""
+    w = S.WORKLOADS["llama3_8b_layer"].with_(B=5, Hkv=2, Hq=16, T=1300, kf=32)
+    K, V = S.gen_kv(w)
+    cache = dkv.Cache(w.B, w.Hkv, w.T, "delta", kf=32)
+    cache.encode(K.to(DEV), V.to(DEV))
+    q = (S.gen_q(w) * 4).to(DEV)
+    out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=DEV)
+    dkv.dkv_decode_attn_noalloc(cache.c, q, dkv.DKV_F16, w.Hq, 0.3, out)
+    torch.cuda.synchronize()
+
+
 @pytest.mark.parametrize("fmt,kf", [("delta", 32), ("delta", 512), ("q4", 32)])
 def test_noalloc_matches_workspace_entry_point(dkv_gpu, fmt, kf):
     dkv = dkv_gpu
+    _stale_call(dkv)
     w = S.WORKLOADS["llama3_70b_layer"].with_(B=3, Hkv=4, Hq=32, T=900, kf=kf)
     K, V = S.gen_kv(w)
     cache = dkv.Cache(w.B, w.Hkv, w.T, fmt, kf=kf)
@@ -37,8 +52,7 @@ def test_noalloc_matches_workspace_entry_point(dkv_gpu, fmt, kf):
         dkv.dkv_decode_attn_noalloc(cache.c, q, qcode, w.Hq, scale, got)
         torch.cuda.synchronize()
         assert cache.device_status() == 0
-        err = row_rel_err(got.cpu().numpy(), ref.cpu().numpy()).max()
-        assert err <= ATTN_TOL, (call, err)
+        assert torch.equal(got, ref), (call, (got - ref).abs().max().item())
 
 
 def test_noalloc_rejects_oversized_steps(dkv_gpu):
