@@ -337,17 +337,44 @@ QUALITY_CASES = [("tiny", None, None), ("llama3_8b_layer", None, None),
                  ("ragged_long", 32, None), ("ragged_long", 128, None), ("ragged_long", 512, None)]
 
 
-def quality_report(dev, max_batch: int = 2):
+def attention_space_terms(q, Kf, Vf, kh, vh, scale):
+    """The six sums behind the error report of one batch entry, over its
+    kv heads: squared reconstruction error and signal of K and V together;
+    sum (q.k^ - q.k)^2 and sum (q.k)^2 over the scores; |P V^ - P V|^2 and
+    |P V|^2, P the softmax over exact keys.  q [Hkv, G, D]; Kf, Vf, kh, vh
+    [Hkv, T, D] (float tensors, any device)."""
+    import torch
+    s_ref = torch.einsum("hgd,htd->hgt", q, Kf)
+    P = torch.softmax(s_ref * scale, dim=-1)
+    o_ref = torch.einsum("hgt,htd->hgd", P, Vf)
+    s_h = torch.einsum("hgd,htd->hgt", q, kh)
+    o_h = torch.einsum("hgt,htd->hgd", P, vh)
+    return [((kh - Kf) ** 2).sum().item() + ((vh - Vf) ** 2).sum().item(),
+            (Kf ** 2).sum().item() + (Vf ** 2).sum().item(),
+            ((s_h - s_ref) ** 2).sum().item(), (s_ref ** 2).sum().item(),
+            ((o_h - o_ref) ** 2).sum().item(), (o_ref ** 2).sum().item()]
+
+
+def quality_report(dev, max_batch: int = 2, recon=None, cases=None):
     """Per workload (and kf): relative reconstruction MSE of the delta, Q4_0 and
     fp16 caches against the input, and the attention-space errors
     D_K = sum (q.k^ - q.k)^2 / sum (q.k)^2 and D_V = |P V^ - P V|^2 / |P V|^2
-    with P the softmax over exact keys.  Reconstructions come from the
-    library's dequantize; the first `max_batch` batch entries of each."""
-    import torch
-    import delta_quantized_kv_b200 as dkv
+    with P the softmax over exact keys.  Reconstructions come from
+    `recon(fmt, K, V, kf)` ([Hkv, T, D] each; default: the library's
+    dequantize of a one-entry cache); the first `max_batch` batch entries of
+    each workload."""
     import synthetic as S
+    if recon is None:
+        import delta_quantized_kv_b200 as dkv
+
+        def recon(fmt, K, V, kf):
+            T = K.shape[1]
+            c = dkv.Cache(1, K.shape[0], T, fmt, kf=kf, device=dev)
+            c.encode(K[None].contiguous(), V[None].contiguous())
+            xh = c.dequantize()[0]                      # [Hkv, 2, cap, D]
+            return xh[:, 0, :T], xh[:, 1, :T]
     rep = {}
-    for name, kf, gen in QUALITY_CASES:
+    for name, kf, gen in (QUALITY_CASES if cases is None else cases):
         w = S.WORKLOADS[name]
         if kf:
             w = w.with_(kf=kf)
@@ -356,30 +383,16 @@ def quality_report(dev, max_batch: int = 2):
         lens = S.gen_lengths(w)
         G = w.Hq // w.Hkv
         scale = 1.0 / math.sqrt(w.D)
-        acc = {f: [0.0, 0.0, 0.0, 0.0, 0.0, 0.0] for f in ("delta", "q4", "fp16")}
+        acc = {f: [0.0] * 6 for f in ("delta", "q4", "fp16")}
         for b in range(min(w.B, max_batch)):
             T = lens[b]
             K, V = S.gen_kv_one(w, b, T, device=dev)
             q = S.gen_q(w, device=dev)[b].float().view(w.Hkv, G, w.D)
-            Kf, Vf = K.float(), V.float()
-            s_ref = torch.einsum("hgd,htd->hgt", q, Kf)
-            P = torch.softmax(s_ref * scale, dim=-1)
-            o_ref = torch.einsum("hgt,htd->hgd", P, Vf)
             for f in acc:
-                c = dkv.Cache(1, w.Hkv, T, f, kf=w.kf, device=dev)
-                c.encode(K[None].contiguous(), V[None].contiguous())
-                xh = c.dequantize()[0]                      # [Hkv, 2, cap, D]
-                kh, vh = xh[:, 0, :T], xh[:, 1, :T]
-                s_h = torch.einsum("hgd,htd->hgt", q, kh)
-                o_h = torch.einsum("hgt,htd->hgd", P, vh)
-                a = acc[f]
-                a[0] += ((kh - Kf) ** 2).sum().item() + ((vh - Vf) ** 2).sum().item()
-                a[1] += (Kf ** 2).sum().item() + (Vf ** 2).sum().item()
-                a[2] += ((s_h - s_ref) ** 2).sum().item()
-                a[3] += (s_ref ** 2).sum().item()
-                a[4] += ((o_h - o_ref) ** 2).sum().item()
-                a[5] += (o_ref ** 2).sum().item()
-                del c, xh
+                kh, vh = recon(f, K, V, w.kf)
+                for i, v in enumerate(attention_space_terms(q, K.float(), V.float(), kh, vh,
+                                                            scale)):
+                    acc[f][i] += v
         key = name + (f"_kf{w.kf}" if kf else "") + (f"_{gen}" if gen else "")
         rep[key] = {f: {"rel_mse": a[0] / a[1], "D_K": a[2] / a[3], "D_V": a[4] / a[5]}
                     for f, a in acc.items()}

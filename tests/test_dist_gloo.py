@@ -106,3 +106,49 @@ def test_long_range_quality_report_logic():
     assert set(row) == {"lr_1_ref", "lr_4_ref", "delta", "q4"}
     assert all(np.isfinite(v) and v >= 0 for v in row.values())
     assert row["lr_1_ref"] < 0.1 * row["q4"]
+
+
+def test_quality_report_arithmetic_against_numpy():
+    """bench.quality_report's error figures, with the oracle's reconstruction
+    standing in for the GPU caches, against the same quantities written out in
+    numpy float64: relative MSE sum (x^ - x)^2 / sum x^2 over K and V;
+    D_K = sum (q.k^ - q.k)^2 / sum (q.k)^2; D_V = |P V^ - P V|^2 / |P V|^2 with
+    P the softmax of the scaled exact scores."""
+    import numpy as np
+    import torch
+    import bench
+    import oracle
+    import synthetic as S
+
+    def recon(fmt, K, V, kf):
+        f = lambda A: torch.stack([torch.from_numpy(
+            oracle.encode_cache(fmt, A[i].float().numpy(), kf)["xhat"]) for i in range(A.shape[0])])
+        return f(K), f(V)
+
+    cases = [("tiny", None, None), ("llama3_8b_layer", None, None)]
+    rep = bench.quality_report("cpu", max_batch=1, recon=recon, cases=cases)
+    for name, _, _ in cases:
+        w = S.WORKLOADS[name]
+        K, V = S.gen_kv_one(w, 0, w.T)
+        G = w.Hq // w.Hkv
+        q = S.gen_q(w)[0].double().numpy().reshape(w.Hkv, G, w.D)
+        x = np.concatenate([K.double().numpy(), V.double().numpy()])
+        for fmt in ("delta", "q4", "fp16"):
+            kh, vh = (t.double().numpy() for t in recon(fmt, K, V, w.kf))
+            xh = np.concatenate([kh, vh])
+            rel = ((xh - x) ** 2).sum() / (x ** 2).sum()
+            s_ref = np.einsum("hgd,htd->hgt", q, K.double().numpy())
+            s_hat = np.einsum("hgd,htd->hgt", q, kh)
+            z = s_ref / np.sqrt(w.D)
+            P = np.exp(z - z.max(axis=-1, keepdims=True))
+            P /= P.sum(axis=-1, keepdims=True)
+            o_ref = np.einsum("hgt,htd->hgd", P, V.double().numpy())
+            o_hat = np.einsum("hgt,htd->hgd", P, vh)
+            dk = ((s_hat - s_ref) ** 2).sum() / (s_ref ** 2).sum()
+            dv = ((o_hat - o_ref) ** 2).sum() / (o_ref ** 2).sum()
+            got = rep[name][fmt]
+            assert got["rel_mse"] == pytest.approx(rel, rel=1e-5, abs=1e-12), (name, fmt)
+            assert got["D_K"] == pytest.approx(dk, rel=2e-2, abs=1e-12), (name, fmt)
+            assert got["D_V"] == pytest.approx(dv, rel=2e-2, abs=1e-12), (name, fmt)
+        assert rep[name]["entries"] == 1
+        assert rep[name]["delta"]["rel_mse"] < rep[name]["q4"]["rel_mse"]
