@@ -464,17 +464,17 @@ __device__ inline float col_scan32(float (&v)[4], int lane) {
 //   (movmatrix) of the K-side accumulator layout.
 
 // K side of one unit: per-position dot products x[t][r][e] (position
-// 4g + 2t + r, head 2tq + e) and the V scales dvw[t][r] of those positions.
+// 4g + 2t + r, head 2tq + e).
 // ZT: zero the scales of slots past the unit's end.  Needed where such a slot
 // can read bytes that are not scale rows (kf < 32: the next record's nibbles,
 // whose fp16 reading may be NaN); with kf = 32 and for Q4_0 a slot past the end
 // reads a scale row of the cache (zeroed at init, else written by the encoder)
 // or of an older stage, always finite, and the softmax mask alone handles it.
-template <int FMT, int MODE, bool ZT>
+template <int FMT, int MODE, bool ZT, bool QHL>
 __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, bool first_seg,
                               int gq, int tq, uint32_t m1024, uint32_t m64,
-                              const uint32_t (&qb)[8][2], float (&x)[2][2][2],
-                              uint32_t (&dvw)[2][2][2]) {
+                              const uint32_t (&qb)[8][2], const uint32_t (&ql)[8][2],
+                              float (&x)[2][2][2]) {
     const bool kfrow = first_seg && gq == 0;   // this thread's row 0 of tile 0 is the keyframe
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
@@ -488,10 +488,13 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
                 const uint4 u1 = *reinterpret_cast<const uint4 *>(k0 + 256 + 16 * q4);
                 mma16816(acc, u0.x, u1.x, u0.y, u1.y, qb[2 * q4][0], qb[2 * q4][1]);
                 mma16816(acc, u0.z, u1.z, u0.w, u1.w, qb[2 * q4 + 1][0], qb[2 * q4 + 1][1]);
+                if (QHL) {
+                    mma16816(acc, u0.x, u1.x, u0.y, u1.y, ql[2 * q4][0], ql[2 * q4][1]);
+                    mma16816(acc, u0.z, u1.z, u0.w, u1.w, ql[2 * q4 + 1][0], ql[2 * q4 + 1][1]);
+                }
             }
             x[t][0][0] = acc[0]; x[t][0][1] = acc[1];
             x[t][1][0] = acc[2]; x[t][1][1] = acc[3];
-            dvw[t][0][0] = dvw[t][0][1] = dvw[t][1][0] = dvw[t][1][1] = 0u;
         } else {
             const uint4 w0 = *reinterpret_cast<const uint4 *>(st + sm.kn0 + p0 * NIB_BYTES + 16 * tq);
             const uint4 w1 = *reinterpret_cast<const uint4 *>(st + sm.kn0 + (p0 + 1) * NIB_BYTES + 16 * tq);
@@ -528,22 +531,22 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
                          qb[2 * j][0], qb[2 * j][1]);
                 mma16816(acc[j], a[2 * j + 1][0], a[2 * j + 1][1], a[2 * j + 1][2],
                          a[2 * j + 1][3], qb[2 * j + 1][0], qb[2 * j + 1][1]);
+                if (QHL) {
+                    mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
+                             ql[2 * j][0], ql[2 * j][1]);
+                    mma16816(acc[j], a[2 * j + 1][0], a[2 * j + 1][1], a[2 * j + 1][2],
+                             a[2 * j + 1][3], ql[2 * j + 1][0], ql[2 * j + 1][1]);
+                }
             }
-            // scales of positions p0, p0+1: dK (blocks 0..3) then dV
-            uint4 s0 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + p0 * SC_BYTES);
-            uint4 s1 = *reinterpret_cast<const uint4 *>(st + sm.sc0 + (p0 + 1) * SC_BYTES);
-            if (FMT == DKV_FMT_DELTA && t == 0 && kfrow) {
-                // keyframe: unit K weights; no V weight in the MMAs (its V
-                // contribution is added apart, in fp32)
-                s0.x = s0.y = 0x3C003C00u;
-                s0.z = s0.w = 0u;
-            }
+            // K scales of positions p0, p0+1 (blocks 0..3; the V scales
+            // follow in the same 16-byte row and are read by the V side)
+            uint2 s0 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + p0 * SC_BYTES);
+            uint2 s1 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + (p0 + 1) * SC_BYTES);
+            if (FMT == DKV_FMT_DELTA && t == 0 && kfrow) s0.x = s0.y = 0x3C003C00u;  // keyframe: unit
             if (ZT) {
-                if (p0 >= npos) s0 = make_uint4(0u, 0u, 0u, 0u);
-                if (p0 + 1 >= npos) s1 = make_uint4(0u, 0u, 0u, 0u);
+                if (p0 >= npos) s0 = make_uint2(0u, 0u);
+                if (p0 + 1 >= npos) s1 = make_uint2(0u, 0u);
             }
-            dvw[t][0][0] = s0.z; dvw[t][0][1] = s0.w;
-            dvw[t][1][0] = s1.z; dvw[t][1][1] = s1.w;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 float x0 = acc[0][e] * h_lo(s0.x);
@@ -561,11 +564,12 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
 
 // V side of one unit: o += sum over positions of dequantised V rows times the
 // weights w[t][r][e] (position 4g + 2t + r, head 2tq + e) and their V scales.
-template <int FMT, int MODE>
+// The V scales are read here rather than kept from the K side (registers).
+template <int FMT, int MODE, bool ZT>
 __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, bool first_seg,
                               int gq, int tq, uint32_t m1024, uint32_t m64,
-                              const float (&w)[2][2][2], const uint32_t (&dvw)[2][2][2],
-                              float (&o)[8][4], float (&racc)[8][4], uint32_t (&vkf_keep)[8]) {
+                              const float (&w)[2][2][2], float (&o)[8][4], float (&racc)[8][4],
+                              uint32_t (&vkf_keep)[8]) {
     uint32_t vkf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     if (FMT == DKV_FMT_DELTA && first_seg) {
         const uint4 v0 = *reinterpret_cast<const uint4 *>(st + sm.vk0 + 32 * gq);
@@ -605,6 +609,22 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
             }
             continue;
         }
+        // V scales of positions 4g + 2t + r (the weights' positions): zero on the
+        // keyframe row (its V part is added apart, in fp32) and, with ZT, on
+        // slots past the unit's end
+        uint32_t dvw[2][2];
+        {
+            const int p0 = 4 * gq + 2 * t;
+            uint2 s0 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + p0 * SC_BYTES + 8);
+            uint2 s1 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + (p0 + 1) * SC_BYTES + 8);
+            if (FMT == DKV_FMT_DELTA && t == 0 && first_seg && gq == 0) s0 = make_uint2(0u, 0u);
+            if (ZT) {
+                if (p0 >= npos) s0 = make_uint2(0u, 0u);
+                if (p0 + 1 >= npos) s1 = make_uint2(0u, 0u);
+            }
+            dvw[0][0] = s0.x; dvw[0][1] = s0.y;
+            dvw[1][0] = s1.x; dvw[1][1] = s1.y;
+        }
         // V nibbles of positions 8tq + 2t + {0, 1, 4, 5}, chunk g
         const uint8_t *vb = st + sm.vn0 + (8 * tq + 2 * t) * NIB_BYTES + 8 * gq;
         const uint2 wP0 = *reinterpret_cast<const uint2 *>(vb);
@@ -622,25 +642,52 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
             dq_pair(m23, m1024, m64, a2, a3);
         };
         if (MODE != PREFIX) {
-            // B fragments (k = positions, n = head g) of block j: the weights
-            // packed to fp16 once, times block j's V scale in one fp16x2
-            // multiply, then the 8x8 transpose into the B layout
+            // B fragments (k = positions, n = head g) of block j: the weight of
+            // each row times block j's V scale, then the 8x8 transpose into the
+            // B layout.  Delta format: the weights are suffix sums S_s, and the
+            // terms delta^_s * S_s cancel to the much smaller output whenever
+            // consecutive tokens differ a lot (jumps, unrelated tokens), so one
+            // fp16 value of S_s * d_s (relative error 2^-11) can give outputs
+            // off by 1 %.  There every B value is an fp16 pair hi + lo:
+            //   hi = fp16(fp16(S) * d);  lo = fp16(fp16(S - fp16(S)) * d +
+            //   (fp16(S) * d - hi)), the bracket exact (one fused multiply-add
+            //   returns the rounding error of a product exactly),
+            // with the second MMA against the same A fragment, for a relative
+            // error near 2^-21.  The comparators (one token per row) keep one
+            // fp16 weight, as flash-decoding does.
+            constexpr bool HL = FMT == DKV_FMT_DELTA;
             const uint32_t wp0 = pack_h2(w[t][0][0], w[t][0][1]);
             const uint32_t wp1 = pack_h2(w[t][1][0], w[t][1][1]);
-            auto make_b = [&](int j, uint32_t (&b)[2]) {
-                const uint32_t u0 = dvw[t][0][j >> 1], u1 = dvw[t][1][j >> 1];
+            uint32_t wl0 = 0, wl1 = 0;
+            if (HL) {
+                wl0 = pack_h2(w[t][0][0] - h_lo(wp0), w[t][0][1] - h_hi(wp0));
+                wl1 = pack_h2(w[t][1][0] - h_lo(wp1), w[t][1][1] - h_hi(wp1));
+            }
+            auto make_b = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2]) {
+                const uint32_t u0 = dvw[0][j >> 1], u1 = dvw[1][j >> 1];
                 const __half2 d0 = (j & 1) ? __high2half2(u32_as_h2(u0)) : __low2half2(u32_as_h2(u0));
                 const __half2 d1 = (j & 1) ? __high2half2(u32_as_h2(u1)) : __low2half2(u32_as_h2(u1));
-                b[0] = movm_t(h2_as_u32(__hmul2(u32_as_h2(wp0), d0)));
-                b[1] = movm_t(h2_as_u32(__hmul2(u32_as_h2(wp1), d1)));
+                const __half2 h0 = __hmul2(u32_as_h2(wp0), d0);
+                const __half2 h1 = __hmul2(u32_as_h2(wp1), d1);
+                b[0] = movm_t(h2_as_u32(h0));
+                b[1] = movm_t(h2_as_u32(h1));
+                if (HL) {
+                    const __half2 l0 = __hfma2(u32_as_h2(wl0), d0,
+                                               __hfma2(u32_as_h2(wp0), d0, __hneg2(h0)));
+                    const __half2 l1 = __hfma2(u32_as_h2(wl1), d1,
+                                               __hfma2(u32_as_h2(wp1), d1, __hneg2(h1)));
+                    bl[0] = movm_t(h2_as_u32(l0));
+                    bl[1] = movm_t(h2_as_u32(l1));
+                }
             };
-            uint32_t bp[2];
+            uint32_t bp[2], bq[2] = {0u, 0u};
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 uint32_t a0, a1, a2, a3;
                 codes(mt, a0, a1, a2, a3);
-                if ((mt & 1) == 0) make_b(mt >> 1, bp);
+                if ((mt & 1) == 0) make_b(mt >> 1, bp, bq);
                 mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
+                if (HL) mma16816(o[mt], a0, a1, a2, a3, bq[0], bq[1]);
             }
             if (FMT == DKV_FMT_DELTA && t == 0) {
                 // keyframe row: o += v_f * (the group's total weight), in fp32;
@@ -663,7 +710,7 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
             auto make_b = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2]) {
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
-                    const uint32_t u = dvw[t][r][j >> 1];
+                    const uint32_t u = dvw[r][j >> 1];
                     const float d = (j & 1) ? h_hi(u) : h_lo(u);
                     const float v0 = w[t][r][0] * d, v1 = w[t][r][1] * d;
                     const uint32_t hi = pack_h2(v0, v1);
@@ -684,7 +731,7 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
                 uint32_t r2[2];
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
-                    const uint32_t u = dvw[t][r][j >> 1];
+                    const uint32_t u = dvw[r][j >> 1];
                     const float d = (j & 1) ? h_hi(u) : h_lo(u);
                     r2[r] = movm_t(pack_h2(d, d));
                 }
@@ -861,9 +908,10 @@ __device__ __noinline__ bool append_range(const SplitArgs &A, int nvs, int b, in
 // MQ: several causal queries per sequence (virtual heads with their own
 // position limits); the one-query instance keeps the plain tail mask.  APP:
 // the fused append (the kernel parameters stay in the constant bank while the
-// append functions take their address).
-template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP>
-__global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB))
+// append functions take their address).  QHL: fp32 queries as an fp16 hi + lo
+// pair (two MMAs per K-side step; the extra registers cost a CTA per SM).
+template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP, bool QHL>
+__global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
     split_kernel(const __grid_constant__ SplitArgs A) {
     using Cfg = KCfg<FMT, MODE>;
     constexpr int NS = Cfg::NS, STAGE = Cfg::STAGE, NU = Cfg::NU;
@@ -967,6 +1015,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB))
     // per-sequence state (heads 2*tq + e of the current head group)
     int cur_b = -1, cur_vs = -1;
     uint32_t qb[8][2];                  // B fragments of q (column = head gq)
+    uint32_t ql[8][2];                  // QHL: the fp16 remainders q - qb
     int lp[2] = {0, 0};                 // positions heads 2tq + e may see (causal queries)
     float m_run[2] = {-1e30f, -1e30f}, l_run[2] = {0.f, 0.f};
     float o[8][4];
@@ -1055,6 +1104,12 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB))
                 }
                 qb[kk][0] = pack_h2(q0, q1);
                 qb[kk][1] = pack_h2(q8, q9);
+                if (QHL) {
+                    // fp32 queries: q = hi + lo, both fp16, so q . k keeps
+                    // about 22 bits (bf16 and fp16 queries are exact in hi)
+                    ql[kk][0] = pack_h2(q0 - h_lo(qb[kk][0]), q1 - h_hi(qb[kk][0]));
+                    ql[kk][1] = pack_h2(q8 - h_lo(qb[kk][1]), q9 - h_hi(qb[kk][1]));
+                }
             }
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -1076,15 +1131,14 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB))
 
             // ================= K side ======================================
             float x[NU][2][2][2];
-            uint32_t dvw[NU][2][2][2];
             // Both units go through the same straight-line code; a unit the stage
             // does not hold has npos 0, so all its slots are masked and its scales
             // zeroed (its shared-memory bytes are an older stage's, always finite).
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
-                k_side<FMT, MODE, ZT>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, qb, x[u],
-                                      dvw[u]);
+                k_side<FMT, MODE, ZT, QHL>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, qb,
+                                           ql, x[u]);
             }
 
             // ================= scores, online softmax =======================
@@ -1185,7 +1239,7 @@ __global__ void __launch_bounds__(WARPS * 32, (KCfg<FMT, MODE>::MINB))
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
-                v_side<FMT, MODE>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, x[u], dvw[u], o,
+                v_side<FMT, MODE, ZT>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, x[u], o,
                                   racc, vkf_keep);
             }
 
@@ -1375,12 +1429,12 @@ static cudaError_t geom_for(SplitGeom *g) {
         ctas = ctas_of[dev].load(std::memory_order_relaxed);
         if (ctas == 0) {
             const size_t sm = split_smem<FMT, MODE>();
-            e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, false, false, false>,
+            e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, false, false, false, false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
             if (e != cudaSuccess) return e;
             int per_sm = 0, nsm = 0;
             e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                &per_sm, split_kernel<FMT, MODE, ZT, false, false, false>, WARPS * 32, sm);
+                &per_sm, split_kernel<FMT, MODE, ZT, false, false, false, false>, WARPS * 32, sm);
             if (e != cudaSuccess) return e;
             e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
             if (e != cudaSuccess) return e;
@@ -1411,9 +1465,9 @@ cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g) {
 // Every instance runs on the contiguous one-query instance's grid (the merge
 // and the workspace size follow that grid); a persistent grid is correct at
 // any size.
-template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP>
+template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP, bool QHL>
 static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
-    if (PAGED || MQ || APP) {
+    if (PAGED || MQ || APP || QHL) {
         static std::atomic<bool> set_on[kMaxDevices];   // per instance and device
         int dev;
         cudaError_t e = current_device(&dev);
@@ -1421,7 +1475,7 @@ static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
         if (!set_on[dev].load(std::memory_order_acquire)) {
             std::lock_guard<std::mutex> lock(g_launch_mu);
             if (!set_on[dev].load(std::memory_order_relaxed)) {
-                e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, PAGED, MQ, APP>,
+                e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, PAGED, MQ, APP, QHL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)split_smem<FMT, MODE>());
                 if (e != cudaSuccess) return e;
@@ -1429,8 +1483,16 @@ static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
             }
         }
     }
-    split_kernel<FMT, MODE, ZT, PAGED, MQ, APP><<<ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
+    split_kernel<FMT, MODE, ZT, PAGED, MQ, APP, QHL>
+        <<<ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
     return cudaGetLastError();
+}
+
+// fp32 queries take the hi + lo instance
+template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP>
+static cudaError_t launch_q(const SplitArgs &a, int ctas, cudaStream_t st) {
+    return a.q_dtype == DKV_F32 ? launch_inst<FMT, MODE, ZT, PAGED, MQ, APP, true>(a, ctas, st)
+                                : launch_inst<FMT, MODE, ZT, PAGED, MQ, APP, false>(a, ctas, st);
 }
 
 template <int FMT, int MODE, bool ZT>
@@ -1440,17 +1502,17 @@ static cudaError_t launch_split_t(const SplitArgs &a_in, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const SplitArgs &a = a_in;
     const bool paged = a.cv.pg != 0, mq = a.nq > 1, app = a.cv.len_add > 0;
-    if (!paged && !mq && !app) return launch_inst<FMT, MODE, ZT, false, false, false>(a, g.ctas, st);
+    if (!paged && !mq && !app) return launch_q<FMT, MODE, ZT, false, false, false>(a, g.ctas, st);
     if constexpr (FMT == DKV_FMT_DELTA) {        // only the delta format pages / takes queries
         if (app) {
-            if (paged && mq) return launch_inst<FMT, MODE, ZT, true, true, true>(a, g.ctas, st);
-            if (paged) return launch_inst<FMT, MODE, ZT, true, false, true>(a, g.ctas, st);
-            if (mq) return launch_inst<FMT, MODE, ZT, false, true, true>(a, g.ctas, st);
-            return launch_inst<FMT, MODE, ZT, false, false, true>(a, g.ctas, st);
+            if (paged && mq) return launch_q<FMT, MODE, ZT, true, true, true>(a, g.ctas, st);
+            if (paged) return launch_q<FMT, MODE, ZT, true, false, true>(a, g.ctas, st);
+            if (mq) return launch_q<FMT, MODE, ZT, false, true, true>(a, g.ctas, st);
+            return launch_q<FMT, MODE, ZT, false, false, true>(a, g.ctas, st);
         }
-        if (paged && mq) return launch_inst<FMT, MODE, ZT, true, true, false>(a, g.ctas, st);
-        if (paged) return launch_inst<FMT, MODE, ZT, true, false, false>(a, g.ctas, st);
-        return launch_inst<FMT, MODE, ZT, false, true, false>(a, g.ctas, st);
+        if (paged && mq) return launch_q<FMT, MODE, ZT, true, true, false>(a, g.ctas, st);
+        if (paged) return launch_q<FMT, MODE, ZT, true, false, false>(a, g.ctas, st);
+        return launch_q<FMT, MODE, ZT, false, true, false>(a, g.ctas, st);
     } else {
         return cudaErrorInvalidValue;
     }

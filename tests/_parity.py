@@ -41,3 +41,29 @@ def export_np(cache):
             a = a.view(np.uint16)
         out[k] = a
     return out
+
+
+def assert_fields_equal(orc, cache, fmt, K, V, lens, kf, cap):
+    """Every stored field of every (batch, kv head, tensor) sequence of the
+    cache equals the oracle's encoding of the same tokens, bit for bit."""
+    ex = export_np(cache)
+    B, H = K.shape[0], K.shape[1]
+    for b in range(B):
+        for h in range(H):
+            for t, X in enumerate((K, V)):
+                x = np.asarray(X[b, h, :lens[b]], dtype=np.float32)
+                ref = oracle_fields(orc, fmt, x, kf, cap)
+                for k, r in ref.items():
+                    got = ex[k][b, h, t]
+                    if k == "keyframes" and fmt == "delta":
+                        got = got[: r.shape[0]]
+                    if k == "state":
+                        if lens[b] == 0:
+                            continue
+                        assert np.array_equal(got.view(np.uint32), r.view(np.uint32)), \
+                            (b, h, t, k)
+                    else:
+                        bad = np.argwhere(got != r)
+                        assert bad.size == 0, (fmt, b, h, t, k, bad[:3].tolist(),
+                                               [int(got[tuple(i)]) for i in bad[:3]],
+                                               [int(r[tuple(i)]) for i in bad[:3]])
