@@ -609,15 +609,17 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
             }
             continue;
         }
-        // V scales of positions 4g + 2t + r (the weights' positions): zero on the
-        // keyframe row (its V part is added apart, in fp32) and, with ZT, on
-        // slots past the unit's end
+        // V scales of positions 4g + 2t + r (the weights' positions).  On the
+        // keyframe row: 1 for whole groups (v_f rides the MMA, below), 0 for
+        // segments (kf > 32: v_f is added when the group closes).  With ZT, 0
+        // on slots past the unit's end.
         uint32_t dvw[2][2];
         {
             const int p0 = 4 * gq + 2 * t;
             uint2 s0 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + p0 * SC_BYTES + 8);
             uint2 s1 = *reinterpret_cast<const uint2 *>(st + sm.sc0 + (p0 + 1) * SC_BYTES + 8);
-            if (FMT == DKV_FMT_DELTA && t == 0 && first_seg && gq == 0) s0 = make_uint2(0u, 0u);
+            if (FMT == DKV_FMT_DELTA && t == 0 && first_seg && gq == 0)
+                s0 = MODE == PREFIX ? make_uint2(0u, 0u) : make_uint2(0x3C003C00u, 0x3C003C00u);
             if (ZT) {
                 if (p0 >= npos) s0 = make_uint2(0u, 0u);
                 if (p0 + 1 >= npos) s1 = make_uint2(0u, 0u);
@@ -680,28 +682,23 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
                     bl[1] = movm_t(h2_as_u32(l1));
                 }
             };
+            // Delta format: slot 0 of tile 0 is the keyframe position, which has
+            // no delta row; its A entries (the low halves of a0 / a1 on the
+            // lanes with tq = 0) take v_f itself, and its scale is 1, so the
+            // MMA adds v_f times the group's total weight (S of position 0).
+            const bool kf_slot = FMT == DKV_FMT_DELTA && t == 0 && first_seg && tq == 0;
             uint32_t bp[2], bq[2] = {0u, 0u};
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 uint32_t a0, a1, a2, a3;
                 codes(mt, a0, a1, a2, a3);
+                if (kf_slot) {
+                    a0 = prmt(a0, vkf[mt], 0x3254u);   // channel 16mt + g
+                    a1 = prmt(a1, vkf[mt], 0x3276u);   // channel 16mt + g + 8
+                }
                 if ((mt & 1) == 0) make_b(mt >> 1, bp, bq);
                 mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
                 if (HL) mma16816(o[mt], a0, a1, a2, a3, bq[0], bq[1]);
-            }
-            if (FMT == DKV_FMT_DELTA && t == 0) {
-                // keyframe row: o += v_f * (the group's total weight), in fp32;
-                // the total of heads 2tq + e sits in w[0][0][e] of lane tq (g = 0)
-                const float S0 = __shfl_sync(0xffffffffu, w[0][0][0], tq);
-                const float S1 = __shfl_sync(0xffffffffu, w[0][0][1], tq);
-#pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
-                    const float vl = h_lo(vkf[mt]), vh = h_hi(vkf[mt]);
-                    o[mt][0] = fmaf(vl, S0, o[mt][0]);
-                    o[mt][1] = fmaf(vl, S1, o[mt][1]);
-                    o[mt][2] = fmaf(vh, S0, o[mt][2]);
-                    o[mt][3] = fmaf(vh, S1, o[mt][3]);
-                }
             }
         } else {
             // PREFIX (kf > 32): the prefix weights -E_s aggregate up to kf
