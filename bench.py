@@ -434,6 +434,195 @@ def lr_quality(dev, lr_encode, recon):
     return out
 
 
+def lr_decode_bench(dev, T=4096, stride=32, n_refs=1, n_iter=10):
+    """Decode over the long-range reference encoding (dkv_lr_decode_attn)
+    beside the delta cache's decode, on the same window-repeat tokens
+    (batched_decode shape, context T): split/step times, GB/s of the bytes
+    each format stores and reads, and the relative attention difference of
+    the two outputs.  The long-range encoding is the canonical one
+    dkv_lr_encode writes (one byte per code)."""
+    import torch
+    import delta_quantized_kv_b200 as dkv
+    import synthetic as S
+    w = S.WORKLOADS["batched_decode"].with_(T=T, gen="repeat")
+    B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
+    K = torch.empty((B, Hkv, T, D), dtype=w.kv_dtype, device=dev)
+    V = torch.empty_like(K)
+    for b in range(B):
+        K[b], V[b] = S.gen_kv_one(w, b, T, device=dev)
+    q = S.gen_q(w, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    ek = dkv.lr_encode(K.reshape(B * Hkv, T, D).contiguous(), stride, n_refs)
+    ev = dkv.lr_encode(V.reshape(B * Hkv, T, D).contiguous(), stride, n_refs)
+    nbw = dkv.dkv_lr_decode_workspace_bytes(B, Hkv, T, stride)
+    ws = torch.empty(nbw // 4 + 64, dtype=torch.float32, device=dev)
+    out_lr = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    st = torch.cuda.current_stream()
+    run = lambda: dkv.lr_decode_attn(ek, ev, q, scale, stride, Hkv, out=out_lr, workspace=ws)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(n_iter):
+        run()
+    e1.record(st)
+    torch.cuda.synchronize()
+    t_lr = e0.elapsed_time(e1) / n_iter
+    nr = -(-T // stride)
+    lr_bytes = B * Hkv * 2 * (T * (D + 8 + 4 * n_refs) + nr * 2 * D)
+    c = dkv.Cache(B, Hkv, T, "delta", kf=stride, device=dev)
+    c.encode(K, V)
+    out_d = torch.empty_like(out_lr)
+    for _ in range(3):
+        c.decode_attn(q, scale, out=out_d)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(n_iter):
+        c.decode_attn(q, scale, out=out_d)
+    e1.record(st)
+    torch.cuda.synchronize()
+    t_d = e0.elapsed_time(e1) / n_iter
+    d_bytes = kv_bytes("delta", [T] * B, Hkv, stride)
+    diff = ((out_lr - out_d).abs().amax(-1) / out_d.abs().amax(-1)).max().item()
+    return {"workload": f"batched_decode repeat, T {T}, stride/kf {stride}, {n_refs} reference(s)",
+            "lr_step_us": 1e3 * t_lr, "lr_bytes": lr_bytes,
+            "lr_gbps": lr_bytes / (t_lr * 1e-3) / 1e9,
+            "delta_step_us": 1e3 * t_d, "delta_bytes": d_bytes,
+            "delta_gbps": d_bytes / (t_d * 1e-3) / 1e9,
+            "max_row_rel_diff_lr_vs_delta": diff}
+
+
+# ---------------------------------------------------------------------------
+# every workload configuration, timed (kernel-level, rank 0, outside the step)
+# ---------------------------------------------------------------------------
+CONFIG_CASES = [
+    # (label, workload, overrides)
+    ("llama3_8b_layer", "llama3_8b_layer", {}),
+    ("batched_decode_kf32", "batched_decode", {"kf": 32}),
+    ("batched_decode_kf512", "batched_decode", {"kf": 512}),
+    ("batched_decode_kf32_repeat", "batched_decode", {"kf": 32, "gen": "repeat"}),
+    ("ragged_long_kf32", "ragged_long", {"kf": 32}),
+    ("ragged_long_kf128", "ragged_long", {"kf": 128}),
+    ("ragged_long_kf512", "ragged_long", {"kf": 512}),
+]
+
+
+def time_config(dev, w, peak, n_iter=10):
+    """One workload configuration end to end on the GPU: encode its (ragged)
+    prefix, then its per-token appends (ragged workload: 256 single-token
+    dkv_append calls), then the decode step (split and merge launches timed
+    apart with CUDA events).  A cache smaller than 4x L2 is rotated over
+    enough identical copies that every decode reads HBM.  Returns GB/s of
+    compressed bytes, fractions of the peaks and KV-token.heads/s."""
+    import torch
+    import delta_quantized_kv_b200 as dkv
+    import synthetic as S
+    B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
+    lens0 = S.gen_lengths(w)
+    n_app = w.n_append
+    Tmax = max(lens0) + n_app
+    cap = Tmax + 8
+    K = torch.zeros((B, Hkv, Tmax, D), dtype=w.kv_dtype, device=dev)
+    V = torch.zeros_like(K)
+    for b in range(B):
+        k, v = S.gen_kv_one(w, b, lens0[b] + n_app, device=dev)
+        K[b, :, :lens0[b] + n_app] = k
+        V[b, :, :lens0[b] + n_app] = v
+        del k, v
+    T0 = max(lens0)
+    Kp, Vp = K[:, :, :T0].contiguous(), V[:, :, :T0].contiguous()
+    apps_k = [torch.stack([K[b, :, lens0[b] + i:lens0[b] + i + 1] for b in range(B)]).contiguous()
+              for i in range(n_app)]
+    apps_v = [torch.stack([V[b, :, lens0[b] + i:lens0[b] + i + 1] for b in range(B)]).contiguous()
+              for i in range(n_app)]
+    del K, V
+    sl = torch.tensor(lens0, dtype=torch.int32, device=dev)
+    in_elem = torch.finfo(w.kv_dtype).bits // 8
+    st = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    lens = [L + n_app for L in lens0]
+    nbytes = kv_bytes("delta", lens, Hkv, w.kf)
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_copies = max(1, math.ceil(4 * l2_bytes / nbytes))
+    caches = [dkv.Cache(B, Hkv, cap, "delta", kf=w.kf, device=dev) for _ in range(n_copies)]
+    res = {"batch": B, "q_heads": Hq, "kv_heads": Hkv, "kf": w.kf, "generator": w.gen,
+           "context": lens if B <= 4 else lens[0], "kv_bytes": nbytes}
+    e0, e1 = ev(), ev()
+    e0.record(st)
+    caches[0].encode(Kp, Vp, seq_lens=sl)
+    e1.record(st)
+    torch.cuda.synchronize()
+    t_enc = e0.elapsed_time(e1)
+    res["encode_ms"] = t_enc
+    res["encode_gbps"] = encode_bytes("delta", lens0, Hkv, w.kf, in_elem) / (t_enc * 1e-3) / 1e9
+    for c in caches[1:]:
+        c.encode(Kp, Vp, seq_lens=sl)
+    if n_app:
+        ts = []
+        for i in range(n_app):
+            a0, a1 = ev(), ev()
+            a0.record(st)
+            for c in caches:
+                c.append(apps_k[i], apps_v[i])
+            a1.record(st)
+            ts.append((a0, a1))
+        torch.cuda.synchronize()
+        per_call = sum(a.elapsed_time(b) for a, b in ts) / (n_app * len(caches))
+        res["append_us_per_call"] = 1e3 * per_call
+        res["append_gbps"] = append_bytes("delta", lens0, 1, Hkv, w.kf, in_elem) / (per_call * 1e-3) / 1e9
+    q = S.gen_q(w, device=dev)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    qcode = dkv._dtype_code(w.q_dtype)
+    scale = 1.0 / math.sqrt(D)
+    wss = [c.workspace(Hq) for c in caches]
+    for i in range(3):
+        c = caches[i % n_copies]
+        c.decode_attn(q, scale, out=out)
+    torch.cuda.synchronize()
+    sp, mg = [], []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.synchronize()
+        for i in range(max(n_iter, n_copies)):
+            c, ws = caches[i % n_copies], wss[i % n_copies]
+            x0, x1, x2 = ev(), ev(), ev()
+            x0.record(st)
+            dkv.dkv_decode_attn_split(c.c, q, qcode, Hq, scale, ws, ws.numel() * 4, st)
+            x1.record(st)
+            dkv.dkv_decode_attn_merge(c.c, Hq, out, ws, ws.numel() * 4, st)
+            x2.record(st)
+            sp.append((x0, x1))
+            mg.append((x1, x2))
+        torch.cuda.synchronize()
+    status = caches[0].device_status()
+    t_split = statistics.median(a.elapsed_time(b) for a, b in sp)
+    t_merge = statistics.median(a.elapsed_time(b) for a, b in mg)
+    gbps = nbytes / (t_split * 1e-3) / 1e9
+    res.update({"split_us": 1e3 * t_split, "merge_us": 1e3 * t_merge, "gbps": gbps,
+                "pct_of_peak": 100.0 * gbps / peak, "pct_of_nominal_8TBs": 100.0 * gbps / NOMINAL_HBM_GBS,
+                "step_gbps": nbytes / ((t_split + t_merge) * 1e-3) / 1e9,
+                "kv_token_heads_per_s": sum(lens) * Hkv / (t_split * 1e-3),
+                "l2": f"rotated over {n_copies} identical caches (cache < 4x L2)",
+                "clocks": clk.summary(), "device_status": status})
+    if n_copies == 1:
+        res["l2"] = "no flush: the compressed cache read per decode exceeds the 126 MB L2"
+    del caches, wss
+    torch.cuda.empty_cache()
+    return res
+
+
+def config_sweep(dev, peak, n_iter=10):
+    import synthetic as S
+    out = {}
+    for label, name, ov in CONFIG_CASES:
+        w = S.WORKLOADS[name].with_(**ov)
+        try:
+            out[label] = time_config(dev, w, peak, n_iter=n_iter)
+        except Exception as e:          # a reported extra: never costs the bench line
+            out[label] = {"error": repr(e)[:300]}
+    return out
+
+
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
@@ -730,6 +919,8 @@ def run_ours(args, w, rank, world, local):
         res["mse"] = mse
     torch.cuda.synchronize()
 
+    if rank == 0 and args.configs:
+        res["configs"] = config_sweep(dev, measured_peak()[0])
     if rank == 0 and args.comparators:
         res["quality"] = quality_report(dev)
 
@@ -740,6 +931,10 @@ def run_ours(args, w, rank, world, local):
             T_ = K.shape[1]
             return xh[:, 0, :T_], xh[:, 1, :T_]
 
+        try:
+            res["lr_decode"] = lr_decode_bench(dev)
+        except Exception as e:          # a reported extra: never costs the bench line
+            res["lr_decode"] = {"error": repr(e)[:200]}
         try:
             res["quality"]["long_range_refs"] = lr_quality(
                 dev, lambda X, s, m: dkv.lr_encode(X, s, m)["xhat"], _recon)
@@ -801,6 +996,10 @@ def run_ours(args, w, rank, world, local):
         line["comparators"] = extra
     if "mse" in res:
         line["mse"] = res["mse"]
+    if "configs" in res:
+        line["configs"] = res["configs"]
+    if "lr_decode" in res:
+        line["lr_decode"] = res["lr_decode"]
     if "quality" in res:
         line["quality"] = res["quality"]
     print(json.dumps(line), flush=True)
@@ -819,6 +1018,8 @@ def main(argv=None):
     ap.add_argument("--context", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-comparators", dest="comparators", action="store_false")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip timing the other workload configurations")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)

@@ -37,6 +37,11 @@ class dkv_cache_desc(ctypes.Structure):
                 ("max_ctx", ctypes.c_int32), ("fmt", ctypes.c_int32)]
 
 
+class dkv_lr_tensor(ctypes.Structure):
+    _fields_ = [("ref", ctypes.c_void_p), ("ref_values", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("codes", ctypes.c_void_p)]
+
+
 class dkv_cache(ctypes.Structure):
     _fields_ = [("desc", dkv_cache_desc), ("base", ctypes.c_void_p), ("bytes", ctypes.c_size_t),
                 ("seq_stride", ctypes.c_size_t), ("rec_bytes", ctypes.c_size_t),
@@ -56,7 +61,8 @@ EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode",
            "dkv_debug_set_fault", "dkv_cache_meta_bytes", "dkv_page_bytes",
            "dkv_cache_init_paged", "dkv_decode_workspace_bytes_mq", "dkv_decode_attn_mq",
            "dkv_append_decode_attn", "dkv_append_decode_attn_split",
-           "dkv_append_decode_attn_merge", "dkv_lr_encode"]
+           "dkv_append_decode_attn_merge", "dkv_lr_encode", "dkv_lr_decode_workspace_bytes",
+           "dkv_lr_decode_attn"]
 
 
 def load():
@@ -96,6 +102,9 @@ def load():
         "dkv_append_decode_attn_split": ([PC, P, P, I, I, P, I, I, F, P, S, P], I),
         "dkv_append_decode_attn_merge": ([PC, I, I, P, P, S, P], I),
         "dkv_lr_encode": ([P, I, I, I, I, I, P, P, P, P, P, P], I),
+        "dkv_lr_decode_workspace_bytes": ([I, I, I, I], S),
+        "dkv_lr_decode_attn": ([ctypes.POINTER(dkv_lr_tensor), ctypes.POINTER(dkv_lr_tensor),
+                                I, I, I, I, I, P, P, I, I, F, P, P, S, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -257,6 +266,41 @@ def lr_encode(X, stride: int, n_refs: int, stream=None) -> dict:
                                 _ptr(out["ref"]), _ptr(out["ref_values"]), _ptr(out["scales"]),
                                 _ptr(out["codes"]), _ptr(out["xhat"]), _stream(stream)),
            "dkv_lr_encode")
+    return out
+
+
+def dkv_lr_decode_workspace_bytes(batch: int, n_kv_heads: int, T: int, stride: int) -> int:
+    return load().dkv_lr_decode_workspace_bytes(batch, n_kv_heads, T, stride)
+
+
+def _lr_view(enc) -> dkv_lr_tensor:
+    return dkv_lr_tensor(_ptr(enc["ref"]), _ptr(enc["ref_values"]), _ptr(enc["scales"]),
+                         _ptr(enc["codes"]))
+
+
+def lr_decode_attn(enc_k: dict, enc_v: dict, Q, softmax_scale: float, stride: int,
+                   n_kv_heads: int, lens=None, out=None, workspace=None, stream=None):
+    """Decode attention over long-range reference encodings (dkv_lr_decode_attn).
+    enc_k, enc_v: the dicts `lr_encode` returns for K and V, each encoding
+    [B * n_kv_heads, T, 128] sequences (sequence = batch entry * n_kv_heads +
+    kv head) with the same stride and n_refs; Q [B, n_q_heads, 128];
+    lens: device int32 [B] or None.  Returns fp32 [B, n_q_heads, 128]."""
+    import torch
+    n_seq, T, n_refs = enc_k["ref"].shape
+    B = n_seq // n_kv_heads
+    Hq = Q.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, 128), dtype=torch.float32, device=Q.device)
+    nb = dkv_lr_decode_workspace_bytes(B, n_kv_heads, T, stride)
+    if workspace is None:
+        workspace = torch.empty(nb // 4 + 64, dtype=torch.float32, device=Q.device)
+    kv, vv = _lr_view(enc_k), _lr_view(enc_v)
+    Q = Q.contiguous()
+    _check(load().dkv_lr_decode_attn(ctypes.byref(kv), ctypes.byref(vv), B, n_kv_heads, T, stride,
+                                     n_refs, _ptr(lens), _ptr(Q), _dtype_code(Q.dtype), Hq,
+                                     softmax_scale, _ptr(out), _ptr(workspace),
+                                     workspace.numel() * 4, _stream(stream)),
+           "dkv_lr_decode_attn")
     return out
 
 

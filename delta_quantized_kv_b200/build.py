@@ -13,7 +13,7 @@ from pathlib import Path
 PKG = Path(__file__).resolve().parent
 CSRC = PKG / "csrc"
 OUT = PKG / "_lib" / "libdkv.so"
-SOURCES = ["dkv_api.cu", "encode.cu", "decode.cu", "noalloc.cu", "lr_encode.cu"]
+SOURCES = ["dkv_api.cu", "encode.cu", "decode.cu", "noalloc.cu", "lr_encode.cu", "lr_decode.cu"]
 HEADERS = ["dkv_common.cuh", "dkv_internal.h"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared"]
@@ -35,13 +35,33 @@ def stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> Path:
+    """Compile every translation unit in parallel (one nvcc per file), then
+    link the shared library; the result replaces the old one atomically."""
     if not force and not stale():
         return OUT
+    from concurrent.futures import ThreadPoolExecutor
+    import tempfile
     OUT.parent.mkdir(parents=True, exist_ok=True)
-    tmp = OUT.with_name(f"libdkv.{os.getpid()}.tmp.so")
-    cmd = [_nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", str(tmp),
-           *[str(CSRC / s) for s in SOURCES]]
-    subprocess.run(cmd, check=True)
+    nvcc = _nvcc()
+    cflags = [f for f in NVCC_FLAGS if f != "-shared"]
+    with tempfile.TemporaryDirectory(prefix="dkv_build_") as tmpd:
+        objs = [Path(tmpd) / (Path(s).stem + ".o") for s in SOURCES]
+
+        def compile_one(i):
+            cmd = [nvcc, *cflags, *(["-Xptxas", "-v"] if verbose else []), "-c",
+                   str(CSRC / SOURCES[i]), "-o", str(objs[i])]
+            return subprocess.run(cmd, capture_output=True, text=True)
+
+        with ThreadPoolExecutor(max_workers=min(len(SOURCES), os.cpu_count() or 1)) as ex:
+            results = list(ex.map(compile_one, range(len(SOURCES))))
+        for r in results:
+            if verbose or r.returncode:
+                print(r.stdout + r.stderr)
+            if r.returncode:
+                raise subprocess.CalledProcessError(r.returncode, r.args, r.stdout, r.stderr)
+        tmp = OUT.with_name(f"libdkv.{os.getpid()}.tmp.so")
+        subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+                        "-o", str(tmp), *[str(o) for o in objs]], check=True)
     os.replace(tmp, OUT)
     return OUT
 

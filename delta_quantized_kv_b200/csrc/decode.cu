@@ -410,11 +410,6 @@ __device__ inline StageMeta next_stage(const CacheView &cv, Cursor &c, int nvs, 
     return m;
 }
 
-__device__ inline uint32_t pack_h2(float lo, float hi) {
-    return h2_as_u32(__floats2half2_rn(lo, hi));
-}
-__device__ inline float h_lo(uint32_t u) { return __low2float(u32_as_h2(u)); }
-__device__ inline float h_hi(uint32_t u) { return __high2float(u32_as_h2(u)); }
 
 __device__ inline float q_elem(const void *Q, int dt, int64_t i) {
     if (dt == DKV_F32) return static_cast<const float *>(Q)[i];
@@ -422,11 +417,6 @@ __device__ inline float q_elem(const void *Q, int dt, int64_t i) {
     return __bfloat162float(static_cast<const __nv_bfloat16 *>(Q)[i]);
 }
 
-__device__ inline uint32_t movm_t(uint32_t a) {
-    uint32_t d;
-    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
-    return d;
-}
 __device__ inline float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
@@ -811,16 +801,20 @@ __device__ __noinline__ void append_tokens(const SplitArgs &A, int b, int kvh, i
         } else {
             // the eight blocks (K and V, 4 each) are independent chains
             uint32_t codes = 0;         // code of channel 32 j + lane of tensor t at bit 16 t + 4 j
+            float dl[8];
+            int cd[8];
+            __half h16[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dl[i] = __fsub_rn(x[i >> 2][i & 3], xh[i >> 2][i & 3]);
+            quant_lanes<8>(dl, cd, h16);
             __half d16[2][4];
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int code = quant_lane(__fsub_rn(x[t][j], xh[t][j]), &d16[t][j]);
-                    codes |= (uint32_t)code << (16 * t + 4 * j);
-                    xh[t][j] = __fadd_rn(xh[t][j],
-                                         __fmul_rn((float)(code - 8), __half2float(d16[t][j])));
-                }
+            for (int i = 0; i < 8; ++i) {
+                const int t = i >> 2, j = i & 3;
+                d16[t][j] = h16[i];
+                codes |= (uint32_t)cd[i] << (16 * t + 4 * j);
+                xh[t][j] = __fadd_rn(xh[t][j], __fmul_rn((float)(cd[i] - 8), __half2float(h16[i])));
+            }
             if (rec) {
                 // gather the 8 codes of this lane's word from the lanes holding them
                 uint32_t word = 0;

@@ -3,6 +3,7 @@
 // on the caller's stream.
 #include <cstdint>
 #include <cstring>
+#include <initializer_list>
 
 #include "../../include/dkv.h"
 #include "dkv_common.cuh"
@@ -394,6 +395,44 @@ dkv_status dkv_lr_encode(const void *X, int32_t dtype, int32_t n_seq, int32_t T,
         return DKV_EALIGN;
     return cuda_status(dkv::launch_lr_encode(X, dtype, n_seq, T, stride, n_refs, ref, ref_values,
                                              scales, codes, xhat,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+size_t dkv_lr_decode_workspace_bytes(int32_t batch, int32_t n_kv_heads, int32_t T,
+                                     int32_t stride) {
+    if (batch < 1 || n_kv_heads < 1 || T < 1 || stride < 1) return 0;
+    if ((int64_t)batch * n_kv_heads * T > ((int64_t)1 << 31)) return 0;
+    return dkv::lrd_workspace_floats(batch, n_kv_heads, T, stride) * sizeof(float);
+}
+
+dkv_status dkv_lr_decode_attn(const dkv_lr_tensor *K, const dkv_lr_tensor *V, int32_t batch,
+                              int32_t n_kv_heads, int32_t T, int32_t stride, int32_t n_refs,
+                              const int32_t *lens_dev, const void *Q, int32_t q_dtype,
+                              int32_t n_q_heads, float softmax_scale, float *out,
+                              void *workspace, size_t ws_bytes, void *stream) {
+    if (!K || !V || !Q || !out || !workspace || !valid_dtype(q_dtype)) return DKV_EINVAL;
+    for (const dkv_lr_tensor *t : {K, V}) {
+        if (!t->ref || !t->ref_values || !t->scales || !t->codes) return DKV_EINVAL;
+        if (!aligned16(t->ref) || !aligned16(t->ref_values) || !aligned16(t->scales) ||
+            !aligned16(t->codes))
+            return DKV_EALIGN;
+    }
+    if (batch < 1 || batch > 65535 || n_kv_heads < 1 || T < 1 || stride < 1 || n_refs < 1 ||
+        n_refs > 8 || n_q_heads < 1 || n_q_heads % n_kv_heads != 0)
+        return DKV_EINVAL;
+    if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return DKV_EINVAL;
+    if (n_q_heads / n_kv_heads > 8) return DKV_EUNSUPPORTED;
+    if (!aligned16(Q) || !aligned16(out) || !aligned16(workspace) ||
+        (lens_dev && (reinterpret_cast<uintptr_t>(lens_dev) & 3)))
+        return DKV_EALIGN;
+    const size_t need = dkv_lr_decode_workspace_bytes(batch, n_kv_heads, T, stride);
+    if (need == 0) return DKV_ECAPACITY;
+    if (ws_bytes < need) return DKV_ECAPACITY;
+    const dkv::LrdView kv{K->ref, K->ref_values, K->scales, K->codes};
+    const dkv::LrdView vv{V->ref, V->ref_values, V->scales, V->codes};
+    return cuda_status(dkv::launch_lr_decode(kv, vv, batch, n_kv_heads, T, stride, n_refs,
+                                             lens_dev, Q, q_dtype, n_q_heads, softmax_scale, out,
+                                             static_cast<float *>(workspace),
                                              static_cast<cudaStream_t>(stream)));
 }
 

@@ -191,6 +191,19 @@ __device__ inline uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
 __device__ inline uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ inline __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 
+__device__ inline uint32_t pack_h2(float lo, float hi) {
+    return h2_as_u32(__floats2half2_rn(lo, hi));
+}
+__device__ inline float h_lo(uint32_t u) { return __low2float(u32_as_h2(u)); }
+__device__ inline float h_hi(uint32_t u) { return __high2float(u32_as_h2(u)); }
+// 8x8 transpose of b16 elements across the warp (thread t holds row t / 4,
+// columns 2 (t % 4) and 2 (t % 4) + 1).
+__device__ inline uint32_t movm_t(uint32_t a) {
+    uint32_t d;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+    return d;
+}
+
 // D = A(16x16 f16, row) * B(16x8 f16, col) + C, fp32 accumulate.
 __device__ inline void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                 uint32_t b0, uint32_t b1) {
@@ -199,6 +212,19 @@ __device__ inline void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_
         "{%8,%9}, {%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ldmatrix: four 8x8 b16 tiles from shared memory (lane l gives the address
+// of row l % 8 of tile l / 8); .trans delivers each tile transposed.
+__device__ inline void ldsm_x4(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+__device__ inline void ldsm_x4_t(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
 }
 
 // The fp16 bit pattern of 1024.0 in both halves, as a register value the
@@ -303,6 +329,38 @@ __device__ inline int quant_lane(float v, __half *d16_out) {
     float u = __fadd_rn(q, 8.5f);
     int c = (int)truncf(u);
     return min(15, max(0, c));
+}
+
+// The block rule on NC independent blocks at once (element lane of each),
+// written phase by phase -- every block's reduction, then every block's
+// vote, ... -- so the warp-wide steps of the blocks overlap instead of
+// running one block after another.  Each block takes exactly the steps of
+// quant_lane, in the same order.  A zero scale divides by 1 (the code is
+// then 8 regardless), so no division ever sees a zero divisor.
+template <int NC>
+__device__ inline void quant_lanes(const float (&v)[NC], int (&code)[NC], __half (&d16)[NC]) {
+    uint32_t a[NC], mx[NC], ball[NC];
+    float m[NC], d[NC];
+#pragma unroll
+    for (int i = 0; i < NC; ++i) a[i] = __float_as_uint(v[i]) & 0x7fffffffu;
+#pragma unroll
+    for (int i = 0; i < NC; ++i) mx[i] = __reduce_max_sync(0xffffffffu, a[i]);
+#pragma unroll
+    for (int i = 0; i < NC; ++i) ball[i] = __ballot_sync(0xffffffffu, a[i] == mx[i]);
+#pragma unroll
+    for (int i = 0; i < NC; ++i) m[i] = __shfl_sync(0xffffffffu, v[i], __ffs(ball[i]) - 1);
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+        d16[i] = __float2half_rn(__fmul_rn(m[i], -0.125f));
+        d[i] = __half2float(d16[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+        const bool z = d[i] == 0.0f;
+        const float q = __fdiv_rn(v[i], z ? 1.0f : d[i]);
+        const int c = (int)truncf(__fadd_rn(q, 8.5f));
+        code[i] = z ? 8 : min(15, max(0, c));
+    }
 }
 
 }  // namespace dkv

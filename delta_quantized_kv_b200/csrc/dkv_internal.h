@@ -48,4 +48,17 @@ cudaError_t launch_lr_encode(const void *X, int dtype, int n_seq, int T, int s, 
                              int32_t *ref, uint16_t *kfr, uint16_t *scales, uint8_t *codes,
                              float *xhat, cudaStream_t st);
 
+// Decode over the long-range reference encoding (canonical layouts of
+// dkv_lr_encode, one view per tensor); ws holds lrd_workspace_floats floats.
+struct LrdView {
+    const int32_t *ref;
+    const uint16_t *ref_values;
+    const uint16_t *scales;
+    const uint8_t *codes;
+};
+size_t lrd_workspace_floats(int B, int Hkv, int T, int s);
+cudaError_t launch_lr_decode(const LrdView &K, const LrdView &V, int B, int Hkv, int T, int s,
+                             int m, const int32_t *lens, const void *Q, int q_dtype, int Hq,
+                             float softmax_scale, float *out, float *ws, cudaStream_t st);
+
 }  // namespace dkv

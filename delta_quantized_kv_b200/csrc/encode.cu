@@ -215,6 +215,184 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Delta format.  One warp per (batch entry, kv head, keyframe group) of the
+// range being written.  The warp carries the group's eight closed loops side
+// by side -- K and V, four 32-channel blocks each, lane = channel within its
+// block -- so every step of the sequential loop has eight independent
+// quantiser chains in flight; the next position's inputs are loaded while the
+// current one is quantised.  The nibble words are gathered in the permuted
+// layout with warp shuffles (lanes 0-15 write the K words of a position,
+// lanes 16-31 the V words) and the scales by lanes 0 and 1.  The quantiser is
+// quant_lane, in the same order of steps as the encode of every other path.
+// ---------------------------------------------------------------------------
+constexpr int ENC_WARPS = 4;
+
+// Input element (tensor t, channel 32 j + lane) of relative position r.
+__device__ inline float enc_in(const EncodeArgs &a, int t, int64_t base, int r, int j, int lane) {
+    return load_in(t ? a.V : a.K, a.dtype, base + (int64_t)r * D + 32 * j + lane);
+}
+
+#ifndef DKV_ENC_MINB
+#define DKV_ENC_MINB 1
+#endif
+__global__ void __launch_bounds__(ENC_WARPS * 32, DKV_ENC_MINB) encode_delta_kernel(EncodeArgs a, int NG) {
+    const CacheView &cv = a.cv;
+    const int lane = threadIdx.x & 31;
+    const int64_t item = (int64_t)blockIdx.x * ENC_WARPS + (threadIdx.x >> 5);
+    const int kf = cv.kf;
+    if (item < (int64_t)cv.B * cv.Hkv * NG) {
+        const int gi = (int)(item % NG);
+        const int bh = (int)(item / NG);
+        const int b = bh / cv.Hkv, kvh = bh % cv.Hkv;
+        int start, n;
+        encode_range(a, b, start, n);
+        const int parity = cv.header[2] & 1;
+        const int64_t slot = (int64_t)cv.B * cv.Hkv * 2 * D;
+        const int64_t sb = ((int64_t)b * cv.Hkv + kvh) * 2 * D;
+        const float *st_old = cv.state + parity * slot + sb;
+        float *st_new = cv.state + (parity ^ 1) * slot + sb;
+        if (n < 0 && gi == 0 && kvh == 0 && lane == 0)
+            set_status(cv.header, n == -2 ? DKV_DEV_CAPACITY : DKV_DEV_BAD_SEQLEN);
+        if (n <= 0) {
+            if (gi == 0) {                    // nothing written: carry the state over
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int c = t * D + 32 * j + lane;
+                        st_new[c] = a.append ? st_old[c] : 0.0f;
+                    }
+            }
+        } else {
+            const int g = start / kf + gi;
+            const int p0 = max(start, g * kf), p1 = min(start + n, (g + 1) * kf);
+            const bool last = p1 == start + n;
+            uint8_t *rec = p0 < p1 ? rec_ptr(cv, b, kvh, g) : nullptr;
+            if (p0 < p1 && !rec) {
+                // bad block-table entry (flagged by rec_ptr): nothing written
+                if (last) {
+#pragma unroll
+                    for (int t = 0; t < 2; ++t)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int c = t * D + 32 * j + lane;
+                            st_new[c] = (p0 % kf) ? st_old[c] : 0.0f;
+                        }
+                }
+            } else if (p0 < p1) {
+                const int64_t base = ((int64_t)b * cv.Hkv + kvh) * a.T_in * D;
+                float xh[2][4], x[2][4];
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        xh[t][j] = (p0 % kf) ? st_old[t * D + 32 * j + lane] : 0.0f;
+                        x[t][j] = enc_in(a, t, base, p0 - start, j, lane);
+                    }
+                const int wt = lane >> 4, ww = lane & 15;   // this lane's nibble word
+                uint8_t *nib0 = rec + KF_BYTES + (int64_t)(kf - 1) * SC_BYTES +
+                                (int64_t)wt * (kf - 1) * NIB_BYTES + 4 * ww;
+#pragma unroll 1
+                for (int p = p0; p < p1; ++p) {
+                    float xn[2][4];
+                    if (p + 1 < p1) {
+#pragma unroll
+                        for (int t = 0; t < 2; ++t)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                xn[t][j] = enc_in(a, t, base, p + 1 - start, j, lane);
+                    }
+                    const int di = p - g * kf;      // 0: keyframe; else delta di - 1
+                    if (di == 0) {
+#pragma unroll
+                        for (int t = 0; t < 2; ++t)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const __half h = __float2half_rn(x[t][j]);
+                                xh[t][j] = __half2float(h);
+                                const int ch = 32 * j + lane;
+                                reinterpret_cast<__half *>(rec + t * 256)[t == 0 ? k_half_idx(ch)
+                                                                                 : v_half_idx(ch)] = h;
+                            }
+                    } else {
+                        uint32_t codes = 0;         // code of (t, j) at bit 16 t + 4 j
+                        float dl[8];
+                        int cd[8];
+                        __half h16[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) dl[i] = __fsub_rn(x[i >> 2][i & 3], xh[i >> 2][i & 3]);
+                        quant_lanes<8>(dl, cd, h16);
+                        __half d16[2][4];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int t = i >> 2, j = i & 3;
+                            d16[t][j] = h16[i];
+                            codes |= (uint32_t)cd[i] << (16 * t + 4 * j);
+                            xh[t][j] = __fadd_rn(xh[t][j], __fmul_rn((float)(cd[i] - 8),
+                                                                     __half2float(h16[i])));
+                        }
+                        uint32_t word = 0;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const int ch = nib_channel(wt, ww, k);
+                            const uint32_t v = __shfl_sync(0xffffffffu, codes, ch & 31);
+                            word |= ((v >> (16 * wt + 4 * (ch >> 5))) & 15u) << (4 * k);
+                        }
+                        *reinterpret_cast<uint32_t *>(nib0 + (int64_t)(di - 1) * NIB_BYTES) = word;
+                        if (lane < 2) {
+                            uint32_t h[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                h[j] = __half_as_ushort(lane ? d16[1][j] : d16[0][j]);
+                            *reinterpret_cast<uint2 *>(rec + KF_BYTES + (int64_t)(di - 1) * SC_BYTES +
+                                                       lane * 8) =
+                                make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+                        }
+                    }
+                    if (p + 1 < p1) {
+#pragma unroll
+                        for (int t = 0; t < 2; ++t)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) x[t][j] = xn[t][j];
+                    }
+                }
+                if (last) {
+#pragma unroll
+                    for (int t = 0; t < 2; ++t)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) st_new[t * D + 32 * j + lane] = xh[t][j];
+                }
+            }
+        }
+    }
+
+    // The last block to finish publishes the new lengths and flips the state
+    // slot; every block has read seq_len and the old state before it arrives.
+    __shared__ int last_blk;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(reinterpret_cast<unsigned *>(cv.header + 1), 1u);
+        last_blk = prev == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (last_blk) {
+        __threadfence();
+        for (int bb = threadIdx.x; bb < cv.B; bb += blockDim.x) {
+            int s0, nn;
+            encode_range(a, bb, s0, nn);
+            if (nn >= 0) cv.seqlen[bb] = s0 + nn;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            cv.header[2] ^= 1;
+            cv.header[1] = 0;
+            __threadfence();
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Read-back kernels.  Grid: x = position chunk of 32, y = kvh*2 + t, z = b.
 // ---------------------------------------------------------------------------
 struct ExportArgs {
@@ -303,6 +481,15 @@ __global__ void __launch_bounds__(128) readback_kernel(ExportArgs a) {
 cudaError_t launch_encode(const CacheView &cv, const void *K, const void *V, int dtype,
                           const int32_t *seq_lens, int T_in, int append, cudaStream_t st) {
     EncodeArgs a{cv, K, V, dtype, seq_lens, T_in, append};
+    if (cv.fmt == DKV_FMT_DELTA) {
+        // groups a batch entry's range can touch (an append may start mid-group)
+        const int NG = (T_in + cv.kf - 1) / cv.kf + (append ? 1 : 0);
+        const int64_t warps = (int64_t)cv.B * cv.Hkv * NG;
+        const int64_t ctas = (warps + ENC_WARPS - 1) / ENC_WARPS;
+        if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
+        encode_delta_kernel<<<(unsigned)ctas, ENC_WARPS * 32, 0, st>>>(a, NG);
+        return cudaGetLastError();
+    }
     int items;
     if (cv.fmt == DKV_FMT_DELTA)
         items = append ? (T_in + cv.kf - 1) / cv.kf + 1 : (T_in + cv.kf - 1) / cv.kf;

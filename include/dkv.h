@@ -265,11 +265,50 @@ dkv_status dkv_append_decode_attn_merge(dkv_cache *cache, int32_t n_new, int32_t
  *   scales     uint16 [n_seq][T][4]         fp16 bits (0 on reference rows)
  *   codes      uint8  [n_seq][T][128]       0..15 (0 on reference rows)
  *   xhat       float  [n_seq][T][128]       reconstruction (NULL: not written)
- * 1 <= n_refs <= 8, stride >= 1.  Encoding only: there is no decode over this
- * format yet. */
+ * 1 <= n_refs <= 8, stride >= 1.  dkv_lr_decode_attn attends over these
+ * outputs. */
 dkv_status dkv_lr_encode(const void *X, int32_t dtype, int32_t n_seq, int32_t T, int32_t stride,
                          int32_t n_refs, int32_t *ref, uint16_t *ref_values, uint16_t *scales,
                          uint8_t *codes, float *xhat, void *stream);
+
+/* One tensor (K or V) of a long-range reference encoding, in the canonical
+ * layouts dkv_lr_encode writes (device arrays, 16-byte aligned, caller-owned);
+ * sequence index = batch entry * n_kv_heads + kv head. */
+typedef struct {
+    const int32_t *ref;          /* [n_seq][T][n_refs] */
+    const uint16_t *ref_values;  /* [n_seq][ceil(T/stride)][128] */
+    const uint16_t *scales;      /* [n_seq][T][4] */
+    const uint8_t *codes;        /* [n_seq][T][128] */
+} dkv_lr_tensor;
+
+/* Decode attention over the long-range reference encoding (page "DeltaKV"
+ * summary, section A, "Reconstruction": the residual plus the mean of the
+ * chosen references; the decode step of page "KV 캐시 벡터 양자화와 주의 보존
+ * 변환", section "KV 캐시가 왜 병목인가").  For batch entry b and query head h
+ * (kv head h / (n_q_heads / n_kv_heads)): out[b][h] = softmax over p < len_b
+ * of softmax_scale * q . k^_p, applied to v^_p, where x^ is the encoding's
+ * reconstruction (a reference token: its fp16 value; any other token: the
+ * mean of its references plus its dequantised residual).  The reconstruction
+ * is never formed: the scores are the mean of the references' dot products
+ * plus q . residual, and the output is sum_r W_r v^_r plus the residuals
+ * weighted by the softmax (W_r: the weight each reference receives from the
+ * tokens that use it).  K and V are encoded separately (each with its own
+ * choices), with the same T, stride and n_refs.
+ * lens_dev: device int32[batch], 0 <= len_b <= T (NULL: every len_b = T); a
+ * sequence of length 0 gives zeros.  Q: [batch][n_q_heads][128] of q_dtype
+ * (fp32 queries are split into an fp16 hi + lo pair); out: the same shape,
+ * fp32.  n_q_heads / n_kv_heads must be 1..8 (DKV_EUNSUPPORTED otherwise);
+ * softmax_scale finite and > 0.  workspace: >= dkv_lr_decode_workspace_bytes.
+ * Three launches on `stream`: the references' dot products, one warp per
+ * 256-token chunk (scores, softmax, residual part), one block per sequence
+ * (combine and reference part). */
+size_t dkv_lr_decode_workspace_bytes(int32_t batch, int32_t n_kv_heads, int32_t T,
+                                     int32_t stride);
+dkv_status dkv_lr_decode_attn(const dkv_lr_tensor *K, const dkv_lr_tensor *V, int32_t batch,
+                              int32_t n_kv_heads, int32_t T, int32_t stride, int32_t n_refs,
+                              const int32_t *lens_dev, const void *Q, int32_t q_dtype,
+                              int32_t n_q_heads, float softmax_scale, float *out,
+                              void *workspace, size_t ws_bytes, void *stream);
 
 /* Size of the library-owned scratch array used by dkv_decode_attn_noalloc. */
 #define DKV_NOALLOC_SCRATCH_BYTES (16u << 20)

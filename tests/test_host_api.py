@@ -135,6 +135,30 @@ def test_noalloc_gives_invalid_caches_the_statuses_of_dkv_decode_attn(dkv):
                                        None) == dkv.DKV_EINVAL
 
 
+def test_lr_decode_rejects_bad_arguments_on_host(dkv):
+    """dkv_lr_decode_attn validates everything before any launch."""
+    lib = dkv.load()
+    A = 1 << 12
+    t = dkv.dkv_lr_tensor(A, A, A, A)
+    bad = dkv.dkv_lr_tensor(A, A + 2, A, A)
+    nb = dkv.dkv_lr_decode_workspace_bytes(2, 2, 100, 8)
+    assert nb > 0 and dkv.dkv_lr_decode_workspace_bytes(0, 2, 100, 8) == 0
+    call = lambda K=t, V=t, B=2, H=2, T=100, s=8, m=2, q=A, qd=1, hq=8, sc=0.1, o=A, ws=A, wsb=nb: \
+        lib.dkv_lr_decode_attn(ctypes.byref(K), ctypes.byref(V), B, H, T, s, m, None, q, qd, hq,
+                               sc, o, ws, wsb, None)
+    assert call(K=dkv.dkv_lr_tensor(0, A, A, A)) == dkv.DKV_EINVAL
+    assert call(V=bad) == dkv.DKV_EALIGN
+    assert call(m=0) == dkv.DKV_EINVAL and call(m=9) == dkv.DKV_EINVAL
+    assert call(s=0) == dkv.DKV_EINVAL and call(T=0) == dkv.DKV_EINVAL
+    assert call(hq=3) == dkv.DKV_EINVAL
+    assert call(hq=18) == dkv.DKV_EUNSUPPORTED            # 9 query heads per kv head
+    assert call(sc=0.0) == dkv.DKV_EINVAL and call(qd=7) == dkv.DKV_EINVAL
+    assert call(q=A + 4) == dkv.DKV_EALIGN
+    assert call(wsb=nb - 4) == dkv.DKV_ECAPACITY
+    assert lib.dkv_lr_decode_attn(None, ctypes.byref(t), 2, 2, 100, 8, 2, None, A, 1, 8, 0.1,
+                                  A, A, nb, None) == dkv.DKV_EINVAL
+
+
 def test_bad_dtype_and_sizes_rejected_on_host(dkv):
     """A well-formed view whose arguments are wrong: nothing is launched."""
     lib = dkv.load()
