@@ -62,7 +62,7 @@ EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode",
            "dkv_cache_init_paged", "dkv_decode_workspace_bytes_mq", "dkv_decode_attn_mq",
            "dkv_append_decode_attn", "dkv_append_decode_attn_split",
            "dkv_append_decode_attn_merge", "dkv_lr_encode", "dkv_lr_decode_workspace_bytes",
-           "dkv_lr_decode_attn"]
+           "dkv_lr_decode_attn", "dkv_debug_division_check"]
 
 
 def load():
@@ -103,6 +103,7 @@ def load():
         "dkv_append_decode_attn_merge": ([PC, I, I, P, P, S, P], I),
         "dkv_lr_encode": ([P, I, I, I, I, I, P, P, P, P, P, P], I),
         "dkv_lr_decode_workspace_bytes": ([I, I, I, I], S),
+        "dkv_debug_division_check": ([P, I, P, P], I),
         "dkv_lr_decode_attn": ([ctypes.POINTER(dkv_lr_tensor), ctypes.POINTER(dkv_lr_tensor),
                                 I, I, I, I, I, P, P, I, I, F, P, P, S, P], I),
     }
@@ -344,6 +345,14 @@ def dkv_dequantize(cache: dkv_cache, out, stream=None) -> None:
 def dkv_debug_set_fault(mode: int) -> None:
     """Test support: mode 1 makes later split launches time out by design."""
     load().dkv_debug_set_fault(int(mode))
+
+
+def dkv_debug_division_check(u, mismatches, stream=None) -> None:
+    """Test support: count (into the device uint64 `mismatches`) the encoder
+    quotients that differ from IEEE division, over every fp16 divisor and the
+    dividends RN(u_i b) and their neighbours (u: device fp32)."""
+    _check(load().dkv_debug_division_check(_ptr(u), u.numel(), _ptr(mismatches),
+                                           _stream(stream)), "dkv_debug_division_check")
 
 
 def dkv_get_device_status(cache: dkv_cache, stream=None) -> int:

@@ -476,6 +476,15 @@ dkv_status dkv_get_device_status(const dkv_cache *cache, int32_t *host_out, void
 
 void dkv_debug_set_fault(int32_t mode) { g_debug_fault = mode == 1 ? 1 : 0; }
 
+dkv_status dkv_debug_division_check(const float *u_dev, int32_t n, uint64_t *mismatches_dev,
+                                    void *stream) {
+    if (!u_dev || !mismatches_dev || n < 1) return DKV_EINVAL;
+    if (!aligned16(u_dev) || !aligned16(mismatches_dev)) return DKV_EALIGN;
+    return cuda_status(dkv::launch_division_check(
+        u_dev, n, reinterpret_cast<unsigned long long *>(mismatches_dev),
+        static_cast<cudaStream_t>(stream)));
+}
+
 const char *dkv_status_str(dkv_status s) {
     switch (s) {
         case DKV_OK: return "ok";

@@ -331,6 +331,23 @@ __device__ inline int quant_lane(float v, __half *d16_out) {
     return min(15, max(0, c));
 }
 
+// Correctly rounded binary32 quotient a / b, given r = RN(1/b) (one
+// correctly rounded reciprocal serves every quotient by the same b).  One
+// refinement q1 = q0 + r (a - b q0) makes q1 faithful (relative error about
+// 4u^2 before rounding, u = 2^-24); then, with q1 faithful, the residual
+// a - b q1 is exact in one fused multiply-add and RN(q1 + r (a - b q1)) is
+// RN(a / b): the correction theorem of P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990.  Holds without overflow or underflow; a quotient below
+// the normal range (only for a subnormal dividend here) may differ in its last
+// bit, and feeds code 8 either way.  Checked against __fdiv_rn over every fp16
+// divisor by dkv_debug_division_check.
+__device__ inline float div_rn_markstein(float a, float b, float r) {
+    const float q0 = __fmul_rn(a, r);
+    const float q1 = __fmaf_rn(__fmaf_rn(-b, q0, a), r, q0);
+    return __fmaf_rn(__fmaf_rn(-b, q1, a), r, q1);
+}
+
 // The block rule on NC independent blocks at once (element lane of each),
 // written phase by phase -- every block's reduction, then every block's
 // vote, ... -- so the warp-wide steps of the blocks overlap instead of

@@ -17,6 +17,8 @@ struct CacheView;
 
 cudaError_t launch_encode(const CacheView &cv, const void *K, const void *V, int dtype,
                           const int32_t *seq_lens, int T_in, int append, cudaStream_t st);
+cudaError_t launch_division_check(const float *u, int n, unsigned long long *bad,
+                                  cudaStream_t st);
 cudaError_t launch_readback(const CacheView &cv, uint8_t *codes, uint16_t *scales,
                             uint16_t *keyframes, float *state, float *xhat, cudaStream_t st);
 

@@ -62,7 +62,10 @@ __device__ inline void pack_nibbles(const uint8_t (*codes)[D], int cnt, int t, u
 
 // Grid: x = work item within the batch entry's range (a group for DELTA, a
 // 32-position chunk otherwise), y = kvh * 2 + tensor, z = batch.  128 threads:
-// warp j handles channels 32j..32j+31 (one quantisation block).
+// warp j handles channels 32j..32j+31 (one quantisation block).  For the
+// delta format this is the variant with the most threads per step (a warp per
+// block): it serves appends of a few tokens, where the one-lane-per-block
+// kernel below would leave most of the GPU idle.
 template <int FMT>
 __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
     __shared__ uint8_t codes[SEG][D];
@@ -215,53 +218,70 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Delta format.  One warp per (batch entry, kv head, keyframe group) of the
-// range being written.  The warp carries the group's eight closed loops side
-// by side -- K and V, four 32-channel blocks each, lane = channel within its
-// block -- so every step of the sequential loop has eight independent
-// quantiser chains in flight; the next position's inputs are loaded while the
-// current one is quantised.  The nibble words are gathered in the permuted
-// layout with warp shuffles (lanes 0-15 write the K words of a position,
-// lanes 16-31 the V words) and the scales by lanes 0 and 1.  The quantiser is
-// quant_lane, in the same order of steps as the encode of every other path.
+// Delta format.  One lane per closed loop: a lane owns one 32-channel block of
+// one tensor of one keyframe group of one (batch entry, kv head) and runs the
+// group's positions in order with the whole block in its registers, so the
+// block rule needs no warp-wide step (the signed element of largest
+// magnitude is a scan in channel order with a strict comparison, which keeps
+// the lowest index on ties, as the rule states).  Lane l of a warp takes
+// block l & 3 of tensor (l >> 2) & 1 of group 4 q + (l >> 3), q the warp's
+// group quad.  The next position's 64 input bytes are loaded before the
+// current position is quantised.  Every quantiser step is one IEEE binary32
+// operation in the order of quant_lane.
 // ---------------------------------------------------------------------------
 constexpr int ENC_WARPS = 4;
+// Closed loops (group x tensor x block) from which the one-lane-per-loop
+// kernel is used: about two resident waves of its lanes on 148 SMs.
+constexpr int64_t kLaneKernelMinChains = 148 * 12 * 32 * 2;
 
-// Input element (tensor t, channel 32 j + lane) of relative position r.
-__device__ inline float enc_in(const EncodeArgs &a, int t, int64_t base, int r, int j, int lane) {
-    return load_in(t ? a.V : a.K, a.dtype, base + (int64_t)r * D + 32 * j + lane);
-}
+// The 32 inputs of one block at one position, as raw words (fp32: 32 words;
+// fp16 / bf16: 16 words of two halves).
+template <int DT>
+struct EncRow {
+    static constexpr int NW = DT == DKV_F32 ? 32 : 16;
+    uint32_t w[NW];
+    __device__ inline void load(const void *src, int64_t elem) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(
+            static_cast<const uint8_t *>(src) + elem * (DT == DKV_F32 ? 4 : 2));
+#pragma unroll
+        for (int k = 0; k < NW / 4; ++k) {
+            const uint4 v = __ldg(p + k);
+            w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+        }
+    }
+    __device__ inline float get(int c) const {
+        if (DT == DKV_F32) return __uint_as_float(w[c]);
+        const uint32_t u = w[c >> 1];
+        const unsigned short h = (c & 1) ? (unsigned short)(u >> 16) : (unsigned short)(u & 0xffffu);
+        if (DT == DKV_F16) return __half2float(__ushort_as_half(h));
+        return __bfloat162float(__ushort_as_bfloat16(h));
+    }
+};
 
-#ifndef DKV_ENC_MINB
-#define DKV_ENC_MINB 1
-#endif
-__global__ void __launch_bounds__(ENC_WARPS * 32, DKV_ENC_MINB) encode_delta_kernel(EncodeArgs a, int NG) {
+template <int DT>
+__global__ void __launch_bounds__(ENC_WARPS * 32) encode_delta_kernel(EncodeArgs a, int NQ) {
     const CacheView &cv = a.cv;
     const int lane = threadIdx.x & 31;
     const int64_t item = (int64_t)blockIdx.x * ENC_WARPS + (threadIdx.x >> 5);
     const int kf = cv.kf;
-    if (item < (int64_t)cv.B * cv.Hkv * NG) {
-        const int gi = (int)(item % NG);
-        const int bh = (int)(item / NG);
+    if (item < (int64_t)cv.B * cv.Hkv * NQ) {
+        const int qd = (int)(item % NQ);
+        const int bh = (int)(item / NQ);
         const int b = bh / cv.Hkv, kvh = bh % cv.Hkv;
+        const int gi = 4 * qd + (lane >> 3), t = (lane >> 2) & 1, j = lane & 3;
         int start, n;
         encode_range(a, b, start, n);
         const int parity = cv.header[2] & 1;
         const int64_t slot = (int64_t)cv.B * cv.Hkv * 2 * D;
-        const int64_t sb = ((int64_t)b * cv.Hkv + kvh) * 2 * D;
+        const int64_t sb = (((int64_t)b * cv.Hkv + kvh) * 2 + t) * D + 32 * j;
         const float *st_old = cv.state + parity * slot + sb;
         float *st_new = cv.state + (parity ^ 1) * slot + sb;
-        if (n < 0 && gi == 0 && kvh == 0 && lane == 0)
+        if (n < 0 && qd == 0 && kvh == 0 && lane == 0)
             set_status(cv.header, n == -2 ? DKV_DEV_CAPACITY : DKV_DEV_BAD_SEQLEN);
         if (n <= 0) {
-            if (gi == 0) {                    // nothing written: carry the state over
+            if (gi == 0) {                         // nothing written: carry the state over
 #pragma unroll
-                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int c = t * D + 32 * j + lane;
-                        st_new[c] = a.append ? st_old[c] : 0.0f;
-                    }
+                for (int c = 0; c < 32; ++c) st_new[c] = a.append ? st_old[c] : 0.0f;
             }
         } else {
             const int g = start / kf + gi;
@@ -272,95 +292,127 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, DKV_ENC_MINB) encode_delta_ker
                 // bad block-table entry (flagged by rec_ptr): nothing written
                 if (last) {
 #pragma unroll
-                    for (int t = 0; t < 2; ++t)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int c = t * D + 32 * j + lane;
-                            st_new[c] = (p0 % kf) ? st_old[c] : 0.0f;
-                        }
+                    for (int c = 0; c < 32; ++c) st_new[c] = (p0 % kf) ? st_old[c] : 0.0f;
                 }
             } else if (p0 < p1) {
-                const int64_t base = ((int64_t)b * cv.Hkv + kvh) * a.T_in * D;
-                float xh[2][4], x[2][4];
+                const void *src = t ? a.V : a.K;
+                const int64_t base = (((int64_t)b * cv.Hkv + kvh) * a.T_in - start) * D + 32 * j;
+                float xh[32];
 #pragma unroll
-                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        xh[t][j] = (p0 % kf) ? st_old[t * D + 32 * j + lane] : 0.0f;
-                        x[t][j] = enc_in(a, t, base, p0 - start, j, lane);
-                    }
-                const int wt = lane >> 4, ww = lane & 15;   // this lane's nibble word
-                uint8_t *nib0 = rec + KF_BYTES + (int64_t)(kf - 1) * SC_BYTES +
-                                (int64_t)wt * (kf - 1) * NIB_BYTES + 4 * ww;
+                for (int c = 0; c < 32; ++c) xh[c] = (p0 % kf) ? st_old[c] : 0.0f;
+                uint8_t *scl = rec + KF_BYTES + t * 8 + 2 * j;
+                uint8_t *nib = rec + KF_BYTES + (int64_t)(kf - 1) * SC_BYTES +
+                               (int64_t)t * (kf - 1) * NIB_BYTES;
+                EncRow<DT> cur, nxt;
+                cur.load(src, base + (int64_t)p0 * D);
 #pragma unroll 1
                 for (int p = p0; p < p1; ++p) {
-                    float xn[2][4];
-                    if (p + 1 < p1) {
-#pragma unroll
-                        for (int t = 0; t < 2; ++t)
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                xn[t][j] = enc_in(a, t, base, p + 1 - start, j, lane);
-                    }
+                    if (p + 1 < p1) nxt.load(src, base + (int64_t)(p + 1) * D);
                     const int di = p - g * kf;      // 0: keyframe; else delta di - 1
                     if (di == 0) {
+                        // keyframe: fp16 values at their permuted halfword slots
+                        __half h[32];
 #pragma unroll
-                        for (int t = 0; t < 2; ++t)
+                        for (int c = 0; c < 32; ++c) {
+                            h[c] = __float2half_rn(cur.get(c));
+                            xh[c] = __half2float(h[c]);
+                        }
+                        __half *kfr = reinterpret_cast<__half *>(rec + t * 256);
+                        if (t == 0) {
+                            // halfword t4 * 32 + 8 j + 4 s + 2 e + hh = channel 16 s + 8 e + 2 t4 + hh
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const __half h = __float2half_rn(x[t][j]);
-                                xh[t][j] = __half2float(h);
-                                const int ch = 32 * j + lane;
-                                reinterpret_cast<__half *>(rec + t * 256)[t == 0 ? k_half_idx(ch)
-                                                                                 : v_half_idx(ch)] = h;
+                            for (int t4 = 0; t4 < 4; ++t4) {
+                                uint32_t w4[4];
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const int s2 = k >> 1, e = k & 1;
+                                    const int c0 = 16 * s2 + 8 * e + 2 * t4;
+                                    w4[k] = (uint32_t)__half_as_ushort(h[c0]) |
+                                            ((uint32_t)__half_as_ushort(h[c0 + 1]) << 16);
+                                }
+                                *reinterpret_cast<uint4 *>(kfr + t4 * 32 + 8 * j) =
+                                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
                             }
+                        } else {
+                            // halfword gg * 16 + 4 j + 2 u + e = channel 16 u + gg + 8 e
+#pragma unroll
+                            for (int gg = 0; gg < 8; ++gg) {
+                                const uint32_t lo = (uint32_t)__half_as_ushort(h[gg]) |
+                                                    ((uint32_t)__half_as_ushort(h[gg + 8]) << 16);
+                                const uint32_t hi = (uint32_t)__half_as_ushort(h[16 + gg]) |
+                                                    ((uint32_t)__half_as_ushort(h[24 + gg]) << 16);
+                                *reinterpret_cast<uint2 *>(kfr + gg * 16 + 4 * j) = make_uint2(lo, hi);
+                            }
+                        }
                     } else {
-                        uint32_t codes = 0;         // code of (t, j) at bit 16 t + 4 j
-                        float dl[8];
-                        int cd[8];
-                        __half h16[8];
+                        float dl[32];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) dl[i] = __fsub_rn(x[i >> 2][i & 3], xh[i >> 2][i & 3]);
-                        quant_lanes<8>(dl, cd, h16);
-                        __half d16[2][4];
+                        for (int c = 0; c < 32; ++c) dl[c] = __fsub_rn(cur.get(c), xh[c]);
+                        // the signed element of largest magnitude, lowest index on
+                        // ties: a pairwise tree that keeps the left (lower-index)
+                        // element unless the right one is strictly larger
+                        float ta[16], tm[16];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int t = i >> 2, j = i & 3;
-                            d16[t][j] = h16[i];
-                            codes |= (uint32_t)cd[i] << (16 * t + 4 * j);
-                            xh[t][j] = __fadd_rn(xh[t][j], __fmul_rn((float)(cd[i] - 8),
-                                                                     __half2float(h16[i])));
+                        for (int i = 0; i < 16; ++i) {
+                            const float l = fabsf(dl[2 * i]), r = fabsf(dl[2 * i + 1]);
+                            const bool right = r > l;
+                            ta[i] = right ? r : l;
+                            tm[i] = right ? dl[2 * i + 1] : dl[2 * i];
                         }
-                        uint32_t word = 0;
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const int ch = nib_channel(wt, ww, k);
-                            const uint32_t v = __shfl_sync(0xffffffffu, codes, ch & 31);
-                            word |= ((v >> (16 * wt + 4 * (ch >> 5))) & 15u) << (4 * k);
-                        }
-                        *reinterpret_cast<uint32_t *>(nib0 + (int64_t)(di - 1) * NIB_BYTES) = word;
-                        if (lane < 2) {
-                            uint32_t h[4];
+                        for (int w = 8; w >= 1; w >>= 1)
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                h[j] = __half_as_ushort(lane ? d16[1][j] : d16[0][j]);
-                            *reinterpret_cast<uint2 *>(rec + KF_BYTES + (int64_t)(di - 1) * SC_BYTES +
-                                                       lane * 8) =
-                                make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+                            for (int i = 0; i < w; ++i) {
+                                const bool right = ta[2 * i + 1] > ta[2 * i];
+                                tm[i] = right ? tm[2 * i + 1] : tm[2 * i];
+                                ta[i] = right ? ta[2 * i + 1] : ta[2 * i];
+                            }
+                        const float m = tm[0];
+                        const __half d16 = __float2half_rn(__fmul_rn(m, -0.125f));
+                        const float d = __half2float(d16);
+                        const bool z = d == 0.0f;
+                        const float dd = z ? 1.0f : d;
+                        const float rd = __frcp_rn(dd);      // one reciprocal per block and position
+                        uint32_t code[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int cc =
+                                (int)truncf(__fadd_rn(div_rn_markstein(dl[c], dd, rd), 8.5f));
+                            code[c] = z ? 8u : (uint32_t)min(15, max(0, cc));
+                            xh[c] = __fadd_rn(xh[c], __fmul_rn((float)((int)code[c] - 8), d));
                         }
+                        uint8_t *row = nib + (int64_t)(di - 1) * NIB_BYTES;
+                        if (t == 0) {
+                            // word t4 * 4 + j, nibble 4 hh + 2 s + e = channel 16 s + 8 e + 2 t4 + hh
+#pragma unroll
+                            for (int t4 = 0; t4 < 4; ++t4) {
+                                uint32_t wd = 0;
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) {
+                                    const int hh = i >> 2, s2 = (i >> 1) & 1, e = i & 1;
+                                    wd |= code[16 * s2 + 8 * e + 2 * t4 + hh] << (4 * i);
+                                }
+                                reinterpret_cast<uint32_t *>(row)[t4 * 4 + j] = wd;
+                            }
+                        } else {
+                            // byte gg * 8 + 2 j + u = channel 16 u + gg (low) | 16 u + gg + 8 (high)
+#pragma unroll
+                            for (int gg = 0; gg < 8; ++gg) {
+                                const uint32_t b0 = code[gg] | (code[gg + 8] << 4);
+                                const uint32_t b1 = code[16 + gg] | (code[24 + gg] << 4);
+                                *reinterpret_cast<uint16_t *>(row + gg * 8 + 2 * j) =
+                                    (uint16_t)(b0 | (b1 << 8));
+                            }
+                        }
+                        *reinterpret_cast<__half *>(scl + (int64_t)(di - 1) * SC_BYTES) = d16;
                     }
-                    if (p + 1 < p1) {
-#pragma unroll
-                        for (int t = 0; t < 2; ++t)
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) x[t][j] = xn[t][j];
-                    }
+                    if (p + 1 < p1) cur = nxt;
                 }
                 if (last) {
 #pragma unroll
-                    for (int t = 0; t < 2; ++t)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) st_new[t * D + 32 * j + lane] = xh[t][j];
+                    for (int c = 0; c < 32; c += 4)
+                        *reinterpret_cast<float4 *>(st_new + c) =
+                            make_float4(xh[c], xh[c + 1], xh[c + 2], xh[c + 3]);
                 }
             }
         }
@@ -476,18 +528,60 @@ __global__ void __launch_bounds__(128) readback_kernel(ExportArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Test support: the encoder's quotient against __fdiv_rn.  Block x = one fp16
+// bit pattern of the divisor (every finite non-zero one); each thread takes
+// multipliers u_i and checks a = RN(u_i b) and its two neighbours.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) division_check_kernel(const float *u, int n,
+                                                             unsigned long long *bad) {
+    const uint16_t hb = (uint16_t)blockIdx.x;
+    const __half h = __ushort_as_half(hb);
+    const float b = __half2float(h);
+    if (!(b != 0.0f) || isinf(b) || isnan(b)) return;     // uniform over the block
+    const float r = __frcp_rn(b);
+    unsigned long long local = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const float a0 = __fmul_rn(u[i], b);
+        const float as[3] = {a0, nextafterf(a0, INFINITY), nextafterf(a0, -INFINITY)};
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const float x = __fdiv_rn(as[k], b), y = div_rn_markstein(as[k], b, r);
+            // the bits where the quotient is normal; the code it gives always
+            const bool normal = fabsf(x) >= 1.17549435e-38f;
+            const int cx = min(15, max(0, (int)truncf(__fadd_rn(x, 8.5f))));
+            const int cy = min(15, max(0, (int)truncf(__fadd_rn(y, 8.5f))));
+            if ((normal && __float_as_uint(x) != __float_as_uint(y)) || cx != cy) ++local;
+        }
+    }
+    if (local) atomicAdd(bad, local);
+}
+
+cudaError_t launch_division_check(const float *u, int n, unsigned long long *bad,
+                                  cudaStream_t st) {
+    division_check_kernel<<<65536, 256, 0, st>>>(u, n, bad);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------
 cudaError_t launch_encode(const CacheView &cv, const void *K, const void *V, int dtype,
                           const int32_t *seq_lens, int T_in, int append, cudaStream_t st) {
     EncodeArgs a{cv, K, V, dtype, seq_lens, T_in, append};
-    if (cv.fmt == DKV_FMT_DELTA) {
-        // groups a batch entry's range can touch (an append may start mid-group)
-        const int NG = (T_in + cv.kf - 1) / cv.kf + (append ? 1 : 0);
-        const int64_t warps = (int64_t)cv.B * cv.Hkv * NG;
+    // groups a batch entry's range can touch (an append may start mid-group)
+    const int NG = (T_in + cv.kf - 1) / cv.kf + (append ? 1 : 0);
+    if (cv.fmt == DKV_FMT_DELTA && (int64_t)cv.B * cv.Hkv * NG * 8 >= kLaneKernelMinChains) {
+        // enough closed loops to fill the GPU one lane each; four groups per warp
+        const int NQ = (NG + 3) / 4;
+        const int64_t warps = (int64_t)cv.B * cv.Hkv * NQ;
         const int64_t ctas = (warps + ENC_WARPS - 1) / ENC_WARPS;
         if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
-        encode_delta_kernel<<<(unsigned)ctas, ENC_WARPS * 32, 0, st>>>(a, NG);
+        if (dtype == DKV_F32)
+            encode_delta_kernel<DKV_F32><<<(unsigned)ctas, ENC_WARPS * 32, 0, st>>>(a, NQ);
+        else if (dtype == DKV_F16)
+            encode_delta_kernel<DKV_F16><<<(unsigned)ctas, ENC_WARPS * 32, 0, st>>>(a, NQ);
+        else
+            encode_delta_kernel<DKV_BF16><<<(unsigned)ctas, ENC_WARPS * 32, 0, st>>>(a, NQ);
         return cudaGetLastError();
     }
     int items;

@@ -364,6 +364,21 @@ dkv_status dkv_get_device_status(const dkv_cache *cache, int32_t *host_out, void
  * or faults either way.  Not thread-safe; meant for tests. */
 void dkv_debug_set_fault(int32_t mode);
 
+/* Test support (no counterpart on the pages): checks the quotient the
+ * delta encoder uses (one correctly rounded reciprocal of the block scale,
+ * then Markstein's exact-residual correction) against the IEEE division
+ * __fdiv_rn, for every finite non-zero fp16 divisor b and, for each of the n
+ * multipliers u_dev[i] (device fp32, 16-byte aligned), the dividends
+ * a = RN(u_i b) and its two floating-point neighbours.  Adds to
+ * *mismatches_dev (device uint64, 16-byte aligned; the caller zeroes it) the
+ * number of cases where the two quotients differ in a bit while the IEEE
+ * quotient is a normal number, or give different codes trunc(q + 8.5)
+ * clamped to 0..15 (a quotient below the normal range -- possible only when
+ * a itself is subnormal -- always gives code 8, so its last bit is free).
+ * Asynchronous on `stream`. */
+dkv_status dkv_debug_division_check(const float *u_dev, int32_t n, uint64_t *mismatches_dev,
+                                    void *stream);
+
 /* Static description of a status code. */
 const char *dkv_status_str(dkv_status s);
 

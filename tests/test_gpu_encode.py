@@ -117,3 +117,25 @@ def test_dequantize_matches_oracle_reconstruction(orc, dkv_gpu):
             for t, X in enumerate((K, V)):
                 ref = orc.encode_cache(fmt, X[0, h].float().numpy(), 32)["xhat"]
                 assert np.array_equal(xh[0, h, t].view(np.uint32), ref.view(np.uint32)), (fmt, h, t)
+
+
+def test_encoder_quotient_is_ieee_division(dkv_gpu):
+    """The delta encoder divides each delta by the block scale with one
+    correctly rounded reciprocal and Markstein's correction; it must give the
+    IEEE quotient bit for bit wherever that quotient is a normal number, and
+    the same code everywhere (a subnormal quotient, which needs a subnormal
+    delta, always gives code 8).  Checked for every finite non-zero fp16 scale
+    b and dividends RN(u b) (and their neighbours, including the smallest
+    subnormals next to an underflowed 0) with u over the quotients the block
+    rule meets: dense in [-17, 17], the exact halves k + 1/2, and small powers
+    of two down to 2^-60."""
+    g = torch.Generator().manual_seed(0)
+    u = torch.cat([torch.linspace(-17.0, 17.0, 24001, dtype=torch.float64),
+                   torch.arange(-34, 35, dtype=torch.float64) / 2.0,
+                   torch.rand(8000, generator=g, dtype=torch.float64) * 34.0 - 17.0,
+                   torch.tensor([s * 2.0 ** -k for k in range(1, 61) for s in (1, -1)],
+                                dtype=torch.float64)]).float().to(DEV)
+    bad = torch.zeros(2, dtype=torch.int64, device=DEV)
+    dkv_gpu.dkv_debug_division_check(u, bad)
+    torch.cuda.synchronize()
+    assert bad[0].item() == 0, bad[0].item()

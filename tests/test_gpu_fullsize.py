@@ -87,3 +87,34 @@ def test_ragged_long_with_appends(orc, dkv_gpu, kf):
     w = S.WORKLOADS["ragged_long"].with_(kf=kf)
     lens = [L + w.n_append for L in S.gen_lengths(w)]
     _check(orc, dkv_gpu, w, lens, n_append=w.n_append, samples=((0, 0), (3, 6)))
+
+
+def test_large_block_append_mid_group(orc, dkv_gpu):
+    """One append of 4000 tokens per sequence onto a prefix that ends inside a
+    keyframe group, at the batched-decode shape: enough closed loops that the
+    append runs one lane per loop (the prefill kernel), continuing from the
+    stored reconstruction."""
+    w = S.WORKLOADS["batched_decode"].with_(T=16384 - 37)
+    Tg = w.T
+    n = 4000
+    K = torch.empty((w.B, w.Hkv, Tg, w.D), dtype=w.kv_dtype, device=DEV)
+    V = torch.empty_like(K)
+    for b in range(w.B):
+        K[b], V[b] = S.gen_kv_one(w, b, Tg, device=DEV)
+    cache = dkv_gpu.Cache(w.B, w.Hkv, Tg, "delta", kf=w.kf)
+    cache.encode(K[:, :, :Tg - n].contiguous(), V[:, :, :Tg - n].contiguous())
+    cache.append(K[:, :, Tg - n:].contiguous(), V[:, :, Tg - n:].contiguous())
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    assert cache.seq_lens().tolist() == [Tg] * w.B
+    ex = cache.export()
+    for (b, h) in ((0, 0), (9, 4), (15, 7)):
+        for t, X in enumerate((K, V)):
+            ref = orc.delta_encode(X[b, h].float().cpu().numpy(), w.kf, cap=Tg)
+            assert np.array_equal(ex["codes"][b, h, t].cpu().numpy(), ref.codes), (b, h, t)
+            assert np.array_equal(ex["scales"][b, h, t].cpu().numpy().view(np.uint16), ref.scales)
+            ng = -(-Tg // w.kf)
+            assert np.array_equal(ex["keyframes"][b, h, t].cpu().numpy().view(np.uint16)[:ng],
+                                  ref.kfr[:ng])
+            assert np.array_equal(ex["state"][b, h, t].cpu().numpy().view(np.uint32),
+                                  ref.state.view(np.uint32))

@@ -159,6 +159,13 @@ def test_lr_decode_rejects_bad_arguments_on_host(dkv):
                                   A, A, nb, None) == dkv.DKV_EINVAL
 
 
+def test_division_check_rejects_bad_arguments(dkv):
+    lib = dkv.load()
+    assert lib.dkv_debug_division_check(None, 4, 1 << 12, None) == dkv.DKV_EINVAL
+    assert lib.dkv_debug_division_check(1 << 12, 0, 1 << 12, None) == dkv.DKV_EINVAL
+    assert lib.dkv_debug_division_check(1 << 12, 4, (1 << 12) + 8, None) == dkv.DKV_EALIGN
+
+
 def test_bad_dtype_and_sizes_rejected_on_host(dkv):
     """A well-formed view whose arguments are wrong: nothing is launched."""
     lib = dkv.load()
