@@ -113,6 +113,7 @@ struct SplitArgs {
     int Hq, G, NHG;            // query heads, heads per kv head, head groups of 8
     int nq;                    // queries per sequence (the newest nq tokens' own, causal)
     float scale_log2;          // softmax_scale * log2(e), > 0
+    float wshift;              // log2 of the factor every softmax weight is scaled down by
     float *ws;                 // partial records
     int fault;                 // test support: 1 = arm the copy barriers but issue no copy
     // fused append (cv.len_add = n > 0): the n new tokens of each sequence,
@@ -692,37 +693,39 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
             }
         } else {
             // PREFIX (kf > 32): the prefix weights -E_s aggregate up to kf
-            // positions, so every row's weight (times its V scale, in fp32) is an
-            // fp16 hi + lo pair.
-            auto make_b = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2]) {
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const uint32_t u = dvw[r][j >> 1];
-                    const float d = (j & 1) ? h_hi(u) : h_lo(u);
-                    const float v0 = w[t][r][0] * d, v1 = w[t][r][1] * d;
-                    const uint32_t hi = pack_h2(v0, v1);
-                    b[r] = movm_t(hi);
-                    bl[r] = movm_t(pack_h2(v0 - h_lo(hi), v1 - h_hi(hi)));
-                }
+            // positions; every B value is an fp16 hi + lo pair, made as for
+            // whole groups (above), and a third MMA against the scales alone
+            // (exact fp16 values) sums the group's dequantised deltas R_g.
+            const uint32_t wp0 = pack_h2(w[t][0][0], w[t][0][1]);
+            const uint32_t wp1 = pack_h2(w[t][1][0], w[t][1][1]);
+            const uint32_t wl0 = pack_h2(w[t][0][0] - h_lo(wp0), w[t][0][1] - h_hi(wp0));
+            const uint32_t wl1 = pack_h2(w[t][1][0] - h_lo(wp1), w[t][1][1] - h_hi(wp1));
+            auto make_b = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2], uint32_t (&rr)[2]) {
+                const uint32_t u0 = dvw[0][j >> 1], u1 = dvw[1][j >> 1];
+                const __half2 d0 = (j & 1) ? __high2half2(u32_as_h2(u0)) : __low2half2(u32_as_h2(u0));
+                const __half2 d1 = (j & 1) ? __high2half2(u32_as_h2(u1)) : __low2half2(u32_as_h2(u1));
+                const __half2 h0 = __hmul2(u32_as_h2(wp0), d0);
+                const __half2 h1 = __hmul2(u32_as_h2(wp1), d1);
+                const __half2 l0 = __hfma2(u32_as_h2(wl0), d0,
+                                           __hfma2(u32_as_h2(wp0), d0, __hneg2(h0)));
+                const __half2 l1 = __hfma2(u32_as_h2(wl1), d1,
+                                           __hfma2(u32_as_h2(wp1), d1, __hneg2(h1)));
+                b[0] = movm_t(h2_as_u32(h0));
+                b[1] = movm_t(h2_as_u32(h1));
+                bl[0] = movm_t(h2_as_u32(l0));
+                bl[1] = movm_t(h2_as_u32(l1));
+                rr[0] = movm_t(h2_as_u32(d0));
+                rr[1] = movm_t(h2_as_u32(d1));
             };
-            uint32_t bp[2], bl[2];
+            uint32_t bp[2], bl[2], rr[2];
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 uint32_t a0, a1, a2, a3;
                 codes(mt, a0, a1, a2, a3);
-                const int j = mt >> 1;
-                if ((mt & 1) == 0) make_b(j, bp, bl);
+                if ((mt & 1) == 0) make_b(mt >> 1, bp, bl, rr);
                 mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
                 mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
-                // R += sum_s (code-8) * d_s : B = the scales alone
-                uint32_t r2[2];
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const uint32_t u = dvw[r][j >> 1];
-                    const float d = (j & 1) ? h_hi(u) : h_lo(u);
-                    r2[r] = movm_t(pack_h2(d, d));
-                }
-                mma16816(racc[mt], a0, a1, a2, a3, r2[0], r2[1]);
+                mma16816(racc[mt], a0, a1, a2, a3, rr[0], rr[1]);   // R += (code - 8) d
             }
         }
     }
@@ -1182,12 +1185,16 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
                 const float m_new = fmaxf(m_run[e], mx * A.scale_log2);
                 alpha[e] = ex2(m_run[e] - m_new);
                 m_run[e] = m_new;
+                // every weight (and so the sum and the output) times 2^-wshift:
+                // a weight's sum over a group times a V scale then stays inside
+                // the fp16 range; out = O / L does not change
+                const float m_sh = -m_new - A.wshift;
                 float psum = 0.f;
 #pragma unroll
                 for (int u = 0; u < NU; ++u)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        v[u][i] = ex2(fmaf(v[u][i], A.scale_log2, -m_new));
+                        v[u][i] = ex2(fmaf(v[u][i], A.scale_log2, m_sh));
                         psum += v[u][i];
                     }
                 l_run[e] = l_run[e] * alpha[e] + psum;
@@ -1340,16 +1347,9 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
     auto has = [&](int64_t w) {
         return w <= w1 && (dense || range_start(w, NW, T) < range_start(w + 1, NW, T));
     };
-    float M = -INFINITY;
-    for (int64_t w = w0; w <= w1; w += BATCH) {
-        float mv[BATCH];
-#pragma unroll
-        for (int i = 0; i < BATCH; ++i)
-            mv[i] = has(w + i) ? ws[(w + i + vseq) * PARTIAL_FLOATS + j] : -INFINITY;
-#pragma unroll
-        for (int i = 0; i < BATCH; ++i) M = fmaxf(M, mv[i]);
-    }
-    float L = 0.f, O = 0.f;
+    // one pass, rescaling online: each batch of 8 records moves the running
+    // maximum once (records of warps that saw no position carry -1e30)
+    float M = -1e30f, L = 0.f, O = 0.f;
     for (int64_t w = w0; w <= w1; w += BATCH) {
         float mv[BATCH], lv[BATCH], ov[BATCH];
         bool ok[BATCH];
@@ -1357,17 +1357,23 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
         for (int i = 0; i < BATCH; ++i) {
             ok[i] = has(w + i);
             const float *rec = ws + (w + i + vseq) * PARTIAL_FLOATS;
-            mv[i] = ok[i] ? rec[j] : 0.f;
+            mv[i] = ok[i] ? rec[j] : -1e30f;
             lv[i] = ok[i] ? rec[8 + j] : 0.f;
             ov[i] = ok[i] ? rec[16 + j * 128 + c] : 0.f;
         }
+        float Mn = M;
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) Mn = fmaxf(Mn, mv[i]);
+        const float sc = exp2f(M - Mn);
+        L *= sc;
+        O *= sc;
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
-            if (!ok[i]) continue;
-            const float sc = exp2f(mv[i] - M);
-            L += lv[i] * sc;
-            O += ov[i] * sc;
+            const float e = exp2f(mv[i] - Mn);
+            L = fmaf(lv[i], e, L);
+            O = fmaf(ov[i], e, O);
         }
+        M = Mn;
     }
     dst[c] = L > 0.f ? O / L : 0.f;     // a causal query with no position gets 0
 }
@@ -1440,17 +1446,37 @@ static cudaError_t geom_for(SplitGeom *g) {
 
 // The kernel instance for a cache: format, mode (kf <= 32: whole groups per
 // unit; kf > 32: 32-position segments) and whether tail slots need their
-// scales zeroed (kf != 32 for the delta format).  The merge derives the warp
-// count from the same instance the split launched.
-cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g) {
-    (void)batch;
+// scales zeroed (kf != 32 for the delta format).  The persistent grid fills
+// the GPU, but never gives a warp fewer than kMinUnitsPerWarp of the most
+// units the cache can hold (max_units), so a small cache is not spread over
+// warps that would own nothing (the merge walks the warps of a sequence).
+// The merge and the workspace size derive the warp count the same way.
+constexpr int64_t kMinUnitsPerWarp = 4;
+
+static void clamp_geometry(SplitGeom *g, int64_t max_units) {
+    const int64_t want = (max_units + kMinUnitsPerWarp * WARPS - 1) / (kMinUnitsPerWarp * WARPS);
+    if (want < g->ctas) g->ctas = (int)(want < 1 ? 1 : want);
+}
+
+cudaError_t split_geometry(int fmt, int kf, int64_t max_units, SplitGeom *g) {
+    cudaError_t e;
     if (fmt == DKV_FMT_DELTA) {
-        if (kf == SEG) return geom_for<DKV_FMT_DELTA, SUFFIX, false>(g);
-        return kf < SEG ? geom_for<DKV_FMT_DELTA, SUFFIX, true>(g)
-                        : geom_for<DKV_FMT_DELTA, PREFIX, true>(g);
+        if (kf == SEG) e = geom_for<DKV_FMT_DELTA, SUFFIX, false>(g);
+        else e = kf < SEG ? geom_for<DKV_FMT_DELTA, SUFFIX, true>(g)
+                          : geom_for<DKV_FMT_DELTA, PREFIX, true>(g);
+    } else if (fmt == DKV_FMT_Q4_0) {
+        e = geom_for<DKV_FMT_Q4_0, PLAIN, false>(g);
+    } else {
+        e = geom_for<DKV_FMT_FP16, PLAIN, false>(g);
     }
-    if (fmt == DKV_FMT_Q4_0) return geom_for<DKV_FMT_Q4_0, PLAIN, false>(g);
-    return geom_for<DKV_FMT_FP16, PLAIN, false>(g);
+    if (e == cudaSuccess) clamp_geometry(g, max_units);
+    return e;
+}
+
+// Units the split kernel can see for a cache: every sequence (b, kv head,
+// head group) at capacity.
+int64_t split_max_units(int fmt, int kf, int B, int Hkv, int nhg, int cap) {
+    return (int64_t)B * Hkv * nhg * units_of(fmt, fmt == DKV_FMT_DELTA ? kf : 1, cap);
 }
 
 // Every instance runs on the contiguous one-query instance's grid (the merge
@@ -1491,6 +1517,8 @@ static cudaError_t launch_split_t(const SplitArgs &a_in, cudaStream_t st) {
     SplitGeom g;
     cudaError_t e = geom_for<FMT, MODE, ZT>(&g);
     if (e != cudaSuccess) return e;
+    clamp_geometry(&g, split_max_units(a_in.cv.fmt, a_in.cv.kf, a_in.cv.B, a_in.cv.Hkv, a_in.NHG,
+                                       a_in.cv.cap));
     const SplitArgs &a = a_in;
     const bool paged = a.cv.pg != 0, mq = a.nq > 1, app = a.cv.len_add > 0;
     if (!paged && !mq && !app) return launch_q<FMT, MODE, ZT, false, false, false>(a, g.ctas, st);
@@ -1526,6 +1554,14 @@ cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq
     a.nq = nq;
     a.NHG = (nq * a.G + 7) / 8;
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
+    // weight scaling: 2^-ceil(log2 kf) for the delta format (a weight sum over
+    // a group is at most kf), none for the comparators (one token per row)
+    a.wshift = 0.f;
+    if (cv.fmt == DKV_FMT_DELTA) {
+        int sh = 0;
+        while ((1 << sh) < cv.kf && sh < 24) ++sh;
+        a.wshift = (float)sh;
+    }
     a.ws = ws;
     if (cv.fmt == DKV_FMT_DELTA) {
         if (cv.kf == SEG) return launch_split_t<DKV_FMT_DELTA, SUFFIX, false>(a, st);
@@ -1538,11 +1574,12 @@ cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq
 
 cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const float *ws,
                          cudaStream_t st) {
-    SplitGeom g;
-    cudaError_t e = split_geometry(cv.fmt, cv.kf, cv.B, &g);
-    if (e != cudaSuccess) return e;
     const int G = Hq / cv.Hkv;
     const int NHG = (nq * G + 7) / 8;
+    SplitGeom g;
+    cudaError_t e = split_geometry(cv.fmt, cv.kf, split_max_units(cv.fmt, cv.kf, cv.B, cv.Hkv, NHG,
+                                                                  cv.cap), &g);
+    if (e != cudaSuccess) return e;
     dim3 grid(nq * Hq, cv.B);
     const int64_t NW = (int64_t)g.ctas * g.warps_per_cta;
     if (cv.len_add > 0)

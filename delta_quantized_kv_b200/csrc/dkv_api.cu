@@ -125,10 +125,14 @@ int64_t workspace_floats(const dkv_cache_desc *d, int32_t Hq, int32_t nq, bool *
     *ok = false;
     if (check_desc(d) != DKV_OK || Hq < 1 || Hq % d->n_kv_heads != 0) return 0;
     if (nq < 1 || nq > kMaxQueries) return 0;
-    dkv::SplitGeom g;
-    if (dkv::split_geometry(d->fmt, d->kf, d->batch, &g) != cudaSuccess) return 0;
     const int G = Hq / d->n_kv_heads;
     const int64_t nhg = ((int64_t)nq * G + 7) / 8;
+    dkv::SplitGeom g;
+    if (dkv::split_geometry(d->fmt, d->kf,
+                            dkv::split_max_units(d->fmt, d->kf, d->batch, d->n_kv_heads, (int)nhg,
+                                                 d->max_ctx),
+                            &g) != cudaSuccess)
+        return 0;
     const int64_t slots = (int64_t)g.ctas * g.warps_per_cta + (int64_t)d->batch * d->n_kv_heads * nhg;
     *ok = true;
     // + the decoded lengths of a fused append + decode, int32[B]

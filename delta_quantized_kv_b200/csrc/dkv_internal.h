@@ -28,7 +28,11 @@ struct SplitGeom {
     int ctas;
     int warps_per_cta;
 };
-cudaError_t split_geometry(int fmt, int kf, int batch, SplitGeom *g);
+cudaError_t split_geometry(int fmt, int kf, int64_t max_units, SplitGeom *g);
+// Units (keyframe groups, kf > 32: 32-position segments, or 32-position
+// chunks) of every sequence of a cache at capacity; nhg = head groups of 8
+// virtual heads per kv head.
+int64_t split_max_units(int fmt, int kf, int B, int Hkv, int nhg, int cap);
 
 // Floats per partial record: m[8], l[8], o[8][128].
 constexpr int PARTIAL_FLOATS = 8 + 8 + 8 * 128;

@@ -230,8 +230,9 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
 // operation in the order of quant_lane.
 // ---------------------------------------------------------------------------
 constexpr int ENC_WARPS = 4;
-// Closed loops (group x tensor x block) from which the one-lane-per-loop
-// kernel is used: about two resident waves of its lanes on 148 SMs.
+// Closed loops (group x tensor x block) from which an append uses the
+// one-lane-per-loop kernel: about two resident waves of its lanes on 148
+// SMs.  Encodes always use it.
 constexpr int64_t kLaneKernelMinChains = 148 * 12 * 32 * 2;
 
 // The 32 inputs of one block at one position, as raw words (fp32: 32 words;
@@ -570,8 +571,10 @@ cudaError_t launch_encode(const CacheView &cv, const void *K, const void *V, int
     EncodeArgs a{cv, K, V, dtype, seq_lens, T_in, append};
     // groups a batch entry's range can touch (an append may start mid-group)
     const int NG = (T_in + cv.kf - 1) / cv.kf + (append ? 1 : 0);
-    if (cv.fmt == DKV_FMT_DELTA && (int64_t)cv.B * cv.Hkv * NG * 8 >= kLaneKernelMinChains) {
-        // enough closed loops to fill the GPU one lane each; four groups per warp
+    if (cv.fmt == DKV_FMT_DELTA &&
+        (!append || (int64_t)cv.B * cv.Hkv * NG * 8 >= kLaneKernelMinChains)) {
+        // an encode, or an append with enough closed loops to fill the GPU one
+        // lane each; four groups per warp
         const int NQ = (NG + 3) / 4;
         const int64_t warps = (int64_t)cv.B * cv.Hkv * NQ;
         const int64_t ctas = (warps + ENC_WARPS - 1) / ENC_WARPS;

@@ -84,3 +84,34 @@ def test_attention_stress(orc, dkv_gpu, kf, seed):
             worst = max(worst, e)
             assert e <= ATTN_TOL, (qdt, scale, e, bi, hi)
     WORST[kf, seed] = worst
+
+
+@pytest.mark.parametrize("kf", [32, 512])
+def test_attention_large_magnitudes(orc, dkv_gpu, kf):
+    """Keys and values near the top of the fp16 range with whole-token jumps:
+    block scales of several thousand.  A weight summed over a keyframe group
+    times such a scale would pass the fp16 range if the weights were not
+    scaled down; the output must stay finite and within tolerance."""
+    lens = LENS[kf]
+    B, Hkv, G = len(lens), 2, 8
+    T = max(lens)
+    w = S.WORKLOADS["llama3_70b_layer"].with_(B=B, Hkv=Hkv, Hq=Hkv * G, T=T, kf=kf,
+                                              jump_p=0.2, seed=5100 + kf)
+    K, V = S.gen_kv(w)
+    K = (K.float() * 600.0).clamp(-6.0e4, 6.0e4).to(torch.float16)
+    V = (V.float() * 2000.0).clamp(-6.0e4, 6.0e4).to(torch.float16)
+    cache = dkv_gpu.Cache(B, Hkv, T, "delta", kf=kf)
+    cache.encode(K.to(DEV), V.to(DEV), seq_lens=torch.tensor(lens, dtype=torch.int32,
+                                                             device=DEV))
+    q = S.gen_q(w)
+    for scale in (1e-4, 1e-3):
+        out = cache.decode_attn(q.to(DEV), scale)
+        torch.cuda.synchronize()
+        assert cache.device_status() == 0
+        got = out.cpu().double().numpy()
+        assert np.isfinite(got).all()
+        ref = orc.decode_attention("delta", q.double().numpy(), K.float().numpy(),
+                                   V.float().numpy(), kf=kf, scale=scale, lengths=lens)
+        e = float(row_rel_err(got, ref).max())
+        print(f"[stress-large] kf={kf} scale={scale} worst={e:.3e}")
+        assert e <= ATTN_TOL, (scale, e)
