@@ -93,9 +93,23 @@ template <int FMT, int MODE> struct SmemMap {
 };
 
 
+// Work units of a sequence of len tokens: keyframe groups for the delta
+// format with kf <= 32; 32-position segments of the groups for kf > 32 (a
+// group of kf tokens holds ceil(kf / 32) of them); 32-position chunks for the
+// comparators.
+__host__ __device__ inline int seg_per_group(int kf) { return (kf + SEG - 1) / SEG; }
 __host__ __device__ inline int units_of(int fmt, int kf, int len) {
     if (len <= 0) return 0;
-    return fmt == DKV_FMT_DELTA ? (len + kf - 1) / kf : (len + SEG - 1) / SEG;
+    if (fmt != DKV_FMT_DELTA) return (len + SEG - 1) / SEG;
+    if (kf <= SEG) return (len + kf - 1) / kf;
+    return (len / kf) * seg_per_group(kf) + (len % kf + SEG - 1) / SEG;
+}
+// First position of unit u of a sequence (units are contiguous in position).
+__host__ __device__ inline int64_t unit_pos(int fmt, int kf, int64_t u) {
+    if (fmt != DKV_FMT_DELTA) return u * SEG;
+    if (kf <= SEG) return u * kf;
+    const int spg = seg_per_group(kf);
+    return (u / spg) * kf + (u % spg) * SEG;
 }
 
 // Warp w of NW owns units [w*T/NW, (w+1)*T/NW).
@@ -115,6 +129,7 @@ struct SplitArgs {
     float scale_log2;          // softmax_scale * log2(e), > 0
     float wshift;              // log2 of the factor every softmax weight is scaled down by
     float *ws;                 // partial records
+    float *heads, *hands;      // kf > 32: the records of groups entered midway, the handoffs
     int fault;                 // test support: 1 = arm the copy barriers but issue no copy
     // fused append (cv.len_add = n > 0): the n new tokens of each sequence,
     // [B][Hkv][n][D] of kv_dtype
@@ -140,10 +155,12 @@ __device__ inline int clamp_len(const CacheView &cv, int b) {
 // Iterates the (unit, segment) stage items of one warp's range in order.
 struct Cursor {
     int64_t left;              // units left in the range, the current one included
-    int b, vs, g;              // batch entry, sequence within the batch entry, unit
+    int b, vs, g;              // batch entry, sequence within the batch entry, group / chunk
     int units_b;               // units per sequence of batch entry b
+    int groups_b;              // values of g per sequence of batch entry b
     int len_b;                 // tokens of batch entry b
-    int seg, nseg;             // segment within the unit (kf > 32 only)
+    int seg, nseg;             // segment within group g and the group's segments (kf > 32)
+    bool head;                 // kf > 32: group g was entered after its first segment
     const uint8_t *seq;        // data of sequence (b, kv head of vs) (contiguous caches)
     // paged caches, issuing lane only: the page last looked up
     int pb, pv, pidx;          // its batch entry, sequence and block-table column
@@ -204,8 +221,19 @@ __device__ inline void cursor_seek(Cursor &c, const CacheView &cv, int nvs, int 
     c.units_b = units_of(cv.fmt, cv.kf, c.len_b);
     const int64_t r = x - base;
     c.vs = (int)(r / c.units_b);
-    c.g = (int)(r % c.units_b);
-    c.seg = 0;
+    const int u = (int)(r % c.units_b);
+    if (MODE == PREFIX) {
+        const int spg = seg_per_group(cv.kf);
+        c.groups_b = (c.len_b + cv.kf - 1) / cv.kf;
+        c.g = u / spg;
+        c.seg = u % spg;
+        c.head = c.seg != 0;
+    } else {
+        c.groups_b = c.units_b;
+        c.g = u;
+        c.seg = 0;
+        c.head = false;
+    }
     c.nseg = nseg_of<MODE>(cv, c.len_b, c.g);
     c.seq = seq_ptr(cv, c.b, c.vs, nhg);
     c.pb = -1;
@@ -213,10 +241,11 @@ __device__ inline void cursor_seek(Cursor &c, const CacheView &cv, int nvs, int 
 
 template <int MODE>
 __device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs, int nhg) {
+    if (--c.left == 0) return;
     if (MODE == PREFIX && ++c.seg < c.nseg) return;
     c.seg = 0;
-    if (--c.left == 0) return;
-    if (++c.g == c.units_b) {
+    c.head = false;
+    if (++c.g == c.groups_b) {
         c.g = 0;
         if (++c.vs == nvs) {
             c.vs = 0;
@@ -225,6 +254,7 @@ __device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs, int 
                 c.len_b = clamp_len(cv, c.b);
                 c.units_b = units_of(cv.fmt, cv.kf, c.len_b);
             } while (c.units_b == 0);
+            c.groups_b = MODE == PREFIX ? (c.len_b + cv.kf - 1) / cv.kf : c.units_b;
         }
         c.seq = seq_ptr(cv, c.b, c.vs, nhg);
     }
@@ -236,17 +266,37 @@ __device__ inline void cursor_next(Cursor &c, const CacheView &cv, int nvs, int 
 __host__ __device__ inline int32_t *merge_lengths(float *ws, int64_t NW, int64_t nseq) {
     return reinterpret_cast<int32_t *>(ws + (NW + nseq) * PARTIAL_FLOATS);
 }
+// kf > 32, after the lengths: per warp slot, the partial record of the group
+// its range entered after the group's first segment (scores relative to the
+// state before its first position); then the log2 softmax scale (a header of
+// HAND_HDR floats) and, per warp slot, the state it hands to the next warp
+// when its range ends inside a group: the dot of each head's query with the
+// reconstructed key of its last position (8 floats) and the reconstructed
+// value row there (128 floats).  Both are relative to the state the warp
+// entered the group with when it entered it after the first segment,
+// absolute otherwise.
+__host__ __device__ inline float *head_records(float *ws, int64_t NW, int64_t nseq, int B) {
+    return ws + (NW + nseq) * PARTIAL_FLOATS + ((int64_t)B + 3) / 4 * 4;
+}
+__host__ __device__ inline float *handoffs(float *ws, int64_t NW, int64_t nseq, int B) {
+    return head_records(ws, NW, nseq, B) + NW * PARTIAL_FLOATS;
+}
 
 // What the consumer needs to know about a stage, written next to the stage by
 // the issuing lane before it arms the barrier.
 struct StageMeta {
     int b, vs;                 // batch entry, sequence within it
     int npos;                  // valid positions: unit 0 in bits 0-7, unit 1 in bits 8-15
-    int flags;                 // bit 0: first segment of a group; bit 1: last segment
+    int flags;                 // kf > 32: the STG_* bits below
     int pos0;                  // position of unit 0's first slot in its sequence
     int pad[3];
 };
 static_assert(sizeof(StageMeta) == 32, "stage descriptors are 32 bytes");
+// Stage flags (kf > 32, one segment per stage).
+constexpr int STG_FIRST = 1;   // first segment of its group: slot 0 is the keyframe
+constexpr int STG_CLOSE = 2;   // the group's last segment in this warp's range
+constexpr int STG_HEAD = 4;    // the range entered this group after its first segment
+constexpr int STG_HAND = 8;    // the range ends inside this group (hand the state on)
 
 // Positions of the current unit of c.
 __device__ inline int unit_npos(const CacheView &cv, const Cursor &c, int g) {
@@ -400,7 +450,13 @@ __device__ inline StageMeta next_stage(const CacheView &cv, Cursor &c, int nvs, 
     m.b = c.b;
     m.vs = c.vs;
     m.npos = np0 | (np1 << 8);
-    m.flags = MODE == PREFIX ? ((c.seg == 0 ? 1 : 0) | (c.seg == c.nseg - 1 ? 2 : 0)) : 3;
+    if (MODE == PREFIX) {
+        const bool group_end = c.seg == c.nseg - 1, range_end = c.left == 1;
+        m.flags = (c.seg == 0 ? STG_FIRST : 0) | (group_end || range_end ? STG_CLOSE : 0) |
+                  (c.head ? STG_HEAD : 0) | (range_end && !group_end ? STG_HAND : 0);
+    } else {
+        m.flags = STG_FIRST | STG_CLOSE;
+    }
     m.pos0 = FMT == DKV_FMT_DELTA ? c.g * cv.kf + c.seg * SEG : c.g * SEG;
     if (lane == 0) {
         if (KCfg<FMT, MODE>::NS > 1) *meta = m;
@@ -756,8 +812,8 @@ __device__ inline float load_new(const void *src, int dtype, int64_t row, int c)
 }
 
 template <bool PAGED>
-__device__ __noinline__ void append_tokens(const SplitArgs &A, int b, int kvh, int L0, int g_lo,
-                                           int g_hi, bool write_state) {
+__device__ __noinline__ void append_tokens(const SplitArgs &A, int b, int kvh, int L0, int p_lo,
+                                           int p_hi, bool write_state) {
     const CacheView &cv = A.cv;
     const int lane = threadIdx.x & 31, kf = cv.kf, n = cv.len_add;
     const int64_t sb = ((int64_t)b * cv.Hkv + kvh) * 2 * D;          // (b, kvh) in a slot
@@ -787,8 +843,8 @@ __device__ __noinline__ void append_tokens(const SplitArgs &A, int b, int kvh, i
 #pragma unroll 1
     for (int i = 0; i < n; ++i) {
         const int p = L0 + i, g = p / kf, di = p - g * kf;   // di 0: keyframe; else delta di - 1
-        if (g > g_hi) break;
-        uint8_t *rec = g >= g_lo ? rec_ptr<PAGED>(cv, b, kvh, g) : nullptr;
+        if (p >= p_hi) break;
+        uint8_t *rec = p >= p_lo ? rec_ptr<PAGED>(cv, b, kvh, g) : nullptr;
         if (di == 0) {
 #pragma unroll
             for (int t = 0; t < 2; ++t)
@@ -858,36 +914,37 @@ __device__ __noinline__ void append_tokens(const SplitArgs &A, int b, int kvh, i
 }
 
 // The new tokens that land in units [lo, hi) of a warp's range (offsets from
-// the range's first unit, which is group g0 of sequence vs of batch entry b,
-// a sequence of ub units): walk the sequences those units belong to and
-// quantise, for each, the new tokens of the groups held there.  The owner of a
-// sequence's last group (head group 0) writes the state.  Returns whether this
-// warp stored anything.
+// the range's first unit, which is unit u0 of sequence vs of batch entry b, a
+// sequence of ub units): walk the sequences those units belong to and
+// quantise, for each, the new tokens from the first one on, storing those at
+// the positions of the units held there.  The owner of a sequence's last unit
+// (head group 0) writes the state.  Returns whether this warp stored anything.
 template <bool PAGED>
-__device__ __noinline__ bool append_range(const SplitArgs &A, int nvs, int b, int vs, int g0,
+__device__ __noinline__ bool append_range(const SplitArgs &A, int nvs, int b, int vs, int u0,
                                           int ub, int64_t lo, int64_t hi) {
     const CacheView &cv = A.cv;
     bool wrote = false;
-    int64_t off = 0;                    // offset of group g0 of (b, vs) in the range
+    int64_t off = 0;                    // offset of unit u0 of (b, vs) in the range
 #pragma unroll 1
     while (off < hi) {
-        const int64_t seg = ub - g0;    // units of this sequence from g0 on
-        if (off + seg > lo) {
-            const int ga = g0 + (int)max((int64_t)0, lo - off);
-            const int gb = g0 + (int)(min(hi, off + seg) - off) - 1;
+        const int64_t here = ub - u0;   // units of this sequence from u0 on
+        if (off + here > lo) {
+            const int ua = u0 + (int)max((int64_t)0, lo - off);
+            const int ue = u0 + (int)(min(hi, off + here) - off);       // exclusive
             int L;
             if (takes_append(cv, b, L)) {
-                const int first = max(ga, L / cv.kf);
-                if (first <= gb) {
-                    append_tokens<PAGED>(A, b, A.NHG == 1 ? vs : vs / A.NHG, L, first, gb,
-                                         gb == ub - 1 && vs % A.NHG == 0);
+                const int p_lo = max((int)unit_pos(cv.fmt, cv.kf, ua), L);
+                const int p_hi = min((int)unit_pos(cv.fmt, cv.kf, ue), L + cv.len_add);
+                if (p_lo < p_hi) {
+                    append_tokens<PAGED>(A, b, A.NHG == 1 ? vs : vs / A.NHG, L, p_lo, p_hi,
+                                         ue == ub && vs % A.NHG == 0);
                     wrote = true;
                 }
             }
         }
-        off += seg;
+        off += here;
         if (off >= hi) break;
-        g0 = 0;
+        u0 = 0;
         if (++vs == nvs) {
             vs = 0;
             do {
@@ -964,6 +1021,7 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
             }
         }
     }
+    if (MODE == PREFIX && gw == 0 && lane == 0) A.hands[0] = A.scale_log2;   // for the merge
     if (total == 0) return;
     const int64_t r0 = range_start(gw, NW, total), r1 = range_start(gw + 1, NW, total);
     if (r0 >= r1) return;
@@ -974,7 +1032,8 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
     // are stored before those copies are issued; the rest after, while the
     // first copies are in flight (each warp copies a record only after its
     // own stores and a proxy fence)
-    const int ab = ic.b, avs = ic.vs, ag = ic.g, aub = ic.units_b;
+    const int ab = ic.b, avs = ic.vs, aub = ic.units_b;
+    const int ag = MODE == PREFIX ? ic.g * seg_per_group(cv.kf) + ic.seg : ic.g;   // unit
     constexpr int64_t PRE = (int64_t)NS * NU;
     if constexpr (APP) {
         if (append_range<PAGED>(A, nvs, ab, avs, ag, aub, 0, min(PRE, r1 - r0))) {
@@ -1023,8 +1082,9 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
 #pragma unroll
     for (int i = 0; i < 8; ++i) vkf_keep[i] = 0;
 
-    auto flush = [&]() {
-        // write the partial record of the current sequence
+    auto write_record = [&](float *rec) {
+        // the partial record (m, l, o) of heads 2tq, 2tq + 1 (l summed over
+        // the warp here)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             float l = l_run[e];
@@ -1033,8 +1093,6 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
             l += __shfl_xor_sync(0xffffffffu, l, 16);
             l_run[e] = l;
         }
-        const int64_t vseq = (int64_t)cur_b * nvs + cur_vs;
-        float *rec = A.ws + (gw + vseq) * PARTIAL_FLOATS;
         if (gq == 0) {
             rec[2 * tq] = m_run[0];
             rec[2 * tq + 1] = m_run[1];
@@ -1049,6 +1107,10 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
             rec[16 + (2 * tq) * 128 + c0 + 8] = o[mt][2];
             rec[16 + (2 * tq + 1) * 128 + c0 + 8] = o[mt][3];
         }
+    };
+    // the partial record of the current sequence
+    auto flush = [&]() {
+        write_record(A.ws + (gw + (int64_t)cur_b * nvs + cur_vs) * PARTIAL_FLOATS);
     };
 
 #pragma unroll 1
@@ -1241,18 +1303,45 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
                                   racc, vkf_keep);
             }
 
-            // PREFIX: close the group  o += W_g (v_f + R_g)
+            // PREFIX: close the group (or this range's part of it)
+            //   o += W_g (v_f + R_g)
+            // where v_f is 0 for a group entered midway (its rows are then
+            // relative to the value row before the range's first position)
             if (MODE == PREFIX && last_seg) {
+                // a range that ends inside the group hands the next warp the
+                // scaled dots of its last position and that position's value row
+                const bool hand = (meta.flags & STG_HAND) != 0;
+                float *hd = A.hands + HAND_HDR + gw * HANDOFF_FLOATS;
+                if (hand && gq == 0) {
+                    hd[2 * tq] = dot_carry[0];
+                    hd[2 * tq + 1] = dot_carry[1];
+                }
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
                     const float v_lo = h_lo(vkf_keep[mt]) + racc[mt][0];   // channel 16mt+g
                     const float v_hi = h_hi(vkf_keep[mt]) + racc[mt][2];   // channel 16mt+g+8
+                    if (hand && tq == 0) {
+                        hd[8 + 16 * mt + gq] = v_lo;
+                        hd[8 + 16 * mt + gq + 8] = v_hi;
+                    }
                     o[mt][0] += e_carry[0] * v_lo; o[mt][1] += e_carry[1] * v_lo;
                     o[mt][2] += e_carry[0] * v_hi; o[mt][3] += e_carry[1] * v_hi;
                     racc[mt][0] = racc[mt][1] = racc[mt][2] = racc[mt][3] = 0.f;
                 }
 #pragma unroll
                 for (int e = 0; e < 2; ++e) { e_carry[e] = 0.f; dot_carry[e] = 0.f; }
+                if (meta.flags & STG_HEAD) {
+                    // a group entered midway has its own record (its scores
+                    // lack the dot of the state before it, which the merge
+                    // adds); the sequence's record starts afresh
+                    write_record(A.heads + gw * PARTIAL_FLOATS);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) { m_run[e] = -1e30f; l_run[e] = 0.f; }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
+                }
             }
         }
 
@@ -1295,9 +1384,11 @@ __device__ inline int merge_len(const CacheView &cv, const int32_t *lenv, int b)
     else return clamp_len(cv, b);
 }
 
-template <bool FIN>
+// SEGS (delta format, kf > 32): unit ranges may start and end inside a
+// keyframe group (below); wfl holds one flag byte per warp of the sequence.
+template <bool FIN, bool SEGS>
 __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, int nq, int64_t NW,
-                                  const float *ws, float *out) {
+                                  const float *ws, float *out, uint8_t *wfl) {
     const int t = blockIdx.x / Hq, h = blockIdx.x % Hq, b = blockIdx.y, c = threadIdx.x;
     const int nvs = cv.Hkv * NHG;
     const int32_t *lenv = FIN ? merge_lengths(const_cast<float *>(ws), NW, cv.B * nvs) : nullptr;
@@ -1311,7 +1402,7 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
     const int kvh = h / G, vh = t * G + h % G, hg = vh >> 3, j = vh & 7;
     const int vsl = kvh * NHG + hg;
     // the warps whose unit ranges touch this sequence: found once per block
-    __shared__ int64_t sh_w0, sh_w1, sh_total;
+    __shared__ int64_t sh_w0, sh_w1, sh_total, sh_xs;
     if (threadIdx.x < 32) {
         // units of all batch entries, and of those before b
         int64_t total = 0, mine = 0;
@@ -1333,11 +1424,12 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
             sh_w0 = warp_of(xs, NW, total);
             sh_w1 = warp_of(xe - 1, NW, total);
             sh_total = total;
+            sh_xs = xs;
         }
     }
     __syncthreads();
     const int64_t vseq = (int64_t)b * nvs + vsl;
-    const int64_t T = sh_total, w0 = sh_w0, w1 = sh_w1;
+    const int64_t T = sh_total, w0 = sh_w0, w1 = sh_w1, xs = sh_xs, xe = xs + ub;
     // with at least one unit per warp every range is non-empty; otherwise
     // skip the warps that own no unit (they wrote no record)
     const bool dense = T >= NW;
@@ -1349,21 +1441,89 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
     };
     // one pass, rescaling online: each batch of 8 records moves the running
     // maximum once (records of warps that saw no position carry -1e30)
+    // SEGS: ranges may start and end inside a keyframe group.  A warp that
+    // entered a group midway wrote that part as a separate record with scores
+    // and value rows relative to the state before its first position; the
+    // warp before it handed that state on (absolute, or relative to its own
+    // entry state when it too entered the group midway).  Walking the warps
+    // in order, the state is carried and each such record made absolute:
+    //   m += scaled dot of the state,  o += l * value row of the state.
+    // Which warps do what follows from the ranges alone; the flags are worked
+    // out once per block, one warp per thread.
+    constexpr uint8_t W_ANY = 1, W_HEAD = 2, W_HAND = 4, W_REL = 8;
+    const float *heads = nullptr, *hands = nullptr;
+    float sl2 = 0.f;
+    if constexpr (SEGS) {
+        const int spg = seg_per_group(cv.kf);
+        for (int64_t k = threadIdx.x; k <= w1 - w0; k += blockDim.x) {
+            const int64_t rs = range_start(w0 + k, NW, T), re = range_start(w0 + k + 1, NW, T);
+            uint8_t f = 0;
+            if (rs < re) {
+                f = W_ANY;
+                if (rs > xs && (rs - xs) % spg != 0) f |= W_HEAD;
+                if (re > xs && re < xe && (re - xs) % spg != 0) f |= W_HAND;
+                if ((f & (W_HEAD | W_HAND)) == (W_HEAD | W_HAND) &&
+                    (rs - xs) / spg == (re - 1 - xs) / spg)
+                    f |= W_REL;
+            }
+            wfl[k] = f;
+        }
+        __syncthreads();
+        heads = head_records(const_cast<float *>(ws), NW, (int64_t)cv.B * nvs, cv.B);
+        hands = handoffs(const_cast<float *>(ws), NW, (int64_t)cv.B * nvs, cv.B);
+        sl2 = hands[0];                 // the log2 softmax scale the split kernel used
+        hands += HAND_HDR;
+    }
+    float cdot = 0.f, cval = 0.f;       // the carried state: head j's scaled dot, value c
     float M = -1e30f, L = 0.f, O = 0.f;
     for (int64_t w = w0; w <= w1; w += BATCH) {
         float mv[BATCH], lv[BATCH], ov[BATCH];
+        float hm[BATCH], hl[BATCH], ho[BATCH], hdot[BATCH], hval[BATCH];
+        uint8_t fl[BATCH];
         bool ok[BATCH];
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
-            ok[i] = has(w + i);
+            if constexpr (SEGS) {
+                fl[i] = w + i <= w1 ? wfl[w + i - w0] : 0;
+                ok[i] = fl[i] & W_ANY;
+            } else {
+                ok[i] = has(w + i);
+            }
             const float *rec = ws + (w + i + vseq) * PARTIAL_FLOATS;
             mv[i] = ok[i] ? rec[j] : -1e30f;
             lv[i] = ok[i] ? rec[8 + j] : 0.f;
             ov[i] = ok[i] ? rec[16 + j * 128 + c] : 0.f;
+            if constexpr (SEGS) {
+                const bool hd = fl[i] & W_HEAD, tl = fl[i] & W_HAND;
+                const float *hr = heads + (w + i) * PARTIAL_FLOATS;
+                const float *hh = hands + (w + i) * HANDOFF_FLOATS;
+                hm[i] = hd ? hr[j] : -1e30f;
+                hl[i] = hd ? hr[8 + j] : 0.f;
+                ho[i] = hd ? hr[16 + j * 128 + c] : 0.f;
+                hdot[i] = tl ? hh[j] * sl2 : 0.f;
+                hval[i] = tl ? hh[8 + c] : 0.f;
+            }
+        }
+        if constexpr (SEGS) {
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                if (fl[i] & W_HEAD) {
+                    hm[i] += cdot;
+                    ho[i] = fmaf(hl[i], cval, ho[i]);
+                }
+                if (fl[i] & W_HAND) {
+                    const bool rel = fl[i] & W_REL;
+                    cdot = rel ? cdot + hdot[i] : hdot[i];
+                    cval = rel ? cval + hval[i] : hval[i];
+                }
+            }
         }
         float Mn = M;
 #pragma unroll
-        for (int i = 0; i < BATCH; ++i) Mn = fmaxf(Mn, mv[i]);
+        for (int i = 0; i < BATCH; ++i) {
+            Mn = fmaxf(Mn, mv[i]);
+            if constexpr (SEGS) Mn = fmaxf(Mn, hm[i]);
+        }
         const float sc = exp2f(M - Mn);
         L *= sc;
         O *= sc;
@@ -1372,16 +1532,22 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
             const float e = exp2f(mv[i] - Mn);
             L = fmaf(lv[i], e, L);
             O = fmaf(ov[i], e, O);
+            if constexpr (SEGS) {
+                const float eh = exp2f(hm[i] - Mn);
+                L = fmaf(hl[i], eh, L);
+                O = fmaf(ho[i], eh, O);
+            }
         }
         M = Mn;
     }
     dst[c] = L > 0.f ? O / L : 0.f;     // a causal query with no position gets 0
 }
 
-template <bool FIN>
+template <bool FIN, bool SEGS>
 __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G, int NHG, int nq,
                                                     int64_t NW, const float *ws, float *out) {
-    merge_body<FIN>(cv, Hq, G, NHG, nq, NW, ws, out);
+    extern __shared__ uint8_t merge_flags[];        // SEGS: one byte per warp slot
+    merge_body<FIN, SEGS>(cv, Hq, G, NHG, nq, NW, ws, out, merge_flags);
     if constexpr (FIN) {
         // fused append: publish batch entry b's new length (no other block of
         // this launch reads it) and make the state slot the split kernel
@@ -1519,7 +1685,13 @@ static cudaError_t launch_split_t(const SplitArgs &a_in, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     clamp_geometry(&g, split_max_units(a_in.cv.fmt, a_in.cv.kf, a_in.cv.B, a_in.cv.Hkv, a_in.NHG,
                                        a_in.cv.cap));
-    const SplitArgs &a = a_in;
+    SplitArgs a = a_in;
+    {
+        const int64_t NW = (int64_t)g.ctas * g.warps_per_cta;
+        const int64_t nseq = (int64_t)a.cv.B * a.cv.Hkv * a.NHG;
+        a.heads = head_records(a.ws, NW, nseq, a.cv.B);
+        a.hands = handoffs(a.ws, NW, nseq, a.cv.B);
+    }
     const bool paged = a.cv.pg != 0, mq = a.nq > 1, app = a.cv.len_add > 0;
     if (!paged && !mq && !app) return launch_q<FMT, MODE, ZT, false, false, false>(a, g.ctas, st);
     if constexpr (FMT == DKV_FMT_DELTA) {        // only the delta format pages / takes queries
@@ -1582,10 +1754,19 @@ cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const 
     if (e != cudaSuccess) return e;
     dim3 grid(nq * Hq, cv.B);
     const int64_t NW = (int64_t)g.ctas * g.warps_per_cta;
-    if (cv.len_add > 0)
-        merge_kernel<true><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
-    else
-        merge_kernel<false><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+    if (cv.fmt == DKV_FMT_DELTA && cv.kf > SEG) {
+        // a flag byte for each warp slot a sequence can span
+        const size_t fl = (size_t)(NW + 15) / 16 * 16;
+        if (fl > 48 * 1024) return cudaErrorInvalidConfiguration;
+        if (cv.len_add > 0)
+            merge_kernel<true, true><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+        else
+            merge_kernel<false, true><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+    } else if (cv.len_add > 0) {
+        merge_kernel<true, false><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+    } else {
+        merge_kernel<false, false><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+    }
     return cudaGetLastError();
 }
 

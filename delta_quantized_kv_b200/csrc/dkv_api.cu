@@ -133,10 +133,16 @@ int64_t workspace_floats(const dkv_cache_desc *d, int32_t Hq, int32_t nq, bool *
                                                  d->max_ctx),
                             &g) != cudaSuccess)
         return 0;
-    const int64_t slots = (int64_t)g.ctas * g.warps_per_cta + (int64_t)d->batch * d->n_kv_heads * nhg;
+    const int64_t NW = (int64_t)g.ctas * g.warps_per_cta;
+    const int64_t slots = NW + (int64_t)d->batch * d->n_kv_heads * nhg;
     *ok = true;
     // + the decoded lengths of a fused append + decode, int32[B]
-    return slots * dkv::PARTIAL_FLOATS + ((int64_t)d->batch + 3) / 4 * 4;
+    int64_t f = slots * dkv::PARTIAL_FLOATS + ((int64_t)d->batch + 3) / 4 * 4;
+    // kf > 32: + per warp, a record of the group its range enters midway and
+    // the state it hands on
+    if (d->fmt == DKV_FMT_DELTA && d->kf > 32)
+        f += NW * (dkv::PARTIAL_FLOATS + dkv::HANDOFF_FLOATS) + dkv::HAND_HDR;
+    return f;
 }
 
 dkv_status check_decode(const dkv_cache *cache, const void *Q, int32_t q_dtype, int32_t Hq,

@@ -36,6 +36,10 @@ int64_t split_max_units(int fmt, int kf, int B, int Hkv, int nhg, int cap);
 
 // Floats per partial record: m[8], l[8], o[8][128].
 constexpr int PARTIAL_FLOATS = 8 + 8 + 8 * 128;
+// Floats per state handed from warp to warp inside a keyframe group (kf > 32):
+// the scaled query-key dot of 8 heads and one reconstructed value row.
+constexpr int HANDOFF_FLOATS = 8 + 128;
+constexpr int HAND_HDR = 4;    // floats before the handoffs: the log2 softmax scale, padding
 
 // nq queries per sequence: query t attends to the positions before
 // seq_len - (nq - 1 - t); Q and out are [B][nq][Hq][D].  With cv.len_add = n
