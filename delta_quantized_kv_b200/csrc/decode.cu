@@ -56,6 +56,12 @@ constexpr int WARPS = DKV_WARPS;             // warps per CTA (independent pipel
 // Two groups per stage and one stage per warp (a warp's next stage is copied
 // while the other warps of the SM compute) measured fastest on B200: the
 // shared memory this frees buys a third CTA per SM.
+#ifndef DKV_PFX_NU
+#define DKV_PFX_NU 2             // kf > 32: consecutive segments of one group per stage
+#endif
+#ifndef DKV_PFX_MINB
+#define DKV_PFX_MINB 3           // kf > 32: CTAs per SM the registers are sized for
+#endif
 #ifndef DKV_NIB_NU
 #define DKV_NIB_NU 2
 #endif
@@ -71,10 +77,10 @@ constexpr int WARPS = DKV_WARPS;             // warps per CTA (independent pipel
 // a group (delta, kf > 32), or one 32-position chunk (Q4_0, fp16).
 template <int FMT, int MODE> struct KCfg {
     static constexpr bool NIB = FMT != DKV_FMT_FP16 && MODE != PREFIX;
-    static constexpr int NU = NIB ? DKV_NIB_NU : 1;
+    static constexpr int NU = NIB ? DKV_NIB_NU : (MODE == PREFIX ? DKV_PFX_NU : 1);
     static constexpr int STAGE = FMT == DKV_FMT_FP16 ? 16384 : NU * 5120;
-    static constexpr int NS = NIB ? DKV_NIB_NS : 2;
-    static constexpr int MINB = FMT == DKV_FMT_FP16 ? 1 : (MODE == PREFIX ? 3 : DKV_NIB_MINB);
+    static constexpr int NS = NIB ? DKV_NIB_NS : (MODE == PREFIX && NU == 2 ? 1 : 2);
+    static constexpr int MINB = FMT == DKV_FMT_FP16 ? 1 : (MODE == PREFIX ? DKV_PFX_MINB : DKV_NIB_MINB);
 };
 
 // Shared-memory map of the split kernel: [mbarriers WARPS*NS x 8 B]
@@ -311,8 +317,8 @@ __device__ inline int unit_npos(const CacheView &cv, const Cursor &c, int g) {
 //  DELTA, kf <= 32: NU consecutive group records copied as one run, record u
 //      at u * rec: [K kf 256][V kf 256][scales (kf-1)x16][K nib (kf-1)x64]
 //      [V nib (kf-1)x64];
-//  DELTA, kf > 32 (NU = 1, one 32-position segment):
-//      [K kf 256][V kf 256][scales 32x16][K nib 32x64][V nib 32x64];
+//  DELTA, kf > 32 (NU consecutive 32-position segments of one group):
+//      [K kf 256][V kf 256][scales NU*32 x16][K nib NU*32 x64][V nib NU*32 x64];
 //  Q4_0 (NU chunks of 32 positions): [scales NU x 512][K nib NU x 2048]
 //      [V nib NU x 2048];
 //  FP16 (NU = 1): [K 32x256][V 32x256].
@@ -332,6 +338,12 @@ __device__ inline StageMap stage_map(int kf, int64_t rec, int u) {
         m.kn0 = base + KF_BYTES + (kf - 1) * SC_BYTES - NIB_BYTES;
         m.vk0 = base + 256;
         m.vn0 = base + KF_BYTES + (kf - 1) * (SC_BYTES + NIB_BYTES) - NIB_BYTES;
+    } else if (FMT == DKV_FMT_DELTA) {
+        m.kf0 = 0;
+        m.vk0 = 256;
+        m.sc0 = 512 + 512 * u;
+        m.kn0 = 512 + 512 * NU + 2048 * u;
+        m.vn0 = 512 + 2560 * NU + 2048 * u;
     } else if (FMT == DKV_FMT_Q4_0) {
         m.kf0 = 0;
         m.sc0 = 512 * u;
@@ -387,10 +399,10 @@ __device__ inline void issue_stage(const CacheView &cv, Cursor &c, int nhg, int 
         mbar_arrive_expect_tx(bar, bytes);
         bulk_g2s(stage, rec, bytes, bar);
     } else if (FMT == DKV_FMT_DELTA) {
+        // nu consecutive segments of group c.g from segment c.seg on
         const int kf = cv.kf;
-        const int glen = min(kf, c.len_b - c.g * kf);
         const int a = c.seg * SEG;
-        const int npos = min(SEG, glen - a);
+        const int npos = npos_all;
         const uint8_t *rec = stage_rec<PAGED>(cv, c, nhg);
         if (!rec) {
             mbar_arrive_expect_tx(bar, 0);
@@ -407,10 +419,12 @@ __device__ inline void issue_stage(const CacheView &cv, Cursor &c, int nhg, int 
         mbar_arrive_expect_tx(bar, bytes);
         if (a == 0) bulk_g2s(stage, rec, KF_BYTES, bar);
         if (nd > 0) {
-            bulk_g2s(stage + 512 + s0 * SC_BYTES, scs + (int64_t)di0 * SC_BYTES, nd * SC_BYTES, bar);
-            bulk_g2s(stage + 1024 + s0 * NIB_BYTES, kns + (int64_t)di0 * NIB_BYTES,
+            const StageMap sm = stage_map<FMT, MODE>(kf, cv.rec_bytes, 0);
+            bulk_g2s(stage + sm.sc0 + s0 * SC_BYTES, scs + (int64_t)di0 * SC_BYTES, nd * SC_BYTES,
+                     bar);
+            bulk_g2s(stage + sm.kn0 + s0 * NIB_BYTES, kns + (int64_t)di0 * NIB_BYTES,
                      nd * NIB_BYTES, bar);
-            bulk_g2s(stage + 3072 + s0 * NIB_BYTES, vns + (int64_t)di0 * NIB_BYTES,
+            bulk_g2s(stage + sm.vn0 + s0 * NIB_BYTES, vns + (int64_t)di0 * NIB_BYTES,
                      nd * NIB_BYTES, bar);
         }
     } else if (FMT == DKV_FMT_Q4_0) {
@@ -441,8 +455,15 @@ __device__ inline StageMeta next_stage(const CacheView &cv, Cursor &c, int nvs, 
     constexpr int NU = KCfg<FMT, MODE>::NU;
     const int np0 = unit_npos(cv, c, c.g);
     int nu = 1, np1 = 0;
-    // two consecutive groups per stage, never across a page boundary
-    if (NU == 2 && c.left >= 2 && c.g + 1 < c.units_b && (!PAGED || (c.g + 1) % cv.pg != 0)) {
+    if (MODE == PREFIX) {
+        // two consecutive segments of one group per stage
+        if (NU == 2 && c.left >= 2 && c.seg + 1 < c.nseg) {
+            nu = 2;
+            np1 = min(SEG, min(cv.kf, c.len_b - c.g * cv.kf) - (c.seg + 1) * SEG);
+        }
+    } else if (NU == 2 && c.left >= 2 && c.g + 1 < c.units_b &&
+               (!PAGED || (c.g + 1) % cv.pg != 0)) {
+        // two consecutive groups per stage, never across a page boundary
         nu = 2;
         np1 = unit_npos(cv, c, c.g + 1);
     }
@@ -451,7 +472,8 @@ __device__ inline StageMeta next_stage(const CacheView &cv, Cursor &c, int nvs, 
     m.vs = c.vs;
     m.npos = np0 | (np1 << 8);
     if (MODE == PREFIX) {
-        const bool group_end = c.seg == c.nseg - 1, range_end = c.left == 1;
+        // the stage's last segment ends the group, or the range
+        const bool group_end = c.seg + nu == c.nseg, range_end = c.left == nu;
         m.flags = (c.seg == 0 ? STG_FIRST : 0) | (group_end || range_end ? STG_CLOSE : 0) |
                   (c.head ? STG_HEAD : 0) | (range_end && !group_end ? STG_HAND : 0);
     } else {
@@ -1193,8 +1215,9 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
-                k_side<FMT, MODE, ZT, QHL>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, qb,
-                                           ql, x[u]);
+                // kf > 32: only a stage's first segment can hold a keyframe
+                k_side<FMT, MODE, ZT, QHL>(st, sm, npos[u], first_seg && (MODE != PREFIX || u == 0),
+                                           gq, tq, m1024, m64, qb, ql, x[u]);
             }
 
             // ================= scores, online softmax =======================
@@ -1204,7 +1227,7 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 if (MQ) {
-                    const int us = meta.pos0 + u * (FMT == DKV_FMT_DELTA ? cv.kf : SEG);
+                    const int us = meta.pos0 + u * (MODE == SUFFIX ? cv.kf : SEG);
 #pragma unroll
                     for (int e = 0; e < 2; ++e) lim[u][e] = min(npos[u], lp[e] - us) - 4 * gq;
                 } else {
@@ -1261,6 +1284,7 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
                     }
                 l_run[e] = l_run[e] * alpha[e] + psum;
                 // weights that multiply each position's dequantised row
+                if (MODE == PREFIX) e_carry[e] *= alpha[e];
 #pragma unroll
                 for (int u = 0; u < NU; ++u) {
                     float wv[4];
@@ -1270,7 +1294,6 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
 #pragma unroll
                         for (int i = 0; i < 4; ++i) wv[i] = tot - pin[i] + v[u][i];
                     } else if (MODE == PREFIX) {
-                        e_carry[e] *= alpha[e];
                         float pin[4] = {v[u][0], v[u][1], v[u][2], v[u][3]};
                         const float tot = col_scan32(pin, lane);
 #pragma unroll
@@ -1299,8 +1322,8 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
-                v_side<FMT, MODE, ZT>(st, sm, npos[u], first_seg, gq, tq, m1024, m64, x[u], o,
-                                  racc, vkf_keep);
+                v_side<FMT, MODE, ZT>(st, sm, npos[u], first_seg && (MODE != PREFIX || u == 0), gq,
+                                      tq, m1024, m64, x[u], o, racc, vkf_keep);
             }
 
             // PREFIX: close the group (or this range's part of it)
