@@ -634,7 +634,7 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
 // V side of one unit: o += sum over positions of dequantised V rows times the
 // weights w[t][r][e] (position 4g + 2t + r, head 2tq + e) and their V scales.
 // The V scales are read here rather than kept from the K side (registers).
-template <int FMT, int MODE, bool ZT>
+template <int FMT, int MODE, bool ZT, bool RC>
 __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, bool first_seg,
                               int gq, int tq, uint32_t m1024, uint32_t m64,
                               const float (&w)[2][2][2], float (&o)[8][4], float (&racc)[8][4],
@@ -796,14 +796,44 @@ __device__ inline void v_side(const uint8_t *st, const StageMap &sm, int npos, b
                 rr[1] = movm_t(h2_as_u32(d1));
             };
             uint32_t bp[2], bl[2], rr[2];
+            if constexpr (RC) {
+                // columns 4-7 (threads tq >= 2 before the transpose): the V
+                // scale itself in the hi operand and 0 in the lo one, so those
+                // accumulator columns sum the dequantised deltas
+                const bool rcol = tq >= 2;
+                auto make_b_rc = [&](int j, uint32_t (&b)[2], uint32_t (&bl)[2]) {
+                    const uint32_t u0 = dvw[0][j >> 1], u1 = dvw[1][j >> 1];
+                    const __half2 d0 = (j & 1) ? __high2half2(u32_as_h2(u0)) : __low2half2(u32_as_h2(u0));
+                    const __half2 d1 = (j & 1) ? __high2half2(u32_as_h2(u1)) : __low2half2(u32_as_h2(u1));
+                    const __half2 h0 = __hmul2(u32_as_h2(wp0), d0);
+                    const __half2 h1 = __hmul2(u32_as_h2(wp1), d1);
+                    const __half2 l0 = __hfma2(u32_as_h2(wl0), d0,
+                                               __hfma2(u32_as_h2(wp0), d0, __hneg2(h0)));
+                    const __half2 l1 = __hfma2(u32_as_h2(wl1), d1,
+                                               __hfma2(u32_as_h2(wp1), d1, __hneg2(h1)));
+                    b[0] = movm_t(h2_as_u32(rcol ? d0 : h0));
+                    b[1] = movm_t(h2_as_u32(rcol ? d1 : h1));
+                    bl[0] = movm_t(rcol ? 0u : h2_as_u32(l0));
+                    bl[1] = movm_t(rcol ? 0u : h2_as_u32(l1));
+                };
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                uint32_t a0, a1, a2, a3;
-                codes(mt, a0, a1, a2, a3);
-                if ((mt & 1) == 0) make_b(mt >> 1, bp, bl, rr);
-                mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
-                mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
-                mma16816(racc[mt], a0, a1, a2, a3, rr[0], rr[1]);   // R += (code - 8) d
+                for (int mt = 0; mt < 8; ++mt) {
+                    uint32_t a0, a1, a2, a3;
+                    codes(mt, a0, a1, a2, a3);
+                    if ((mt & 1) == 0) make_b_rc(mt >> 1, bp, bl);
+                    mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
+                    mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
+                }
+            } else {
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    uint32_t a0, a1, a2, a3;
+                    codes(mt, a0, a1, a2, a3);
+                    if ((mt & 1) == 0) make_b(mt >> 1, bp, bl, rr);
+                    mma16816(o[mt], a0, a1, a2, a3, bp[0], bp[1]);
+                    mma16816(o[mt], a0, a1, a2, a3, bl[0], bl[1]);
+                    mma16816(racc[mt], a0, a1, a2, a3, rr[0], rr[1]);   // R += (code - 8) d
+                }
             }
         }
     }
@@ -983,7 +1013,10 @@ __device__ __noinline__ bool append_range(const SplitArgs &A, int nvs, int b, in
 // the fused append (the kernel parameters stay in the constant bank while the
 // append functions take their address).  QHL: fp32 queries as an fp16 hi + lo
 // pair (two MMAs per K-side step; the extra registers cost a CTA per SM).
-template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP, bool QHL>
+// RC (kf > 32, at most 4 heads per head group): the group's sum of dequantised
+// V deltas R_g accumulates in the output accumulators' columns 4-7, which no
+// head uses (their B operand is the V scale), instead of 32 registers of its own.
+template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP, bool QHL, bool RC = false>
 __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
     split_kernel(const __grid_constant__ SplitArgs A) {
     using Cfg = KCfg<FMT, MODE>;
@@ -1322,7 +1355,7 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
-                v_side<FMT, MODE, ZT>(st, sm, npos[u], first_seg && (MODE != PREFIX || u == 0), gq,
+                v_side<FMT, MODE, ZT, RC>(st, sm, npos[u], first_seg && (MODE != PREFIX || u == 0), gq,
                                       tq, m1024, m64, x[u], o, racc, vkf_keep);
             }
 
@@ -1341,8 +1374,12 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
                 }
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
-                    const float v_lo = h_lo(vkf_keep[mt]) + racc[mt][0];   // channel 16mt+g
-                    const float v_hi = h_hi(vkf_keep[mt]) + racc[mt][2];   // channel 16mt+g+8
+                    // RC: R_g of these channels is in the partner thread's
+                    // columns 4-7 (lane ^ 2); threads tq >= 2 add e_carry 0
+                    const float r_lo = RC ? __shfl_xor_sync(0xffffffffu, o[mt][0], 2) : racc[mt][0];
+                    const float r_hi = RC ? __shfl_xor_sync(0xffffffffu, o[mt][2], 2) : racc[mt][2];
+                    const float v_lo = h_lo(vkf_keep[mt]) + r_lo;   // channel 16mt+g
+                    const float v_hi = h_hi(vkf_keep[mt]) + r_hi;   // channel 16mt+g+8
                     if (hand && tq == 0) {
                         hd[8 + 16 * mt + gq] = v_lo;
                         hd[8 + 16 * mt + gq + 8] = v_hi;
@@ -1350,6 +1387,7 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
                     o[mt][0] += e_carry[0] * v_lo; o[mt][1] += e_carry[1] * v_lo;
                     o[mt][2] += e_carry[0] * v_hi; o[mt][3] += e_carry[1] * v_hi;
                     racc[mt][0] = racc[mt][1] = racc[mt][2] = racc[mt][3] = 0.f;
+                    if (RC && tq >= 2) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
                 }
 #pragma unroll
                 for (int e = 0; e < 2; ++e) { e_carry[e] = 0.f; dot_carry[e] = 0.f; }
@@ -1671,9 +1709,9 @@ int64_t split_max_units(int fmt, int kf, int B, int Hkv, int nhg, int cap) {
 // Every instance runs on the contiguous one-query instance's grid (the merge
 // and the workspace size follow that grid); a persistent grid is correct at
 // any size.
-template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP, bool QHL>
+template <int FMT, int MODE, bool ZT, bool PAGED, bool MQ, bool APP, bool QHL, bool RC = false>
 static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
-    if (PAGED || MQ || APP || QHL) {
+    if (PAGED || MQ || APP || QHL || RC) {
         static std::atomic<bool> set_on[kMaxDevices];   // per instance and device
         int dev;
         cudaError_t e = current_device(&dev);
@@ -1681,7 +1719,7 @@ static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
         if (!set_on[dev].load(std::memory_order_acquire)) {
             std::lock_guard<std::mutex> lock(g_launch_mu);
             if (!set_on[dev].load(std::memory_order_relaxed)) {
-                e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, PAGED, MQ, APP, QHL>,
+                e = cudaFuncSetAttribute(split_kernel<FMT, MODE, ZT, PAGED, MQ, APP, QHL, RC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)split_smem<FMT, MODE>());
                 if (e != cudaSuccess) return e;
@@ -1689,7 +1727,7 @@ static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
             }
         }
     }
-    split_kernel<FMT, MODE, ZT, PAGED, MQ, APP, QHL>
+    split_kernel<FMT, MODE, ZT, PAGED, MQ, APP, QHL, RC>
         <<<ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
     return cudaGetLastError();
 }
@@ -1716,7 +1754,13 @@ static cudaError_t launch_split_t(const SplitArgs &a_in, cudaStream_t st) {
         a.hands = handoffs(a.ws, NW, nseq, a.cv.B);
     }
     const bool paged = a.cv.pg != 0, mq = a.nq > 1, app = a.cv.len_add > 0;
-    if (!paged && !mq && !app) return launch_q<FMT, MODE, ZT, false, false, false>(a, g.ctas, st);
+    if (!paged && !mq && !app) {
+        // kf > 32 with at most 4 heads per kv head: R_g in the spare columns
+        if constexpr (FMT == DKV_FMT_DELTA && MODE == PREFIX)
+            if (a.G <= 4 && a.q_dtype != DKV_F32)
+                return launch_inst<FMT, MODE, ZT, false, false, false, false, true>(a, g.ctas, st);
+        return launch_q<FMT, MODE, ZT, false, false, false>(a, g.ctas, st);
+    }
     if constexpr (FMT == DKV_FMT_DELTA) {        // only the delta format pages / takes queries
         if (app) {
             if (paged && mq) return launch_q<FMT, MODE, ZT, true, true, true>(a, g.ctas, st);
