@@ -62,6 +62,9 @@ constexpr int WARPS = DKV_WARPS;             // warps per CTA (independent pipel
 #ifndef DKV_PFX_MINB
 #define DKV_PFX_MINB 3           // kf > 32: CTAs per SM the registers are sized for
 #endif
+#ifndef DKV_QSM
+#define DKV_QSM 1                // q fragments in shared memory (0: registers)
+#endif
 #ifndef DKV_NIB_NU
 #define DKV_NIB_NU 2
 #endif
@@ -91,7 +94,8 @@ template <int FMT, int MODE> struct SmemMap {
     static constexpr int BAR_OFF = 0;
     static constexpr int META_OFF = ((BAR_OFF + 8 * WARPS * NS) + 15) / 16 * 16;
     static constexpr int STAGE_OFF = ((META_OFF + 32 * WARPS * NS) + 127) / 128 * 128;
-    static constexpr int BYTES = STAGE_OFF + WARPS * NS * STAGE;
+    static constexpr int Q_OFF = STAGE_OFF + WARPS * NS * STAGE;       // q fragments (DKV_QSM)
+    static constexpr int BYTES = Q_OFF + (DKV_QSM ? WARPS * 2048 : 0);
     static_assert(META_OFF >= BAR_OFF + 8 * WARPS * NS, "barriers overlap descriptors");
     static_assert(STAGE_OFF >= META_OFF + 32 * WARPS * NS, "descriptors overlap stages");
     static_assert(STAGE % 128 == 0, "stages must stay 128-byte aligned");
@@ -543,8 +547,18 @@ template <int FMT, int MODE, bool ZT, bool QHL>
 __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, bool first_seg,
                               int gq, int tq, uint32_t m1024, uint32_t m64,
                               const uint32_t (&qb)[8][2], const uint32_t (&ql)[8][2],
-                              float (&x)[2][2][2]) {
+                              const uint4 *qs, float (&x)[2][2][2]) {
     const bool kfrow = first_seg && gq == 0;   // this thread's row 0 of tile 0 is the keyframe
+    // B fragments of q for k-steps 2j, 2j + 1: from registers, or (DKV_QSM)
+    // from this lane's slots in shared memory
+    auto qfrag = [&](int j, uint32_t &b0, uint32_t &b1, uint32_t &b2, uint32_t &b3) {
+        if constexpr (DKV_QSM != 0 && !QHL) {
+            const uint4 v = qs[j * 32 + 4 * gq + tq];
+            b0 = v.x; b1 = v.y; b2 = v.z; b3 = v.w;
+        } else {
+            b0 = qb[2 * j][0]; b1 = qb[2 * j][1]; b2 = qb[2 * j + 1][0]; b3 = qb[2 * j + 1][1];
+        }
+    };
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int p0 = 4 * gq + 2 * t;             // positions p0, p0 + 1
@@ -555,8 +569,10 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
             for (int q4 = 0; q4 < 4; ++q4) {
                 const uint4 u0 = *reinterpret_cast<const uint4 *>(k0 + 16 * q4);
                 const uint4 u1 = *reinterpret_cast<const uint4 *>(k0 + 256 + 16 * q4);
-                mma16816(acc, u0.x, u1.x, u0.y, u1.y, qb[2 * q4][0], qb[2 * q4][1]);
-                mma16816(acc, u0.z, u1.z, u0.w, u1.w, qb[2 * q4 + 1][0], qb[2 * q4 + 1][1]);
+                uint32_t b0, b1, b2, b3;
+                qfrag(q4, b0, b1, b2, b3);
+                mma16816(acc, u0.x, u1.x, u0.y, u1.y, b0, b1);
+                mma16816(acc, u0.z, u1.z, u0.w, u1.w, b2, b3);
                 if (QHL) {
                     mma16816(acc, u0.x, u1.x, u0.y, u1.y, ql[2 * q4][0], ql[2 * q4][1]);
                     mma16816(acc, u0.z, u1.z, u0.w, u1.w, ql[2 * q4 + 1][0], ql[2 * q4 + 1][1]);
@@ -596,10 +612,11 @@ __device__ inline void k_side(const uint8_t *st, const StageMap &sm, int npos, b
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-                mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
-                         qb[2 * j][0], qb[2 * j][1]);
+                uint32_t b0, b1, b2, b3;
+                qfrag(j, b0, b1, b2, b3);
+                mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3], b0, b1);
                 mma16816(acc[j], a[2 * j + 1][0], a[2 * j + 1][1], a[2 * j + 1][2],
-                         a[2 * j + 1][3], qb[2 * j + 1][0], qb[2 * j + 1][1]);
+                         a[2 * j + 1][3], b2, b3);
                 if (QHL) {
                     mma16816(acc[j], a[2 * j][0], a[2 * j][1], a[2 * j][2], a[2 * j][3],
                              ql[2 * j][0], ql[2 * j][1]);
@@ -1031,6 +1048,7 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
     uint64_t *mybar = reinterpret_cast<uint64_t *>(smem + Map::BAR_OFF) + warp * NS;
     StageMeta *mymeta = reinterpret_cast<StageMeta *>(smem + Map::META_OFF) + warp * NS;
     uint8_t *mystages = smem + Map::STAGE_OFF + warp * NS * STAGE;
+    uint4 *myq = reinterpret_cast<uint4 *>(smem + Map::Q_OFF) + warp * 128;   // DKV_QSM
     const uint32_t m1024 = magic_1024x2(), m64 = magic_64x2();
 
     if (lane == 0) {
@@ -1215,6 +1233,11 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
                 }
                 qb[kk][0] = pack_h2(q0, q1);
                 qb[kk][1] = pack_h2(q8, q9);
+                if (DKV_QSM != 0 && !QHL && (kk & 1)) {
+                    // this lane's own slots: no other lane reads them
+                    myq[(kk >> 1) * 32 + lane] =
+                        make_uint4(qb[kk - 1][0], qb[kk - 1][1], qb[kk][0], qb[kk][1]);
+                }
                 if (QHL) {
                     // fp32 queries: q = hi + lo, both fp16, so q . k keeps
                     // about 22 bits (bf16 and fp16 queries are exact in hi)
@@ -1250,7 +1273,7 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
                 const StageMap sm = stage_map<FMT, MODE>(cv.kf, cv.rec_bytes, u);
                 // kf > 32: only a stage's first segment can hold a keyframe
                 k_side<FMT, MODE, ZT, QHL>(st, sm, npos[u], first_seg && (MODE != PREFIX || u == 0),
-                                           gq, tq, m1024, m64, qb, ql, x[u]);
+                                           gq, tq, m1024, m64, qb, ql, myq, x[u]);
             }
 
             // ================= scores, online softmax =======================
