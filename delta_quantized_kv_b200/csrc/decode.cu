@@ -65,6 +65,9 @@ constexpr int WARPS = DKV_WARPS;             // warps per CTA (independent pipel
 #ifndef DKV_QSM
 #define DKV_QSM 1                // q fragments in shared memory (0: registers)
 #endif
+#ifndef DKV_MERGE_BATCH
+#define DKV_MERGE_BATCH 16       // partial records the merge loads per round trip
+#endif
 #ifndef DKV_NIB_NU
 #define DKV_NIB_NU 2
 #endif
@@ -1519,7 +1522,7 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
     const bool dense = T >= NW;
     // the records are read in batches of 8 independent loads (one memory
     // round trip per batch); the arithmetic runs over w in order, as written
-    constexpr int BATCH = 8;
+    constexpr int BATCH = DKV_MERGE_BATCH;
     auto has = [&](int64_t w) {
         return w <= w1 && (dense || range_start(w, NW, T) < range_start(w + 1, NW, T));
     };
