@@ -218,28 +218,34 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Delta format.  One lane per closed loop: a lane owns one 32-channel block of
-// one tensor of one keyframe group of one (batch entry, kv head) and runs the
-// group's positions in order with the whole block in its registers, so the
-// block rule needs no warp-wide step (the signed element of largest
-// magnitude is a scan in channel order with a strict comparison, which keeps
-// the lowest index on ties, as the rule states).  Lane l of a warp takes
-// block l & 3 of tensor (l >> 2) & 1 of group 4 q + (l >> 3), q the warp's
-// group quad.  The next position's 64 input bytes are loaded before the
-// current position is quantised.  Every quantiser step is one IEEE binary32
-// operation in the order of quant_lane.
+// Delta format.  LPC lanes per closed loop (1 or 2): the lanes of a loop own
+// one 32-channel block of one tensor of one keyframe group of one (batch
+// entry, kv head), lane u of them channels 32/LPC u .. 32/LPC (u + 1) - 1,
+// and run the group's positions in order with their channels in registers.
+// The block rule's signed element of largest magnitude is a scan in channel
+// order with a strict comparison, which keeps the lowest index on ties, as
+// the rule states: a pairwise tree inside the lane, then (LPC 2) the same
+// comparison between the two halves, lower channels on the left.  Lane l of
+// a warp takes part l % LPC of block (l / LPC) & 3 of tensor (l / 4 LPC) & 1
+// of group (4 / LPC) q + l / 8 LPC, q the warp's group chunk.  The next
+// position's inputs are loaded before the current position is quantised.
+// Every quantiser step is one IEEE binary32 operation in the order of
+// quant_lane.  Two lanes per loop serve caches with few loops per GPU (long
+// keyframe groups, small batches).
 // ---------------------------------------------------------------------------
 constexpr int ENC_WARPS = 4;
 // Closed loops (group x tensor x block) from which an append uses the
 // one-lane-per-loop kernel: about two resident waves of its lanes on 148
-// SMs.  Encodes always use it.
+// SMs.  Encodes always use this kernel, with two lanes per loop below one
+// resident wave of loops.
 constexpr int64_t kLaneKernelMinChains = 148 * 12 * 32 * 2;
+constexpr int64_t kOneLanePerLoopMinChains = 148 * 12 * 32;
 
-// The 32 inputs of one block at one position, as raw words (fp32: 32 words;
-// fp16 / bf16: 16 words of two halves).
-template <int DT>
+// CH consecutive inputs of one block at one position, as raw words (fp32: CH
+// words; fp16 / bf16: CH / 2 words of two halves).
+template <int DT, int CH>
 struct EncRow {
-    static constexpr int NW = DT == DKV_F32 ? 32 : 16;
+    static constexpr int NW = DT == DKV_F32 ? CH : CH / 2;
     uint32_t w[NW];
     __device__ inline void load(const void *src, int64_t elem) {
         const uint4 *p = reinterpret_cast<const uint4 *>(
@@ -259,8 +265,11 @@ struct EncRow {
     }
 };
 
-template <int DT>
+template <int DT, int LPC>
 __global__ void __launch_bounds__(ENC_WARPS * 32) encode_delta_kernel(EncodeArgs a, int NQ) {
+    static_assert(LPC == 1 || LPC == 2, "one or two lanes per closed loop");
+    constexpr int CH = 32 / LPC;              // channels per lane
+    constexpr int GW = 4 / LPC;               // groups per warp
     const CacheView &cv = a.cv;
     const int lane = threadIdx.x & 31;
     const int64_t item = (int64_t)blockIdx.x * ENC_WARPS + (threadIdx.x >> 5);
@@ -269,12 +278,15 @@ __global__ void __launch_bounds__(ENC_WARPS * 32) encode_delta_kernel(EncodeArgs
         const int qd = (int)(item % NQ);
         const int bh = (int)(item / NQ);
         const int b = bh / cv.Hkv, kvh = bh % cv.Hkv;
-        const int gi = 4 * qd + (lane >> 3), t = (lane >> 2) & 1, j = lane & 3;
+        const int u = lane % LPC, j = (lane / LPC) & 3, t = (lane / (4 * LPC)) & 1;
+        const int gi = GW * qd + lane / (8 * LPC);
+        // the lanes of one loop, for their exchanges (LPC 2)
+        const unsigned pair = LPC == 2 ? 3u << (lane & ~1) : 1u << lane;
         int start, n;
         encode_range(a, b, start, n);
         const int parity = cv.header[2] & 1;
         const int64_t slot = (int64_t)cv.B * cv.Hkv * 2 * D;
-        const int64_t sb = (((int64_t)b * cv.Hkv + kvh) * 2 + t) * D + 32 * j;
+        const int64_t sb = (((int64_t)b * cv.Hkv + kvh) * 2 + t) * D + 32 * j + CH * u;
         const float *st_old = cv.state + parity * slot + sb;
         float *st_new = cv.state + (parity ^ 1) * slot + sb;
         if (n < 0 && qd == 0 && kvh == 0 && lane == 0)
@@ -282,7 +294,7 @@ __global__ void __launch_bounds__(ENC_WARPS * 32) encode_delta_kernel(EncodeArgs
         if (n <= 0) {
             if (gi == 0) {                         // nothing written: carry the state over
 #pragma unroll
-                for (int c = 0; c < 32; ++c) st_new[c] = a.append ? st_old[c] : 0.0f;
+                for (int c = 0; c < CH; ++c) st_new[c] = a.append ? st_old[c] : 0.0f;
             }
         } else {
             const int g = start / kf + gi;
@@ -293,18 +305,19 @@ __global__ void __launch_bounds__(ENC_WARPS * 32) encode_delta_kernel(EncodeArgs
                 // bad block-table entry (flagged by rec_ptr): nothing written
                 if (last) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) st_new[c] = (p0 % kf) ? st_old[c] : 0.0f;
+                    for (int c = 0; c < CH; ++c) st_new[c] = (p0 % kf) ? st_old[c] : 0.0f;
                 }
             } else if (p0 < p1) {
                 const void *src = t ? a.V : a.K;
-                const int64_t base = (((int64_t)b * cv.Hkv + kvh) * a.T_in - start) * D + 32 * j;
-                float xh[32];
+                const int64_t base =
+                    (((int64_t)b * cv.Hkv + kvh) * a.T_in - start) * D + 32 * j + CH * u;
+                float xh[CH];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) xh[c] = (p0 % kf) ? st_old[c] : 0.0f;
+                for (int c = 0; c < CH; ++c) xh[c] = (p0 % kf) ? st_old[c] : 0.0f;
                 uint8_t *scl = rec + KF_BYTES + t * 8 + 2 * j;
                 uint8_t *nib = rec + KF_BYTES + (int64_t)(kf - 1) * SC_BYTES +
                                (int64_t)t * (kf - 1) * NIB_BYTES;
-                EncRow<DT> cur, nxt;
+                EncRow<DT, CH> cur, nxt;
                 cur.load(src, base + (int64_t)p0 * D);
 #pragma unroll 1
                 for (int p = p0; p < p1; ++p) {
@@ -312,71 +325,91 @@ __global__ void __launch_bounds__(ENC_WARPS * 32) encode_delta_kernel(EncodeArgs
                     const int di = p - g * kf;      // 0: keyframe; else delta di - 1
                     if (di == 0) {
                         // keyframe: fp16 values at their permuted halfword slots
-                        __half h[32];
+                        __half h[CH];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
+                        for (int c = 0; c < CH; ++c) {
                             h[c] = __float2half_rn(cur.get(c));
                             xh[c] = __half2float(h[c]);
                         }
                         __half *kfr = reinterpret_cast<__half *>(rec + t * 256);
                         if (t == 0) {
-                            // halfword t4 * 32 + 8 j + 4 s + 2 e + hh = channel 16 s + 8 e + 2 t4 + hh
+                            // halfword t4 * 32 + 8 j + 4 s + 2 e + hh = channel 16 s + 8 e + 2 t4 + hh;
+                            // lane u holds the channels with s = u (LPC 2)
 #pragma unroll
                             for (int t4 = 0; t4 < 4; ++t4) {
                                 uint32_t w4[4];
 #pragma unroll
                                 for (int k = 0; k < 4; ++k) {
                                     const int s2 = k >> 1, e = k & 1;
-                                    const int c0 = 16 * s2 + 8 * e + 2 * t4;
+                                    const int c0 = 16 * (LPC == 1 ? s2 : 0) + 8 * e + 2 * t4;
                                     w4[k] = (uint32_t)__half_as_ushort(h[c0]) |
                                             ((uint32_t)__half_as_ushort(h[c0 + 1]) << 16);
                                 }
-                                *reinterpret_cast<uint4 *>(kfr + t4 * 32 + 8 * j) =
-                                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                                if (LPC == 1)
+                                    *reinterpret_cast<uint4 *>(kfr + t4 * 32 + 8 * j) =
+                                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                                else   // halfwords 4 u + 0..3; w4[0..1] hold s = 0 of this lane's view
+                                    *reinterpret_cast<uint2 *>(kfr + t4 * 32 + 8 * j + 4 * u) =
+                                        make_uint2(w4[0], w4[1]);
                             }
                         } else {
-                            // halfword gg * 16 + 4 j + 2 u + e = channel 16 u + gg + 8 e
+                            // halfword gg * 16 + 4 j + 2 v + e = channel 16 v + gg + 8 e;
+                            // lane u holds v = u (LPC 2)
 #pragma unroll
                             for (int gg = 0; gg < 8; ++gg) {
-                                const uint32_t lo = (uint32_t)__half_as_ushort(h[gg]) |
+                                const uint32_t w0 = (uint32_t)__half_as_ushort(h[gg]) |
                                                     ((uint32_t)__half_as_ushort(h[gg + 8]) << 16);
-                                const uint32_t hi = (uint32_t)__half_as_ushort(h[16 + gg]) |
-                                                    ((uint32_t)__half_as_ushort(h[24 + gg]) << 16);
-                                *reinterpret_cast<uint2 *>(kfr + gg * 16 + 4 * j) = make_uint2(lo, hi);
+                                if (LPC == 1) {
+                                    const uint32_t w1 = (uint32_t)__half_as_ushort(h[16 + gg]) |
+                                                        ((uint32_t)__half_as_ushort(h[24 + gg]) << 16);
+                                    *reinterpret_cast<uint2 *>(kfr + gg * 16 + 4 * j) =
+                                        make_uint2(w0, w1);
+                                } else {
+                                    *reinterpret_cast<uint32_t *>(kfr + gg * 16 + 4 * j + 2 * u) = w0;
+                                }
                             }
                         }
                     } else {
-                        float dl[32];
+                        float dl[CH];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) dl[c] = __fsub_rn(cur.get(c), xh[c]);
+                        for (int c = 0; c < CH; ++c) dl[c] = __fsub_rn(cur.get(c), xh[c]);
                         // the signed element of largest magnitude, lowest index on
                         // ties: a pairwise tree that keeps the left (lower-index)
                         // element unless the right one is strictly larger
-                        float ta[16], tm[16];
+                        float ta[CH / 2], tm[CH / 2];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
+                        for (int i = 0; i < CH / 2; ++i) {
                             const float l = fabsf(dl[2 * i]), r = fabsf(dl[2 * i + 1]);
                             const bool right = r > l;
                             ta[i] = right ? r : l;
                             tm[i] = right ? dl[2 * i + 1] : dl[2 * i];
                         }
 #pragma unroll
-                        for (int w = 8; w >= 1; w >>= 1)
+                        for (int w = CH / 4; w >= 1; w >>= 1)
 #pragma unroll
                             for (int i = 0; i < w; ++i) {
                                 const bool right = ta[2 * i + 1] > ta[2 * i];
                                 tm[i] = right ? tm[2 * i + 1] : tm[2 * i];
                                 ta[i] = right ? ta[2 * i + 1] : ta[2 * i];
                             }
-                        const float m = tm[0];
+                        float m = tm[0];
+                        if (LPC == 2) {
+                            // the two halves: the upper channels (lane u = 1)
+                            // win only when strictly larger
+                            const float ao = __shfl_xor_sync(pair, ta[0], 1);
+                            const float mo = __shfl_xor_sync(pair, m, 1);
+                            const float al = u ? ao : ta[0], ml = u ? mo : m;
+                            const float ar = u ? ta[0] : ao, mr = u ? m : mo;
+                            m = ar > al ? mr : ml;
+                        }
                         const __half d16 = __float2half_rn(__fmul_rn(m, -0.125f));
                         const float d = __half2float(d16);
                         const bool z = d == 0.0f;
                         const float dd = z ? 1.0f : d;
                         const float rd = __frcp_rn(dd);      // one reciprocal per block and position
-                        uint32_t code[32];
+                        uint32_t code[CH];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
+                        for (int c = 0; c < CH; ++c) {
                             const int cc =
                                 (int)truncf(__fadd_rn(div_rn_markstein(dl[c], dd, rd), 8.5f));
                             code[c] = z ? 8u : (uint32_t)min(15, max(0, cc));
@@ -384,34 +417,45 @@ __global__ void __launch_bounds__(ENC_WARPS * 32) encode_delta_kernel(EncodeArgs
                         }
                         uint8_t *row = nib + (int64_t)(di - 1) * NIB_BYTES;
                         if (t == 0) {
-                            // word t4 * 4 + j, nibble 4 hh + 2 s + e = channel 16 s + 8 e + 2 t4 + hh
+                            // word t4 * 4 + j, nibble 4 hh + 2 s + e = channel 16 s + 8 e + 2 t4 + hh;
+                            // lane u fills the nibbles with s = u (LPC 2)
 #pragma unroll
                             for (int t4 = 0; t4 < 4; ++t4) {
                                 uint32_t wd = 0;
 #pragma unroll
                                 for (int i = 0; i < 8; ++i) {
                                     const int hh = i >> 2, s2 = (i >> 1) & 1, e = i & 1;
-                                    wd |= code[16 * s2 + 8 * e + 2 * t4 + hh] << (4 * i);
+                                    if (LPC == 1)
+                                        wd |= code[16 * s2 + 8 * e + 2 * t4 + hh] << (4 * i);
+                                    else if (s2 == 0)
+                                        wd |= code[8 * e + 2 * t4 + hh] << (4 * i + 8 * u);
                                 }
-                                reinterpret_cast<uint32_t *>(row)[t4 * 4 + j] = wd;
+                                if (LPC == 2) wd |= __shfl_xor_sync(pair, wd, 1);
+                                if (u == 0) reinterpret_cast<uint32_t *>(row)[t4 * 4 + j] = wd;
                             }
                         } else {
-                            // byte gg * 8 + 2 j + u = channel 16 u + gg (low) | 16 u + gg + 8 (high)
+                            // byte gg * 8 + 2 j + v = channel 16 v + gg (low) | 16 v + gg + 8 (high);
+                            // lane u fills byte v = u (LPC 2)
 #pragma unroll
                             for (int gg = 0; gg < 8; ++gg) {
-                                const uint32_t b0 = code[gg] | (code[gg + 8] << 4);
-                                const uint32_t b1 = code[16 + gg] | (code[24 + gg] << 4);
-                                *reinterpret_cast<uint16_t *>(row + gg * 8 + 2 * j) =
-                                    (uint16_t)(b0 | (b1 << 8));
+                                uint32_t bb = code[gg] | (code[gg + 8] << 4);
+                                if (LPC == 1) {
+                                    bb |= (code[16 + gg] | (code[24 + gg] << 4)) << 8;
+                                } else {
+                                    bb <<= 8 * u;
+                                    bb |= __shfl_xor_sync(pair, bb, 1);
+                                }
+                                if (u == 0)
+                                    *reinterpret_cast<uint16_t *>(row + gg * 8 + 2 * j) = (uint16_t)bb;
                             }
                         }
-                        *reinterpret_cast<__half *>(scl + (int64_t)(di - 1) * SC_BYTES) = d16;
+                        if (u == 0) *reinterpret_cast<__half *>(scl + (int64_t)(di - 1) * SC_BYTES) = d16;
                     }
                     if (p + 1 < p1) cur = nxt;
                 }
                 if (last) {
 #pragma unroll
-                    for (int c = 0; c < 32; c += 4)
+                    for (int c = 0; c < CH; c += 4)
                         *reinterpret_cast<float4 *>(st_new + c) =
                             make_float4(xh[c], xh[c + 1], xh[c + 2], xh[c + 3]);
                 }
@@ -574,17 +618,25 @@ cudaError_t launch_encode(const CacheView &cv, const void *K, const void *V, int
     if (cv.fmt == DKV_FMT_DELTA &&
         (!append || (int64_t)cv.B * cv.Hkv * NG * 8 >= kLaneKernelMinChains)) {
         // an encode, or an append with enough closed loops to fill the GPU one
-        // lane each; four groups per warp
-        const int NQ = (NG + 3) / 4;
+        // lane each; an encode with fewer than a resident wave of loops takes
+        // two lanes per loop.  4 / LPC groups per warp.
+        const int64_t chains = (int64_t)cv.B * cv.Hkv * NG * 8;
+        const int lpc = (!append && chains < kOneLanePerLoopMinChains) ? 2 : 1;
+        const int GW = 4 / lpc;
+        const int NQ = (NG + GW - 1) / GW;
         const int64_t warps = (int64_t)cv.B * cv.Hkv * NQ;
         const int64_t ctas = (warps + ENC_WARPS - 1) / ENC_WARPS;
         if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
-        if (dtype == DKV_F32)
-            encode_delta_kernel<DKV_F32><<<(unsigned)ctas, ENC_WARPS * 32, 0, st>>>(a, NQ);
-        else if (dtype == DKV_F16)
-            encode_delta_kernel<DKV_F16><<<(unsigned)ctas, ENC_WARPS * 32, 0, st>>>(a, NQ);
-        else
-            encode_delta_kernel<DKV_BF16><<<(unsigned)ctas, ENC_WARPS * 32, 0, st>>>(a, NQ);
+        const unsigned grid = (unsigned)ctas, blk = ENC_WARPS * 32;
+        if (lpc == 2) {
+            if (dtype == DKV_F32) encode_delta_kernel<DKV_F32, 2><<<grid, blk, 0, st>>>(a, NQ);
+            else if (dtype == DKV_F16) encode_delta_kernel<DKV_F16, 2><<<grid, blk, 0, st>>>(a, NQ);
+            else encode_delta_kernel<DKV_BF16, 2><<<grid, blk, 0, st>>>(a, NQ);
+        } else {
+            if (dtype == DKV_F32) encode_delta_kernel<DKV_F32, 1><<<grid, blk, 0, st>>>(a, NQ);
+            else if (dtype == DKV_F16) encode_delta_kernel<DKV_F16, 1><<<grid, blk, 0, st>>>(a, NQ);
+            else encode_delta_kernel<DKV_BF16, 1><<<grid, blk, 0, st>>>(a, NQ);
+        }
         return cudaGetLastError();
     }
     int items;
