@@ -1473,7 +1473,8 @@ __device__ inline int merge_len(const CacheView &cv, const int32_t *lenv, int b)
 
 // SEGS (delta format, kf > 32): unit ranges may start and end inside a
 // keyframe group (below); wfl holds one flag byte per warp of the sequence.
-template <bool FIN, bool SEGS>
+// BATCH: partial records loaded per round trip.
+template <bool FIN, bool SEGS, int BATCH>
 __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, int nq, int64_t NW,
                                   const float *ws, float *out, uint8_t *wfl) {
     const int t = blockIdx.x / Hq, h = blockIdx.x % Hq, b = blockIdx.y, c = threadIdx.x;
@@ -1522,7 +1523,6 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
     const bool dense = T >= NW;
     // the records are read in batches of 8 independent loads (one memory
     // round trip per batch); the arithmetic runs over w in order, as written
-    constexpr int BATCH = DKV_MERGE_BATCH;
     auto has = [&](int64_t w) {
         return w <= w1 && (dense || range_start(w, NW, T) < range_start(w + 1, NW, T));
     };
@@ -1630,11 +1630,11 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
     dst[c] = L > 0.f ? O / L : 0.f;     // a causal query with no position gets 0
 }
 
-template <bool FIN, bool SEGS>
+template <bool FIN, bool SEGS, int BATCH>
 __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G, int NHG, int nq,
                                                     int64_t NW, const float *ws, float *out) {
     extern __shared__ uint8_t merge_flags[];        // SEGS: one byte per warp slot
-    merge_body<FIN, SEGS>(cv, Hq, G, NHG, nq, NW, ws, out, merge_flags);
+    merge_body<FIN, SEGS, BATCH>(cv, Hq, G, NHG, nq, NW, ws, out, merge_flags);
     if constexpr (FIN) {
         // fused append: publish batch entry b's new length (no other block of
         // this launch reads it) and make the state slot the split kernel
@@ -1851,14 +1851,26 @@ cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const 
         // a flag byte for each warp slot a sequence can span
         const size_t fl = (size_t)(NW + 15) / 16 * 16;
         if (fl > 48 * 1024) return cudaErrorInvalidConfiguration;
-        if (cv.len_add > 0)
-            merge_kernel<true, true><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
-        else
-            merge_kernel<false, true><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+        // 16 records per round trip need about 160 registers (3 blocks per SM):
+        // when the grid is larger than that wave, 8 per round trip (92)
+        int dev = 0, nsm = 0;
+        cudaError_t e2 = cudaGetDevice(&dev);
+        if (e2 == cudaSuccess) e2 = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        if (e2 != cudaSuccess) return e2;
+        const bool big = (int64_t)grid.x * grid.y <= 3 * (int64_t)nsm;
+        if (cv.len_add > 0) {
+            if (big) merge_kernel<true, true, 16><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+            else merge_kernel<true, true, 8><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+        } else {
+            if (big) merge_kernel<false, true, 16><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+            else merge_kernel<false, true, 8><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+        }
     } else if (cv.len_add > 0) {
-        merge_kernel<true, false><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+        merge_kernel<true, false, DKV_MERGE_BATCH><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws,
+                                                                         out);
     } else {
-        merge_kernel<false, false><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+        merge_kernel<false, false, DKV_MERGE_BATCH><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws,
+                                                                          out);
     }
     return cudaGetLastError();
 }
