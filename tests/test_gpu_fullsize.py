@@ -118,3 +118,107 @@ def test_large_block_append_mid_group(orc, dkv_gpu):
                                   ref.kfr[:ng])
             assert np.array_equal(ex["state"][b, h, t].cpu().numpy().view(np.uint32),
                                   ref.state.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# the other decode forms bench.py times at the headline shape, at full size
+# ---------------------------------------------------------------------------
+def _headline_kv(w, T):
+    K = torch.empty((w.B, w.Hkv, T, w.D), dtype=w.kv_dtype, device=DEV)
+    V = torch.empty_like(K)
+    for b in range(w.B):
+        K[b], V[b] = S.gen_kv_one(w, b, T, device=DEV)
+    return K, V
+
+
+def _sample_refs(orc, K, V, ex, b, h, L, kf, cap):
+    """The oracle's encoding of sequence (b, h): the stored fields must equal
+    it bit for bit; returns its reconstruction of K and V."""
+    xh = []
+    for t, X in enumerate((K, V)):
+        ref = orc.delta_encode(X[b, h, :L].float().cpu().numpy(), kf, cap=cap)
+        if ex is not None:
+            assert np.array_equal(ex["codes"][b, h, t].cpu().numpy()[:L], ref.codes[:L]), (b, h, t)
+            assert np.array_equal(ex["scales"][b, h, t].cpu().numpy().view(np.uint16)[:L],
+                                  ref.scales[:L]), (b, h, t)
+            ng = -(-L // kf)
+            assert np.array_equal(ex["keyframes"][b, h, t].cpu().numpy().view(np.uint16)[:ng],
+                                  ref.kfr[:ng]), (b, h, t)
+            assert np.array_equal(ex["state"][b, h, t].cpu().numpy().view(np.uint32),
+                                  ref.state.view(np.uint32)), (b, h, t)
+        xh.append(ref.xhat[:L])
+    return xh
+
+
+def test_llama3_70b_layer_fused_append_full(orc, dkv_gpu):
+    """dkv_append_decode_attn as bench.py's fused step: one new token per
+    sequence onto 32767 encoded ones, quantised inside the split kernel, then
+    attention over all 32768."""
+    w = S.WORKLOADS["llama3_70b_layer"]
+    T = w.T
+    K, V = _headline_kv(w, T)
+    cache = dkv_gpu.Cache(w.B, w.Hkv, T, "delta", kf=w.kf)
+    cache.encode(K[:, :, :T - 1].contiguous(), V[:, :, :T - 1].contiguous())
+    q = S.gen_q(w, device=DEV)
+    scale = 1.0 / math.sqrt(w.D)
+    out = cache.append_decode_attn(K[:, :, T - 1:].contiguous(), V[:, :, T - 1:].contiguous(), q,
+                                   scale)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    assert cache.seq_lens().tolist() == [T] * w.B
+    ex = cache.export()
+    G = w.Hq // w.Hkv
+    for (b, h) in ((0, 0), (6, 2), (15, 7)):
+        kh, vh = _sample_refs(orc, K, V, ex, b, h, T, w.kf, T)
+        o_ref = orc.attn(q[b, h * G:(h + 1) * G].double().cpu().numpy(), kh, vh, scale)
+        err = row_rel_err(out[b, h * G:(h + 1) * G].cpu().numpy(), o_ref).max()
+        print(f"[fullsize-fused] sample=({b},{h}) max_row_rel_err={err:.3e}")
+        assert err <= ATTN_TOL, (b, h, err)
+
+
+def test_llama3_70b_layer_paged_full(orc, dkv_gpu):
+    """The headline decode through a paged cache: pages of 16 keyframe groups
+    in a shuffled pool (bench.py's paged comparator)."""
+    w = S.WORKLOADS["llama3_70b_layer"]
+    T = w.T
+    K, V = _headline_kv(w, T)
+    cache = dkv_gpu.Cache(w.B, w.Hkv, T, "delta", kf=w.kf, page_groups=16, page_seed=7)
+    cache.encode(K, V)
+    q = S.gen_q(w, device=DEV)
+    scale = 1.0 / math.sqrt(w.D)
+    out = cache.decode_attn(q, scale)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    ex = cache.export()
+    G = w.Hq // w.Hkv
+    for (b, h) in ((1, 1), (14, 6)):
+        kh, vh = _sample_refs(orc, K, V, ex, b, h, T, w.kf, T)
+        o_ref = orc.attn(q[b, h * G:(h + 1) * G].double().cpu().numpy(), kh, vh, scale)
+        err = row_rel_err(out[b, h * G:(h + 1) * G].cpu().numpy(), o_ref).max()
+        print(f"[fullsize-paged] sample=({b},{h}) max_row_rel_err={err:.3e}")
+        assert err <= ATTN_TOL, (b, h, err)
+
+
+def test_llama3_70b_layer_two_queries_full(orc, dkv_gpu):
+    """dkv_decode_attn_mq with 2 causal queries per sequence at the headline
+    shape (bench.py's 2-query comparator: 16 virtual heads per kv head)."""
+    w = S.WORKLOADS["llama3_70b_layer"]
+    T = w.T
+    K, V = _headline_kv(w, T)
+    cache = dkv_gpu.Cache(w.B, w.Hkv, T, "delta", kf=w.kf)
+    cache.encode(K, V)
+    g = torch.Generator().manual_seed(2)
+    Q = torch.randn((w.B, 2, w.Hq, w.D), generator=g).to(w.q_dtype)
+    scale = 1.0 / math.sqrt(w.D)
+    out = cache.decode_attn_mq(Q.to(DEV), scale)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    G = w.Hq // w.Hkv
+    for (b, h) in ((3, 4), (12, 0)):
+        kh, vh = _sample_refs(orc, K, V, None, b, h, T, w.kf, T)
+        for t in range(2):
+            L = T - (1 - t)                          # query t sees the positions before L
+            o_ref = orc.attn(Q[b, t, h * G:(h + 1) * G].double().numpy(), kh[:L], vh[:L], scale)
+            err = row_rel_err(out[b, t, h * G:(h + 1) * G].cpu().numpy(), o_ref).max()
+            print(f"[fullsize-mq] sample=({b},{h}) query={t} max_row_rel_err={err:.3e}")
+            assert err <= ATTN_TOL, (b, h, t, err)
