@@ -305,7 +305,7 @@ struct StageMeta {
     int pad[3];
 };
 static_assert(sizeof(StageMeta) == 32, "stage descriptors are 32 bytes");
-// Stage flags (kf > 32, one segment per stage).
+// Stage flags (kf > 32: one or two segments of one group per stage).
 constexpr int STG_FIRST = 1;   // first segment of its group: slot 0 is the keyframe
 constexpr int STG_CLOSE = 2;   // the group's last segment in this warp's range
 constexpr int STG_HEAD = 4;    // the range entered this group after its first segment

@@ -175,7 +175,10 @@ size_t dkv_decode_workspace_bytes(const dkv_cache_desc *desc, int32_t n_q_heads)
  * sequence gives zeros).
  * Q: [B][n_q_heads][D] device array of q_dtype; out: [B][n_q_heads][D] fp32
  * device array; workspace: device scratch of >= dkv_decode_workspace_bytes;
- * softmax_scale must be finite and > 0 (DKV_EINVAL otherwise).
+ * softmax_scale must be finite and > 0 (DKV_EINVAL otherwise).  The kernels
+ * multiply q as fp16 (fp32 queries as an fp16 hi + lo pair): fp16 and bf16
+ * query values must lie within the fp16 range (|q| <= 65504; bf16 values
+ * below 2^-14 keep an absolute error <= 2^-25).
  * Runs dkv_decode_attn_split then dkv_decode_attn_merge. */
 dkv_status dkv_decode_attn(const dkv_cache *cache, const void *Q, int32_t q_dtype,
                            int32_t n_q_heads, float softmax_scale, float *out,
