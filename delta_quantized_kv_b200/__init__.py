@@ -17,11 +17,15 @@ from pathlib import Path
 
 _PKG = Path(__file__).resolve().parent
 LIB_PATH = _PKG / "_lib" / "libdkv.so"
+# the bounds-checked build (DKV_CHECKED=1, for tests): selected by setting
+# DKV_LIBRARY=checked in the environment before the first load()
+CHECKED_LIB_PATH = _PKG / "_lib" / "libdkv_checked.so"
 
 DKV_OK, DKV_EINVAL, DKV_EALIGN, DKV_ECAPACITY, DKV_EUNSUPPORTED, DKV_ECUDA, DKV_EDEVICE = range(7)
 DKV_FMT_FP16, DKV_FMT_Q4_0, DKV_FMT_DELTA = 0, 1, 2
 DKV_F32, DKV_F16, DKV_BF16 = 0, 1, 2
 DEV_BAD_SEQLEN, DEV_CAPACITY, DEV_TIMEOUT, DEV_BAD_HEADS, DEV_BAD_PAGE = 0x1, 0x2, 0x4, 0x8, 0x10
+DEV_BOUNDS = 0x20
 FORMATS = {"fp16": DKV_FMT_FP16, "q4": DKV_FMT_Q4_0, "delta": DKV_FMT_DELTA}
 
 
@@ -66,14 +70,17 @@ EXPORTS = ["dkv_abi_version", "dkv_cache_bytes", "dkv_cache_init", "dkv_encode",
 
 
 def load():
-    """Load ``libdkv.so`` (raises if it has not been built)."""
+    """Load ``libdkv.so`` (raises if it has not been built), or the
+    bounds-checked ``libdkv_checked.so`` when DKV_LIBRARY=checked."""
     global _lib
     if _lib is not None:
         return _lib
-    if not LIB_PATH.exists():
-        raise RuntimeError(f"libdkv.so not built ({LIB_PATH}); run __graft_entry__.build() "
+    import os
+    path = CHECKED_LIB_PATH if os.environ.get("DKV_LIBRARY") == "checked" else LIB_PATH
+    if not path.exists():
+        raise RuntimeError(f"{path.name} not built ({path}); run __graft_entry__.build() "
                            "or python -m delta_quantized_kv_b200.build")
-    lib = ctypes.CDLL(str(LIB_PATH))
+    lib = ctypes.CDLL(str(path))
     P, S, I, F = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_float
     PC = ctypes.POINTER(dkv_cache)
     PD = ctypes.POINTER(dkv_cache_desc)

@@ -1,7 +1,10 @@
-"""Build the CUDA library ``_lib/libdkv.so`` for sm_100a with nvcc.
+"""Build the CUDA library ``_lib/libdkv.so`` for sm_100a with nvcc, and its
+bounds-checked twin ``_lib/libdkv_checked.so`` (DKV_CHECKED=1: every computed
+global memory range is tested against its buffer; tests load it with
+DKV_LIBRARY=checked).
 
-The library is compiled in-tree so the shared object travels with the source
-tree; nothing is installed into site-packages.
+The libraries are compiled in-tree so the shared objects travel with the
+source tree; nothing is installed into site-packages.
 """
 from __future__ import annotations
 
@@ -13,6 +16,7 @@ from pathlib import Path
 PKG = Path(__file__).resolve().parent
 CSRC = PKG / "csrc"
 OUT = PKG / "_lib" / "libdkv.so"
+OUT_CHECKED = PKG / "_lib" / "libdkv_checked.so"
 SOURCES = ["dkv_api.cu", "encode.cu", "decode.cu", "noalloc.cu", "lr_encode.cu", "lr_decode.cu"]
 HEADERS = ["dkv_common.cuh", "dkv_internal.h"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -26,24 +30,36 @@ def _nvcc() -> str:
     return cand
 
 
-def stale() -> bool:
-    if not OUT.exists():
+def stale(out: Path = OUT) -> bool:
+    if not out.exists():
         return True
-    t = OUT.stat().st_mtime
+    t = out.stat().st_mtime
     deps = [CSRC / s for s in SOURCES + HEADERS] + [PKG.parent / "include" / "dkv.h"]
     return any(d.stat().st_mtime > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> Path:
+def build(force: bool = False, verbose: bool = False, checked: bool = True) -> Path:
+    """Build the library (and, with checked, its bounds-checked twin, at the
+    same time)."""
+    if not checked:
+        return _build_one(OUT, [], force, verbose)
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=2) as ex:
+        jobs = [ex.submit(_build_one, OUT, [], force, verbose),
+                ex.submit(_build_one, OUT_CHECKED, ["-DDKV_CHECKED=1"], force, verbose)]
+        return [j.result() for j in jobs][0]
+
+
+def _build_one(OUT: Path, extra: list, force: bool, verbose: bool) -> Path:
     """Compile every translation unit in parallel (one nvcc per file), then
     link the shared library; the result replaces the old one atomically."""
-    if not force and not stale():
+    if not force and not stale(OUT):
         return OUT
     from concurrent.futures import ThreadPoolExecutor
     import tempfile
     OUT.parent.mkdir(parents=True, exist_ok=True)
     nvcc = _nvcc()
-    cflags = [f for f in NVCC_FLAGS if f != "-shared"]
+    cflags = [f for f in NVCC_FLAGS if f != "-shared"] + extra
     with tempfile.TemporaryDirectory(prefix="dkv_build_") as tmpd:
         objs = [Path(tmpd) / (Path(s).stem + ".o") for s in SOURCES]
 
@@ -59,7 +75,7 @@ def build(force: bool = False, verbose: bool = False) -> Path:
                 print(r.stdout + r.stderr)
             if r.returncode:
                 raise subprocess.CalledProcessError(r.returncode, r.args, r.stdout, r.stderr)
-        tmp = OUT.with_name(f"libdkv.{os.getpid()}.tmp.so")
+        tmp = OUT.with_name(f"{OUT.stem}.{os.getpid()}.tmp.so")
         subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
                         "-o", str(tmp), *[str(o) for o in objs]], check=True)
     os.replace(tmp, OUT)

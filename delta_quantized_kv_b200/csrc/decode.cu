@@ -142,6 +142,7 @@ struct SplitArgs {
     float scale_log2;          // softmax_scale * log2(e), > 0
     float wshift;              // log2 of the factor every softmax weight is scaled down by
     float *ws;                 // partial records
+    int64_t ws_floats;         // workspace size (checked builds test every record against it)
     float *heads, *hands;      // kf > 32: the records of groups entered midway, the handoffs
     int fault;                 // test support: 1 = arm the copy barriers but issue no copy
     // fused append (cv.len_add = n > 0): the n new tokens of each sequence,
@@ -387,7 +388,7 @@ __device__ inline const uint8_t *stage_rec(const CacheView &cv, Cursor &c, int n
 template <int FMT, int MODE, bool PAGED>
 __device__ inline void issue_stage(const CacheView &cv, Cursor &c, int nhg, int nu,
                                    int npos_all, uint8_t *stage, uint64_t *bar, int fault) {
-    constexpr int NU = KCfg<FMT, MODE>::NU;
+    constexpr int NU = KCfg<FMT, MODE>::NU, STAGE = KCfg<FMT, MODE>::STAGE;
     const uint8_t *sb = c.seq;
     if (fault) {
         // test support: expect bytes that never come, so the consumer's bounded
@@ -403,6 +404,10 @@ __device__ inline void issue_stage(const CacheView &cv, Cursor &c, int nhg, int 
             return;
         }
         const uint32_t bytes = (uint32_t)(nu * cv.rec_bytes);
+        if (!rec_ok(cv, rec, bytes) || !range_ok(cv.header, stage, bytes, stage, STAGE)) {
+            mbar_arrive_expect_tx(bar, 0);   // checked build: nothing copied
+            return;
+        }
         mbar_arrive_expect_tx(bar, bytes);
         bulk_g2s(stage, rec, bytes, bar);
     } else if (FMT == DKV_FMT_DELTA) {
@@ -423,10 +428,20 @@ __device__ inline void issue_stage(const CacheView &cv, Cursor &c, int nhg, int 
         const int nd = npos - s0;
         const int di0 = a + s0 - 1;
         const uint32_t bytes = (a == 0 ? KF_BYTES : 0) + nd * (SC_BYTES + 2 * NIB_BYTES);
+        const StageMap sm = stage_map<FMT, MODE>(kf, cv.rec_bytes, 0);
+        if (DKV_CHECKED &&
+            !(rec_ok(cv, rec, (int64_t)cv.rec_bytes) &&
+              rec_ok(cv, scs + (int64_t)di0 * SC_BYTES, (int64_t)nd * SC_BYTES) &&
+              rec_ok(cv, kns + (int64_t)di0 * NIB_BYTES, (int64_t)nd * NIB_BYTES) &&
+              rec_ok(cv, vns + (int64_t)di0 * NIB_BYTES, (int64_t)nd * NIB_BYTES) &&
+              range_ok(cv.header, stage + sm.vn0 + s0 * NIB_BYTES, (int64_t)nd * NIB_BYTES, stage,
+                       STAGE))) {
+            mbar_arrive_expect_tx(bar, 0);   // checked build: nothing copied
+            return;
+        }
         mbar_arrive_expect_tx(bar, bytes);
         if (a == 0) bulk_g2s(stage, rec, KF_BYTES, bar);
         if (nd > 0) {
-            const StageMap sm = stage_map<FMT, MODE>(kf, cv.rec_bytes, 0);
             bulk_g2s(stage + sm.sc0 + s0 * SC_BYTES, scs + (int64_t)di0 * SC_BYTES, nd * SC_BYTES,
                      bar);
             bulk_g2s(stage + sm.kn0 + s0 * NIB_BYTES, kns + (int64_t)di0 * NIB_BYTES,
@@ -436,6 +451,12 @@ __device__ inline void issue_stage(const CacheView &cv, Cursor &c, int nhg, int 
         }
     } else if (FMT == DKV_FMT_Q4_0) {
         const int p0 = c.g * SEG;
+        if (!rec_ok(cv, sb + (int64_t)p0 * SC_BYTES, (int64_t)npos_all * SC_BYTES) ||
+            !rec_ok(cv, sb + (int64_t)cv.cap * (SC_BYTES + NIB_BYTES) + (int64_t)p0 * NIB_BYTES,
+                    (int64_t)npos_all * NIB_BYTES)) {
+            mbar_arrive_expect_tx(bar, 0);   // checked build: nothing copied
+            return;
+        }
         mbar_arrive_expect_tx(bar, npos_all * (SC_BYTES + 2 * NIB_BYTES));
         bulk_g2s(stage, sb + (int64_t)p0 * SC_BYTES, npos_all * SC_BYTES, bar);
         bulk_g2s(stage + 512 * NU, sb + (int64_t)cv.cap * SC_BYTES + (int64_t)p0 * NIB_BYTES,
@@ -444,6 +465,11 @@ __device__ inline void issue_stage(const CacheView &cv, Cursor &c, int nhg, int 
                  npos_all * NIB_BYTES, bar);
     } else {
         const int p0 = c.g * SEG;
+        if (!rec_ok(cv, sb + (int64_t)p0 * 256, (int64_t)npos_all * 256) ||
+            !rec_ok(cv, sb + (int64_t)cv.cap * 256 + (int64_t)p0 * 256, (int64_t)npos_all * 256)) {
+            mbar_arrive_expect_tx(bar, 0);   // checked build: nothing copied
+            return;
+        }
         mbar_arrive_expect_tx(bar, npos_all * 512);
         bulk_g2s(stage, sb + (int64_t)p0 * 256, npos_all * 256, bar);
         bulk_g2s(stage + 8192, sb + (int64_t)cv.cap * 256 + (int64_t)p0 * 256, npos_all * 256, bar);
@@ -891,6 +917,17 @@ __device__ __noinline__ void append_tokens(const SplitArgs &A, int b, int kvh, i
     const int64_t sb = ((int64_t)b * cv.Hkv + kvh) * 2 * D;          // (b, kvh) in a slot
     const int64_t slot = (int64_t)cv.B * cv.Hkv * 2 * D;
     const int64_t row0 = ((int64_t)b * cv.Hkv + kvh) * n;
+    // checked build: the sequence's state in both slots and its n input rows
+    if (DKV_CHECKED) {
+        const int ies = A.kv_dtype == DKV_F32 ? 4 : 2;
+        const int64_t in_bytes = (int64_t)cv.B * cv.Hkv * n * D * ies;
+        if (!state_ok(cv, cv.state + sb, 2 * D) || !state_ok(cv, cv.state + slot + sb, 2 * D) ||
+            !range_ok(cv.header, static_cast<const uint8_t *>(A.Kn) + row0 * D * ies,
+                      (int64_t)n * D * ies, A.Kn, in_bytes) ||
+            !range_ok(cv.header, static_cast<const uint8_t *>(A.Vn) + row0 * D * ies,
+                      (int64_t)n * D * ies, A.Vn, in_bytes))
+            return;
+    }
     // one round trip: the slot word, both state slots and the first token
     const int parity = cv.header[2] & 1;
     const bool cont = (L0 % kf) != 0;            // the first token continues a group
@@ -917,6 +954,7 @@ __device__ __noinline__ void append_tokens(const SplitArgs &A, int b, int kvh, i
         const int p = L0 + i, g = p / kf, di = p - g * kf;   // di 0: keyframe; else delta di - 1
         if (p >= p_hi) break;
         uint8_t *rec = p >= p_lo ? rec_ptr<PAGED>(cv, b, kvh, g) : nullptr;
+        if (rec && !rec_ok(cv, rec, cv.rec_bytes)) rec = nullptr;   // checked build
         if (di == 0) {
 #pragma unroll
             for (int t = 0; t < 2; ++t)
@@ -1075,7 +1113,8 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
             // the new ones); an entry that takes no tokens keeps its
             // reconstruction: carry it into the slot the merge makes current
             int32_t *lenv = merge_lengths(A.ws, NW, cv.B * nvs);
-            for (int b = lane; b < cv.B; b += 32) lenv[b] = clamp_len(cv, b);
+            if (range_ok(cv.header, lenv, (int64_t)cv.B * 4, A.ws, A.ws_floats * 4))
+                for (int b = lane; b < cv.B; b += 32) lenv[b] = clamp_len(cv, b);
             const int parity = cv.header[2] & 1;
             const int64_t per_b = (int64_t)cv.Hkv * 2 * D;
             for (int b = 0; b < cv.B; ++b) {
@@ -1097,7 +1136,8 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
             }
         }
     }
-    if (MODE == PREFIX && gw == 0 && lane == 0) A.hands[0] = A.scale_log2;   // for the merge
+    if (MODE == PREFIX && gw == 0 && lane == 0 && range_ok(cv.header, A.hands, 4, A.ws, A.ws_floats * 4))
+        A.hands[0] = A.scale_log2;   // for the merge
     if (total == 0) return;
     const int64_t r0 = range_start(gw, NW, total), r1 = range_start(gw + 1, NW, total);
     if (r0 >= r1) return;
@@ -1169,6 +1209,8 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
             l += __shfl_xor_sync(0xffffffffu, l, 16);
             l_run[e] = l;
         }
+        // checked build: the record inside the workspace (uniform over the warp)
+        if (!range_ok(cv.header, rec, PARTIAL_FLOATS * 4, A.ws, A.ws_floats * 4)) return;
         if (gq == 0) {
             rec[2 * tq] = m_run[0];
             rec[2 * tq + 1] = m_run[1];
@@ -1224,11 +1266,16 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
             }
             const int64_t qrow =
                 (((int64_t)meta.b * A.nq + qt) * A.Hq + (int64_t)kvh * A.G + hl) * D;
+            // checked build: the q row inside Q ([B][nq][Hq][D] of q_dtype)
+            const int qes = A.q_dtype == DKV_F32 ? 4 : 2;
+            const bool q_in = !qok || range_ok(cv.header, static_cast<const uint8_t *>(A.Q) + qrow * qes,
+                                               (int64_t)D * qes, A.Q,
+                                               (int64_t)cv.B * A.nq * A.Hq * D * qes);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int c = 16 * kk + 2 * tq;
                 float q0 = 0.f, q1 = 0.f, q8 = 0.f, q9 = 0.f;
-                if (qok) {
+                if (qok && q_in) {
                     q0 = q_elem(A.Q, A.q_dtype, qrow + c);
                     q1 = q_elem(A.Q, A.q_dtype, qrow + c + 1);
                     q8 = q_elem(A.Q, A.q_dtype, qrow + c + 8);
@@ -1392,7 +1439,9 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
             if (MODE == PREFIX && last_seg) {
                 // a range that ends inside the group hands the next warp the
                 // scaled dots of its last position and that position's value row
-                const bool hand = (meta.flags & STG_HAND) != 0;
+                const bool hand = (meta.flags & STG_HAND) != 0 &&
+                                  range_ok(cv.header, A.hands + HAND_HDR + gw * HANDOFF_FLOATS,
+                                           HANDOFF_FLOATS * 4, A.ws, A.ws_floats * 4);
                 float *hd = A.hands + HAND_HDR + gw * HANDOFF_FLOATS;
                 if (hand && gq == 0) {
                     hd[2 * tq] = dot_carry[0];
@@ -1476,13 +1525,15 @@ __device__ inline int merge_len(const CacheView &cv, const int32_t *lenv, int b)
 // BATCH: partial records loaded per round trip.
 template <bool FIN, bool SEGS, int BATCH>
 __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, int nq, int64_t NW,
-                                  const float *ws, float *out, uint8_t *wfl) {
+                                  const float *ws, int64_t ws_floats, float *out, uint8_t *wfl) {
     const int t = blockIdx.x / Hq, h = blockIdx.x % Hq, b = blockIdx.y, c = threadIdx.x;
     const int nvs = cv.Hkv * NHG;
     const int32_t *lenv = FIN ? merge_lengths(const_cast<float *>(ws), NW, cv.B * nvs) : nullptr;
     const int len = merge_len<FIN>(cv, lenv, b);
     const int ub = units_of(cv.fmt, cv.kf, len);
     float *dst = out + (((int64_t)b * nq + t) * Hq + h) * D;
+    // checked build: this block's output row inside out ([B][nq][Hq][D])
+    if (!range_ok(cv.header, dst, D * 4, out, (int64_t)cv.B * nq * Hq * D * 4)) return;
     if (ub == 0) {                      // uniform over the block
         dst[c] = 0.f;
         return;
@@ -1558,7 +1609,8 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
         __syncthreads();
         heads = head_records(const_cast<float *>(ws), NW, (int64_t)cv.B * nvs, cv.B);
         hands = handoffs(const_cast<float *>(ws), NW, (int64_t)cv.B * nvs, cv.B);
-        sl2 = hands[0];                 // the log2 softmax scale the split kernel used
+        // the log2 softmax scale the split kernel used
+        sl2 = range_ok(cv.header, hands, 4, ws, ws_floats * 4) ? hands[0] : 0.f;
         hands += HAND_HDR;
     }
     float cdot = 0.f, cval = 0.f;       // the carried state: head j's scaled dot, value c
@@ -1577,13 +1629,18 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
                 ok[i] = has(w + i);
             }
             const float *rec = ws + (w + i + vseq) * PARTIAL_FLOATS;
+            if (DKV_CHECKED && ok[i])
+                ok[i] = range_ok(cv.header, rec, PARTIAL_FLOATS * 4, ws, ws_floats * 4);
             mv[i] = ok[i] ? rec[j] : -1e30f;
             lv[i] = ok[i] ? rec[8 + j] : 0.f;
             ov[i] = ok[i] ? rec[16 + j * 128 + c] : 0.f;
             if constexpr (SEGS) {
-                const bool hd = fl[i] & W_HEAD, tl = fl[i] & W_HAND;
                 const float *hr = heads + (w + i) * PARTIAL_FLOATS;
                 const float *hh = hands + (w + i) * HANDOFF_FLOATS;
+                const bool hd = (fl[i] & W_HEAD) &&
+                                range_ok(cv.header, hr, PARTIAL_FLOATS * 4, ws, ws_floats * 4);
+                const bool tl = (fl[i] & W_HAND) &&
+                                range_ok(cv.header, hh, HANDOFF_FLOATS * 4, ws, ws_floats * 4);
                 hm[i] = hd ? hr[j] : -1e30f;
                 hl[i] = hd ? hr[8 + j] : 0.f;
                 ho[i] = hd ? hr[16 + j * 128 + c] : 0.f;
@@ -1632,9 +1689,10 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
 
 template <bool FIN, bool SEGS, int BATCH>
 __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G, int NHG, int nq,
-                                                    int64_t NW, const float *ws, float *out) {
+                                                    int64_t NW, const float *ws, int64_t ws_floats,
+                                                    float *out) {
     extern __shared__ uint8_t merge_flags[];        // SEGS: one byte per warp slot
-    merge_body<FIN, SEGS, BATCH>(cv, Hq, G, NHG, nq, NW, ws, out, merge_flags);
+    merge_body<FIN, SEGS, BATCH>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out, merge_flags);
     if constexpr (FIN) {
         // fused append: publish batch entry b's new length (no other block of
         // this launch reads it) and make the state slot the split kernel
@@ -1805,9 +1863,10 @@ static cudaError_t launch_split_t(const SplitArgs &a_in, cudaStream_t st) {
 cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq, int nq,
                          float softmax_scale, float *ws, int64_t ws_floats, int fault,
                          cudaStream_t st, const void *K_new, const void *V_new, int kv_dtype) {
-    (void)ws_floats;
     SplitArgs a;
-    a.fault = fault;
+    a.fault = fault == 1 ? 1 : 0;
+    // test support (mode 2): the workspace declared two records short
+    a.ws_floats = fault == 2 ? ws_floats - 2 * PARTIAL_FLOATS : ws_floats;
     a.Kn = K_new;
     a.Vn = V_new;
     a.kv_dtype = kv_dtype;
@@ -1838,7 +1897,7 @@ cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq
 }
 
 cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const float *ws,
-                         cudaStream_t st) {
+                         int64_t ws_floats, cudaStream_t st) {
     const int G = Hq / cv.Hkv;
     const int NHG = (nq * G + 7) / 8;
     SplitGeom g;
@@ -1859,18 +1918,18 @@ cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const 
         if (e2 != cudaSuccess) return e2;
         const bool big = (int64_t)grid.x * grid.y <= 3 * (int64_t)nsm;
         if (cv.len_add > 0) {
-            if (big) merge_kernel<true, true, 16><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
-            else merge_kernel<true, true, 8><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+            if (big) merge_kernel<true, true, 16><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
+            else merge_kernel<true, true, 8><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
         } else {
-            if (big) merge_kernel<false, true, 16><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
-            else merge_kernel<false, true, 8><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, out);
+            if (big) merge_kernel<false, true, 16><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
+            else merge_kernel<false, true, 8><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
         }
     } else if (cv.len_add > 0) {
         merge_kernel<true, false, DKV_MERGE_BATCH><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws,
-                                                                         out);
+                                                                         ws_floats, out);
     } else {
         merge_kernel<false, false, DKV_MERGE_BATCH><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws,
-                                                                          out);
+                                                                          ws_floats, out);
     }
     return cudaGetLastError();
 }

@@ -92,6 +92,7 @@ CacheView view_of(const dkv_cache *c) {
     CacheView v;
     uint8_t *base = static_cast<uint8_t *>(c->base);
     v.data = base + c->off_data;
+    v.data_bytes = (int64_t)c->desc.batch * c->desc.n_kv_heads * (int64_t)c->seq_stride;
     v.state = reinterpret_cast<float *>(base + c->off_state);
     v.seqlen = reinterpret_cast<int32_t *>(base + c->off_seqlen);
     v.header = reinterpret_cast<int32_t *>(base + c->off_header);
@@ -305,7 +306,7 @@ dkv_status dkv_decode_attn_merge(const dkv_cache *cache, int32_t n_q_heads, floa
     if (!aligned16(out)) return DKV_EALIGN;
     CacheView v = view_of(cache);
     return cuda_status(dkv::launch_merge(v, n_q_heads, 1, out, static_cast<const float *>(workspace),
-                                         static_cast<cudaStream_t>(stream)));
+                                         need, static_cast<cudaStream_t>(stream)));
 }
 
 dkv_status dkv_decode_attn(const dkv_cache *cache, const void *Q, int32_t q_dtype,
@@ -335,7 +336,7 @@ dkv_status dkv_decode_attn_mq(const dkv_cache *cache, const void *Q, int32_t q_d
     float *ws = static_cast<float *>(workspace);
     cudaError_t e = dkv::launch_split(v, Q, q_dtype, n_q_heads, n_queries, softmax_scale, ws,
                                       need, g_debug_fault, st);
-    if (e == cudaSuccess) e = dkv::launch_merge(v, n_q_heads, n_queries, out, ws, st);
+    if (e == cudaSuccess) e = dkv::launch_merge(v, n_q_heads, n_queries, out, ws, need, st);
     return cuda_status(e);
 }
 
@@ -376,7 +377,7 @@ dkv_status dkv_append_decode_attn_merge(dkv_cache *cache, int32_t n_new, int32_t
     CacheView v = view_of(cache);
     v.len_add = n_new;
     return cuda_status(dkv::launch_merge(v, n_q_heads, n_new, out,
-                                         static_cast<const float *>(workspace),
+                                         static_cast<const float *>(workspace), need,
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -484,7 +485,7 @@ dkv_status dkv_get_device_status(const dkv_cache *cache, int32_t *host_out, void
     return h ? DKV_EDEVICE : DKV_OK;
 }
 
-void dkv_debug_set_fault(int32_t mode) { g_debug_fault = mode == 1 ? 1 : 0; }
+void dkv_debug_set_fault(int32_t mode) { g_debug_fault = (mode == 1 || mode == 2) ? mode : 0; }
 
 dkv_status dkv_debug_division_check(const float *u_dev, int32_t n, uint64_t *mismatches_dev,
                                     void *stream) {

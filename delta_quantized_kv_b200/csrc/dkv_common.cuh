@@ -88,6 +88,7 @@ __host__ __device__ inline int nib_channel(int t, int w, int i) {
 // Device-side cache view passed by value to kernels.
 struct CacheView {
     uint8_t *data;
+    int64_t data_bytes;    // bytes of the data area (contiguous caches)
     float *state;          // [2][B][Hkv][2][D]
     int32_t *seqlen;       // [B]
     int32_t *header;       // {status, counter, parity, reserved}
@@ -106,6 +107,36 @@ struct CacheView {
 
 __device__ inline void set_status(int32_t *header, int bits) {
     atomicOr(reinterpret_cast<int *>(header), bits);
+}
+
+// Checked builds (DKV_CHECKED=1, for tests): every computed global memory
+// range is tested against the buffer it must lie in; a range outside sets
+// DKV_DEV_BOUNDS and the access is skipped.  In normal builds the tests are
+// compiled out.
+#ifndef DKV_CHECKED
+#define DKV_CHECKED 0
+#endif
+__device__ inline bool range_ok(int32_t *header, const void *p, int64_t n, const void *lo,
+                                int64_t size) {
+    if constexpr (DKV_CHECKED == 0) {
+        return true;
+    } else {
+        const uint8_t *a = static_cast<const uint8_t *>(p), *b = static_cast<const uint8_t *>(lo);
+        const bool ok = n >= 0 && a >= b && a + n <= b + size;
+        if (!ok) set_status(header, DKV_DEV_BOUNDS);
+        return ok;
+    }
+}
+// n bytes at p inside the cache's records: the data area, or the page pool
+__device__ inline bool rec_ok(const CacheView &cv, const void *p, int64_t n) {
+    if constexpr (DKV_CHECKED == 0) return true;
+    return cv.pg ? range_ok(cv.header, p, n, cv.pool, cv.n_pages * cv.page_bytes)
+                 : range_ok(cv.header, p, n, cv.data, cv.data_bytes);
+}
+// n floats at p inside the reconstruction state (both slots)
+__device__ inline bool state_ok(const CacheView &cv, const float *p, int64_t n) {
+    if constexpr (DKV_CHECKED == 0) return true;
+    return range_ok(cv.header, p, n * 4, cv.state, (int64_t)2 * cv.B * cv.Hkv * 2 * D * 4);
 }
 
 // Record g (delta format) of sequence (b, kvh): contiguous, or through the

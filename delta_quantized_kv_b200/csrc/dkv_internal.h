@@ -50,7 +50,7 @@ cudaError_t launch_split(const CacheView &cv, const void *Q, int q_dtype, int Hq
                          cudaStream_t st, const void *K_new = nullptr,
                          const void *V_new = nullptr, int kv_dtype = 0);
 cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const float *ws,
-                         cudaStream_t st);
+                         int64_t ws_floats, cudaStream_t st);
 
 // Long-range reference encoding of n_seq sequences [n_seq][T][D] (layouts
 // of dkv_lr_encode).

@@ -89,6 +89,16 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
     const void *src = t == 0 ? a.K : a.V;
     const int64_t in_base = (((int64_t)b * cv.Hkv + kvh) * a.T_in) * D;
     uint8_t *sb = seq_base(cv, b, kvh);
+    // checked build (block-uniform): this sequence's state rows, its n input
+    // rows and, for the comparators, its data
+    if (DKV_CHECKED && active) {
+        const int es = a.dtype == DKV_F32 ? 4 : 2;
+        const int64_t in_bytes = (int64_t)cv.B * cv.Hkv * a.T_in * D * es;
+        active = state_ok(cv, state_old, D) && state_ok(cv, state_new, D) &&
+                 range_ok(cv.header, static_cast<const uint8_t *>(src) + in_base * es,
+                          (int64_t)n * D * es, src, in_bytes) &&
+                 (FMT == DKV_FMT_DELTA || rec_ok(cv, sb, cv.seq_stride));
+    }
 
     if (active) {
         if (FMT == DKV_FMT_DELTA) {
@@ -96,6 +106,7 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
             const int g = start / kf + blockIdx.x;
             const int p0 = max(start, g * kf), p1 = min(start + n, (g + 1) * kf);
             uint8_t *rec = p0 < p1 ? rec_ptr(cv, b, kvh, g) : nullptr;
+            if (rec && !rec_ok(cv, rec, cv.rec_bytes)) rec = nullptr;   // checked build
             if (p0 < p1 && !rec) {
                 // bad block-table entry (flagged by rec_ptr): nothing written;
                 // the state carries over
@@ -289,9 +300,16 @@ __global__ void __launch_bounds__(ENC_WARPS * 32) encode_delta_kernel(EncodeArgs
         const int64_t sb = (((int64_t)b * cv.Hkv + kvh) * 2 + t) * D + 32 * j + CH * u;
         const float *st_old = cv.state + parity * slot + sb;
         float *st_new = cv.state + (parity ^ 1) * slot + sb;
+        // checked build: the block's 32 state channels in both slots (the same
+        // test in both lanes of a loop); outside, the loop is skipped (every
+        // thread still reaches the grid's last-block step below)
+        const bool st_in = !DKV_CHECKED ||
+                           (state_ok(cv, st_old - CH * u, 32) && state_ok(cv, st_new - CH * u, 32));
         if (n < 0 && qd == 0 && kvh == 0 && lane == 0)
             set_status(cv.header, n == -2 ? DKV_DEV_CAPACITY : DKV_DEV_BAD_SEQLEN);
-        if (n <= 0) {
+        if (!st_in) {
+            // checked build: state outside its buffer, nothing read or written
+        } else if (n <= 0) {
             if (gi == 0) {                         // nothing written: carry the state over
 #pragma unroll
                 for (int c = 0; c < CH; ++c) st_new[c] = a.append ? st_old[c] : 0.0f;
@@ -301,7 +319,19 @@ __global__ void __launch_bounds__(ENC_WARPS * 32) encode_delta_kernel(EncodeArgs
             const int p0 = max(start, g * kf), p1 = min(start + n, (g + 1) * kf);
             const bool last = p1 == start + n;
             uint8_t *rec = p0 < p1 ? rec_ptr(cv, b, kvh, g) : nullptr;
-            if (p0 < p1 && !rec) {
+            if (rec && !rec_ok(cv, rec, cv.rec_bytes)) rec = nullptr;   // checked build
+            bool in_ok = true;
+            if (DKV_CHECKED && p0 < p1) {
+                // the block's input rows [p0, p1) (the same test in both lanes)
+                const int es = DT == DKV_F32 ? 4 : 2;
+                const int64_t row = (((int64_t)b * cv.Hkv + kvh) * a.T_in - start + p0) * D + 32 * j;
+                in_ok = range_ok(cv.header, static_cast<const uint8_t *>(t ? a.V : a.K) + row * es,
+                                 ((int64_t)(p1 - p0 - 1) * D + 32) * es, t ? a.V : a.K,
+                                 (int64_t)cv.B * cv.Hkv * a.T_in * D * es);
+            }
+            if (!in_ok) {
+                // checked build: input outside its buffer, nothing written
+            } else if (p0 < p1 && !rec) {
                 // bad block-table entry (flagged by rec_ptr): nothing written
                 if (last) {
 #pragma unroll

@@ -72,6 +72,8 @@ typedef enum { DKV_F32 = 0, DKV_F16 = 1, DKV_BF16 = 2 } dkv_dtype;
 #define DKV_DEV_TIMEOUT      0x4   /* a bounded pipeline wait ran out */
 #define DKV_DEV_BAD_HEADS    0x8   /* n_q_heads not a multiple of n_kv_heads */
 #define DKV_DEV_BAD_PAGE     0x10  /* a block-table entry outside the page pool (skipped) */
+#define DKV_DEV_BOUNDS       0x20  /* checked build only: a computed memory range outside its
+                                      buffer (the access was skipped) */
 
 typedef struct {
     int32_t batch;         /* B >= 1 (<= 1024) */
@@ -363,8 +365,12 @@ dkv_status dkv_get_device_status(const dkv_cache *cache, int32_t *host_out, void
  * copy barriers without issuing the copies, so every bounded pipeline wait
  * runs out (after about a second) and the kernel records DKV_DEV_TIMEOUT in
  * the status word and returns, instead of hanging; the outputs of such a
- * launch are meaningless.  Mode 0 restores normal operation.  Nothing traps
- * or faults either way.  Not thread-safe; meant for tests. */
+ * launch are meaningless.  With mode 2, those launches are told the workspace
+ * is two partial records smaller than it is: the bounds-checked build
+ * (DKV_CHECKED) then records DKV_DEV_BOUNDS and skips the last record's
+ * writes (the buffer itself is large enough, so nothing is touched out of
+ * range); other builds ignore it.  Mode 0 restores normal operation.  Nothing
+ * traps or faults either way.  Not thread-safe; meant for tests. */
 void dkv_debug_set_fault(int32_t mode);
 
 /* Test support (no counterpart on the pages): checks the quotient the
