@@ -66,7 +66,7 @@ constexpr int WARPS = DKV_WARPS;             // warps per CTA (independent pipel
 #define DKV_QSM 1                // q fragments in shared memory (0: registers)
 #endif
 #ifndef DKV_MERGE_BATCH
-#define DKV_MERGE_BATCH 16       // partial records the merge loads per round trip
+#define DKV_MERGE_BATCH 4        // partial records a merge warp loads per round trip
 #endif
 #ifndef DKV_NIB_NU
 #define DKV_NIB_NU 2
@@ -1572,13 +1572,9 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
     // with at least one unit per warp every range is non-empty; otherwise
     // skip the warps that own no unit (they wrote no record)
     const bool dense = T >= NW;
-    // the records are read in batches of 8 independent loads (one memory
-    // round trip per batch); the arithmetic runs over w in order, as written
     auto has = [&](int64_t w) {
         return w <= w1 && (dense || range_start(w, NW, T) < range_start(w + 1, NW, T));
     };
-    // one pass, rescaling online: each batch of 8 records moves the running
-    // maximum once (records of warps that saw no position carry -1e30)
     // SEGS: ranges may start and end inside a keyframe group.  A warp that
     // entered a group midway wrote that part as a separate record with scores
     // and value rows relative to the state before its first position; the
@@ -1613,27 +1609,57 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
         sl2 = range_ok(cv.header, hands, 4, ws, ws_floats * 4) ? hands[0] : 0.f;
         hands += HAND_HDR;
     }
-    float cdot = 0.f, cval = 0.f;       // the carried state: head j's scaled dot, value c
-    float M = -1e30f, L = 0.f, O = 0.f;
-    for (int64_t w = w0; w <= w1; w += BATCH) {
-        float mv[BATCH], lv[BATCH], ov[BATCH];
-        float hm[BATCH], hl[BATCH], ho[BATCH], hdot[BATCH], hval[BATCH];
+    auto flag = [&](int64_t w) -> uint8_t {
+        if constexpr (SEGS) return wfl[w - w0];
+        else return has(w) ? W_ANY : 0;
+    };
+    // The sequence's warps in four quarters, one per warp of this block; lane
+    // l holds channels 4 l .. 4 l + 3.  The quarters are merged at the end.
+    const int wq = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nw = w1 - w0 + 1;
+    const int64_t qa = w0 + (nw * wq) / 4, qe = w0 + (nw * (wq + 1)) / 4;
+    auto ld4 = [](const float *p) { return *reinterpret_cast<const float4 *>(p); };
+    auto fma4 = [](float4 a, float s, float4 c) {
+        return make_float4(fmaf(a.x, s, c.x), fmaf(a.y, s, c.y), fmaf(a.z, s, c.z), fmaf(a.w, s, c.w));
+    };
+    // the carried state (SEGS): head j's scaled dot and this lane's 4 values
+    float cdot = 0.f;
+    float4 cval = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (SEGS) {
+        // entering the quarter inside a group: sum the handoffs back to the
+        // nearest absolute one (one step unless warps are shorter than groups)
+        if (qa < qe && (flag(qa) & W_HEAD)) {
+            for (int64_t k = qa - 1; k >= w0; --k) {
+                const uint8_t f = flag(k);
+                if (!(f & W_ANY)) continue;
+                const float *hh = hands + k * HANDOFF_FLOATS;
+                if ((f & W_HAND) && range_ok(cv.header, hh, HANDOFF_FLOATS * 4, ws, ws_floats * 4)) {
+                    cdot += hh[j] * sl2;
+                    cval = fma4(ld4(hh + 8 + 4 * lane), 1.f, cval);
+                }
+                if (!(f & W_REL)) break;
+            }
+        }
+    }
+    // one pass per quarter, rescaling online: each batch of records moves the
+    // running maximum once (records of warps that saw no position carry -1e30)
+    float M = -1e30f, L = 0.f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t w = qa; w < qe; w += BATCH) {
+        float mv[BATCH], lv[BATCH], hm[BATCH], hl[BATCH], hdot[BATCH];
+        float4 ov[BATCH], ho[BATCH], hval[BATCH];
         uint8_t fl[BATCH];
         bool ok[BATCH];
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
-            if constexpr (SEGS) {
-                fl[i] = w + i <= w1 ? wfl[w + i - w0] : 0;
-                ok[i] = fl[i] & W_ANY;
-            } else {
-                ok[i] = has(w + i);
-            }
+            fl[i] = w + i < qe ? flag(w + i) : 0;
+            ok[i] = fl[i] & W_ANY;
             const float *rec = ws + (w + i + vseq) * PARTIAL_FLOATS;
             if (DKV_CHECKED && ok[i])
                 ok[i] = range_ok(cv.header, rec, PARTIAL_FLOATS * 4, ws, ws_floats * 4);
             mv[i] = ok[i] ? rec[j] : -1e30f;
             lv[i] = ok[i] ? rec[8 + j] : 0.f;
-            ov[i] = ok[i] ? rec[16 + j * 128 + c] : 0.f;
+            ov[i] = ok[i] ? ld4(rec + 16 + j * 128 + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
             if constexpr (SEGS) {
                 const float *hr = heads + (w + i) * PARTIAL_FLOATS;
                 const float *hh = hands + (w + i) * HANDOFF_FLOATS;
@@ -1641,11 +1667,13 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
                                 range_ok(cv.header, hr, PARTIAL_FLOATS * 4, ws, ws_floats * 4);
                 const bool tl = (fl[i] & W_HAND) &&
                                 range_ok(cv.header, hh, HANDOFF_FLOATS * 4, ws, ws_floats * 4);
+                if (!hd) fl[i] &= ~W_HEAD;
+                if (!tl) fl[i] &= ~W_HAND;
                 hm[i] = hd ? hr[j] : -1e30f;
                 hl[i] = hd ? hr[8 + j] : 0.f;
-                ho[i] = hd ? hr[16 + j * 128 + c] : 0.f;
+                ho[i] = hd ? ld4(hr + 16 + j * 128 + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
                 hdot[i] = tl ? hh[j] * sl2 : 0.f;
-                hval[i] = tl ? hh[8 + c] : 0.f;
+                hval[i] = tl ? ld4(hh + 8 + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
         if constexpr (SEGS) {
@@ -1653,12 +1681,12 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
             for (int i = 0; i < BATCH; ++i) {
                 if (fl[i] & W_HEAD) {
                     hm[i] += cdot;
-                    ho[i] = fmaf(hl[i], cval, ho[i]);
+                    ho[i] = fma4(cval, hl[i], ho[i]);
                 }
                 if (fl[i] & W_HAND) {
                     const bool rel = fl[i] & W_REL;
                     cdot = rel ? cdot + hdot[i] : hdot[i];
-                    cval = rel ? cval + hval[i] : hval[i];
+                    cval = rel ? fma4(hval[i], 1.f, cval) : hval[i];
                 }
             }
         }
@@ -1670,21 +1698,39 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
         }
         const float sc = exp2f(M - Mn);
         L *= sc;
-        O *= sc;
+        O = make_float4(O.x * sc, O.y * sc, O.z * sc, O.w * sc);
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
             const float e = exp2f(mv[i] - Mn);
             L = fmaf(lv[i], e, L);
-            O = fmaf(ov[i], e, O);
+            O = fma4(ov[i], e, O);
             if constexpr (SEGS) {
                 const float eh = exp2f(hm[i] - Mn);
                 L = fmaf(hl[i], eh, L);
-                O = fmaf(ho[i], eh, O);
+                O = fma4(ho[i], eh, O);
             }
         }
         M = Mn;
     }
-    dst[c] = L > 0.f ? O / L : 0.f;     // a causal query with no position gets 0
+    // merge the four quarters (log-sum-exp), one channel per thread
+    __shared__ float q_m[4], q_l[4];
+    __shared__ float4 q_o[4][32];
+    if (lane == 0) { q_m[wq] = M; q_l[wq] = L; }
+    q_o[wq][lane] = O;
+    __syncthreads();
+    float Mx = q_m[0];
+#pragma unroll
+    for (int q = 1; q < 4; ++q) Mx = fmaxf(Mx, q_m[q]);
+    float Lt = 0.f, Ot = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float e = exp2f(q_m[q] - Mx);
+        const float4 v = q_o[q][c >> 2];
+        const float oc = (c & 3) == 0 ? v.x : (c & 3) == 1 ? v.y : (c & 3) == 2 ? v.z : v.w;
+        Lt = fmaf(q_l[q], e, Lt);
+        Ot = fmaf(oc, e, Ot);
+    }
+    dst[c] = Lt > 0.f ? Ot / Lt : 0.f;  // a causal query with no position gets 0
 }
 
 template <bool FIN, bool SEGS, int BATCH>
@@ -1910,20 +1956,12 @@ cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const 
         // a flag byte for each warp slot a sequence can span
         const size_t fl = (size_t)(NW + 15) / 16 * 16;
         if (fl > 48 * 1024) return cudaErrorInvalidConfiguration;
-        // 16 records per round trip need about 160 registers (3 blocks per SM):
-        // when the grid is larger than that wave, 8 per round trip (92)
-        int dev = 0, nsm = 0;
-        cudaError_t e2 = cudaGetDevice(&dev);
-        if (e2 == cudaSuccess) e2 = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-        if (e2 != cudaSuccess) return e2;
-        const bool big = (int64_t)grid.x * grid.y <= 3 * (int64_t)nsm;
-        if (cv.len_add > 0) {
-            if (big) merge_kernel<true, true, 16><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
-            else merge_kernel<true, true, 8><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
-        } else {
-            if (big) merge_kernel<false, true, 16><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
-            else merge_kernel<false, true, 8><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
-        }
+        if (cv.len_add > 0)
+            merge_kernel<true, true, DKV_MERGE_BATCH><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW,
+                                                                             ws, ws_floats, out);
+        else
+            merge_kernel<false, true, DKV_MERGE_BATCH><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW,
+                                                                              ws, ws_floats, out);
     } else if (cv.len_add > 0) {
         merge_kernel<true, false, DKV_MERGE_BATCH><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws,
                                                                          ws_floats, out);
