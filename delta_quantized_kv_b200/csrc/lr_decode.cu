@@ -10,8 +10,10 @@
 //   q . k^_p   = (1/|R_p|) sum_{r in R_p} (q . k^_r) + q . delta^K_p
 //   sum_p w_p v^_p = sum_r W_r v^_r + sum_p w_p delta^V_p,
 //   W_r = sum_{p : r in R^V_p} w_p / |R^V_p|  (+ w_p for the reference token p = r s).
-// Three launches:
-//  1. refdot: q . k^_r for every stored K reference (1/stride of the tokens).
+// Four launches:
+//  1. refdot: q . k^_r for every stored K reference (1/stride of the tokens);
+//     refmean: every token's reference part of its score (the mean of its
+//     references' dots), written where the split kernel completes the score.
 //  2. split: one warp per 256-token chunk of a sequence.  Each 32-token tile's
 //     codes are staged in shared memory as exact fp16 (code - 8); the K side
 //     is an MMA with the tokens as rows (ldmatrix), the scores add the mean of
@@ -152,6 +154,18 @@ __device__ inline float2 lrd_refpart(const LrdArgs &a, int seq, int p, int h0) {
     return make_float2(s0 * inv, s1 * inv);
 }
 
+// 1b. The reference part of every token's score, into S (the split kernel
+//     adds the token's own residual dot): one thread per (token, head pair).
+__global__ void __launch_bounds__(256) lrd_refmean_kernel(LrdArgs a) {
+    const int seq = blockIdx.y, b = seq / a.Hkv;
+    const int len = lrd_len(a, b);
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // token * 4 + head pair
+    const int p = (int)(i >> 2), hp = (int)(i & 3);
+    if (p >= len) return;
+    const float2 rp = lrd_refpart(a, seq, p, 2 * hp);
+    *reinterpret_cast<float2 *>(a.S + ((int64_t)seq * a.T + p) * 8 + 2 * hp) = rp;
+}
+
 // ---------------------------------------------------------------------------
 // 2. split: one warp per (sequence, 256-token chunk).  QHL: fp32 queries as
 //    an fp16 hi + lo pair.
@@ -223,7 +237,7 @@ __global__ void __launch_bounds__(LRD_WARPS * 32) lrd_split_kernel(LrdArgs a) {
                 float2 rp = make_float2(0.f, 0.f);
                 if (p < pe) {
                     sc = *reinterpret_cast<const uint2 *>(a.k.scales + (row0 + p) * NB);
-                    rp = lrd_refpart(a, seq, p, 2 * tq);
+                    rp = *reinterpret_cast<const float2 *>(a.S + (row0 + p) * 8 + 2 * tq);
                 }
                 const float d0 = h_lo(sc.x), d1 = h_hi(sc.x), d2 = h_lo(sc.y), d3 = h_hi(sc.y);
 #pragma unroll
@@ -342,9 +356,14 @@ __global__ void __launch_bounds__(LRD_WARPS * 32) lrd_split_kernel(LrdArgs a) {
 // 3. combine: one block per sequence.
 // ---------------------------------------------------------------------------
 constexpr int LRD_COMBINE_THREADS = 256;
+// W_r of a sequence read back into shared memory for the final sum when NR x 8
+// floats fit in the default 48 KB of dynamic shared memory
+constexpr int LRD_W_SMEM_MAX = 48 * 1024;
 
+template <bool WSM>
 __global__ void __launch_bounds__(LRD_COMBINE_THREADS) lrd_combine_kernel(LrdArgs a) {
     __shared__ float Mh[8], Lh[8];
+    extern __shared__ float w_sm[];              // WSM: [NR][8]
     const int seq = blockIdx.x, b = seq / a.Hkv, kvh = seq % a.Hkv;
     const int len = lrd_len(a, b);
     const int nch = (len + LRD_CHUNK - 1) / LRD_CHUNK;
@@ -389,18 +408,28 @@ __global__ void __launch_bounds__(LRD_COMBINE_THREADS) lrd_combine_kernel(LrdArg
     }
     __threadfence_block();
     __syncthreads();
+    // (WSM) the sequence's W_r once into shared memory: the sum below reads
+    // each of them for every output element
+    const float *Wr = W;
+    if constexpr (WSM) {
+        for (int i = tid; i < nr * 8; i += blockDim.x) w_sm[i] = __ldcg(W + i);
+        __syncthreads();
+        Wr = w_sm;
+    }
     // out = merged delta part + sum_r W_r v^_r
     const uint16_t *rv = a.v.ref_values + (int64_t)seq * a.NR * D;
     for (int i = tid; i < a.G * D; i += blockDim.x) {
         const int h = i / D, c = i % D;
         float acc = 0.f;
+#pragma unroll 4
         for (int ch = 0; ch < nch; ++ch) {
             const float *rec = part + (int64_t)ch * LRD_PARTIAL;
             acc = fmaf(rec[16 + h * D + c], exp2f(rec[h] - Mh[h]), acc);
         }
         acc /= Lh[h];
+#pragma unroll 8
         for (int r = 0; r < nr; ++r)
-            acc = fmaf(__ldcg(W + (int64_t)r * 8 + h),
+            acc = fmaf(WSM ? Wr[r * 8 + h] : __ldcg(W + (int64_t)r * 8 + h),
                        __half2float(__ushort_as_half(rv[(int64_t)r * D + c])), acc);
         out[(int64_t)h * D + c] = acc;
     }
@@ -433,6 +462,10 @@ cudaError_t launch_lr_decode(const LrdView &K, const LrdView &V, int B, int Hkv,
     lrd_refdot_kernel<<<g1, LRD_WARPS * 32, 0, st>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    dim3 g2((unsigned)(((int64_t)T * 4 + 255) / 256), (unsigned)nseq);
+    lrd_refmean_kernel<<<g2, 256, 0, st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     const int64_t warps = nseq * a.n_chunks;
     const unsigned ctas = (unsigned)((warps + LRD_WARPS - 1) / LRD_WARPS);
     const size_t smem = (size_t)LRD_WARPS * 2 * LRD_TILE * LRD_ROW * sizeof(__half);
@@ -448,7 +481,11 @@ cudaError_t launch_lr_decode(const LrdView &K, const LrdView &V, int B, int Hkv,
     if (e != cudaSuccess) return e;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    lrd_combine_kernel<<<(unsigned)nseq, LRD_COMBINE_THREADS, 0, st>>>(a);
+    const size_t wsm = (size_t)a.NR * 8 * sizeof(float);
+    if (wsm <= (size_t)LRD_W_SMEM_MAX)
+        lrd_combine_kernel<true><<<(unsigned)nseq, LRD_COMBINE_THREADS, wsm, st>>>(a);
+    else
+        lrd_combine_kernel<false><<<(unsigned)nseq, LRD_COMBINE_THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 
