@@ -10,7 +10,7 @@
 //   q . k^_p   = (1/|R_p|) sum_{r in R_p} (q . k^_r) + q . delta^K_p
 //   sum_p w_p v^_p = sum_r W_r v^_r + sum_p w_p delta^V_p,
 //   W_r = sum_{p : r in R^V_p} w_p / |R^V_p|  (+ w_p for the reference token p = r s).
-// Four launches:
+// Five launches:
 //  1. refdot: q . k^_r for every stored K reference (1/stride of the tokens);
 //     refmean: every token's reference part of its score (the mean of its
 //     references' dots), written where the split kernel completes the score.
@@ -21,9 +21,10 @@
 //     channels as rows (ldmatrix.trans) against the weights times the V
 //     scales, each an fp16 hi + lo pair.  The raw scores are kept for step 3,
 //     and a partial (max, sum, output) record per chunk.
-//  3. combine: one block per sequence: log-sum-exp over the chunks, the final
-//     weight of every token scattered onto its V references (W_r), then
-//     out = the merged delta part + sum_r W_r v^_r.
+//  3. combine, in two launches: log-sum-exp over the chunks and the final
+//     weight of every token scattered onto its V references (W_r), one block
+//     per chunk; then out = the merged delta part + sum_r W_r v^_r, one block
+//     per head.
 // Inputs are the canonical layouts dkv_lr_encode writes.
 #include <cstdint>
 
@@ -160,6 +161,9 @@ __global__ void __launch_bounds__(256) lrd_refmean_kernel(LrdArgs a) {
     const int seq = blockIdx.y, b = seq / a.Hkv;
     const int len = lrd_len(a, b);
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // token * 4 + head pair
+    // the sequence's reference weights W_r start at 0 (the combine adds to them)
+    for (int64_t k = i; k < (int64_t)a.NR * 8; k += (int64_t)gridDim.x * blockDim.x)
+        a.W[(int64_t)seq * a.NR * 8 + k] = 0.f;
     const int p = (int)(i >> 2), hp = (int)(i & 3);
     if (p >= len) return;
     const float2 rp = lrd_refpart(a, seq, p, 2 * hp);
@@ -353,44 +357,40 @@ __global__ void __launch_bounds__(LRD_WARPS * 32) lrd_split_kernel(LrdArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// 3. combine: one block per sequence.
+// 3. combine, in two launches.
+//  weights: one block per (256-token chunk, sequence): the log-sum-exp over
+//    the sequence's chunks, then the final weight of each of the chunk's
+//    tokens added onto its V references (W_r, zeroed by refmean).
+//  output: one block per (head, sequence), one thread per channel: the merged
+//    delta part plus sum_r W_r v^_r (the head's W_r read once into shared
+//    memory when they fit).
 // ---------------------------------------------------------------------------
-constexpr int LRD_COMBINE_THREADS = 256;
-// W_r of a sequence read back into shared memory for the final sum when NR x 8
-// floats fit in the default 48 KB of dynamic shared memory
-constexpr int LRD_W_SMEM_MAX = 48 * 1024;
+// Log-sum-exp statistics of head h over the nch chunk records of a sequence:
+// the largest chunk maximum M and the sum L of the chunk sums rescaled to it.
+__device__ inline void lrd_lse(const float *part, int nch, int h, float &M, float &L) {
+    M = -INFINITY;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, part[(int64_t)c * LRD_PARTIAL + h]);
+    L = 0.f;
+    for (int c = 0; c < nch; ++c)
+        L += part[(int64_t)c * LRD_PARTIAL + 8 + h] * exp2f(part[(int64_t)c * LRD_PARTIAL + h] - M);
+}
 
-template <bool WSM>
-__global__ void __launch_bounds__(LRD_COMBINE_THREADS) lrd_combine_kernel(LrdArgs a) {
+constexpr int LRD_WEIGHT_THREADS = 256;
+
+__global__ void __launch_bounds__(LRD_WEIGHT_THREADS) lrd_weights_kernel(LrdArgs a) {
     __shared__ float Mh[8], Lh[8];
-    extern __shared__ float w_sm[];              // WSM: [NR][8]
-    const int seq = blockIdx.x, b = seq / a.Hkv, kvh = seq % a.Hkv;
+    const int chunk = blockIdx.x, seq = blockIdx.y, b = seq / a.Hkv;
     const int len = lrd_len(a, b);
+    const int pb = chunk * LRD_CHUNK, pe = min(len, pb + LRD_CHUNK);
+    if (pb >= pe) return;                                   // uniform over the block
     const int nch = (len + LRD_CHUNK - 1) / LRD_CHUNK;
-    const int nr = (len + a.s - 1) / a.s;
-    const int tid = threadIdx.x;
-    float *out = a.out + ((int64_t)b * a.Hq + kvh * a.G) * D;
-    if (len == 0) {                                    // uniform over the block
-        for (int i = tid; i < a.G * D; i += blockDim.x) out[i] = 0.f;
-        return;
-    }
     const float *part = a.part + (int64_t)seq * a.n_chunks * LRD_PARTIAL;
-    if (tid < a.G) {
-        float M = -INFINITY;
-        for (int c = 0; c < nch; ++c) M = fmaxf(M, part[(int64_t)c * LRD_PARTIAL + tid]);
-        float L = 0.f;
-        for (int c = 0; c < nch; ++c)
-            L += part[(int64_t)c * LRD_PARTIAL + 8 + tid] * exp2f(part[(int64_t)c * LRD_PARTIAL + tid] - M);
-        Mh[tid] = M;
-        Lh[tid] = L;
-    }
-    float *W = a.W + (int64_t)seq * a.NR * 8;
-    for (int i = tid; i < nr * 8; i += blockDim.x) W[i] = 0.f;
+    if ((int)threadIdx.x < a.G) lrd_lse(part, nch, threadIdx.x, Mh[threadIdx.x], Lh[threadIdx.x]);
     __syncthreads();
-    // the final weight of every token, onto its V references
+    float *W = a.W + (int64_t)seq * a.NR * 8;
     const int32_t *vref = a.v.ref + (int64_t)seq * a.T * a.m;
     const float *S = a.S + (int64_t)seq * a.T * 8;
-    for (int p = tid; p < len; p += blockDim.x) {
+    for (int p = pb + threadIdx.x; p < pe; p += blockDim.x) {
         const bool isref = p % a.s == 0;
         int me = 0;
         if (!isref)
@@ -406,33 +406,49 @@ __global__ void __launch_bounds__(LRD_COMBINE_THREADS) lrd_combine_kernel(LrdArg
             }
         }
     }
-    __threadfence_block();
+}
+
+// The head's W_r in shared memory when NR floats fit in the default 48 KB.
+constexpr int LRD_W_SMEM_MAX = 48 * 1024;
+
+template <bool WSM>
+__global__ void __launch_bounds__(D) lrd_out_kernel(LrdArgs a) {
+    extern __shared__ float w_sm[];                         // WSM: [NR]
+    __shared__ float Ms, Ls;
+    const int h = blockIdx.x, seq = blockIdx.y, b = seq / a.Hkv, kvh = seq % a.Hkv;
+    const int len = lrd_len(a, b), c = threadIdx.x;
+    float *out = a.out + ((int64_t)b * a.Hq + kvh * a.G + h) * D;
+    if (len == 0) {                                         // uniform over the block
+        out[c] = 0.f;
+        return;
+    }
+    const int nch = (len + LRD_CHUNK - 1) / LRD_CHUNK;
+    const int nr = (len + a.s - 1) / a.s;
+    const float *part = a.part + (int64_t)seq * a.n_chunks * LRD_PARTIAL;
+    if (c == 0) {
+        float M, L;
+        lrd_lse(part, nch, h, M, L);
+        Ms = M;
+        Ls = L;
+    }
+    const float *W = a.W + (int64_t)seq * a.NR * 8;
+    if constexpr (WSM)
+        for (int r = c; r < nr; r += blockDim.x) w_sm[r] = W[(int64_t)r * 8 + h];
     __syncthreads();
-    // (WSM) the sequence's W_r once into shared memory: the sum below reads
-    // each of them for every output element
-    const float *Wr = W;
-    if constexpr (WSM) {
-        for (int i = tid; i < nr * 8; i += blockDim.x) w_sm[i] = __ldcg(W + i);
-        __syncthreads();
-        Wr = w_sm;
-    }
     // out = merged delta part + sum_r W_r v^_r
-    const uint16_t *rv = a.v.ref_values + (int64_t)seq * a.NR * D;
-    for (int i = tid; i < a.G * D; i += blockDim.x) {
-        const int h = i / D, c = i % D;
-        float acc = 0.f;
+    float acc = 0.f;
 #pragma unroll 4
-        for (int ch = 0; ch < nch; ++ch) {
-            const float *rec = part + (int64_t)ch * LRD_PARTIAL;
-            acc = fmaf(rec[16 + h * D + c], exp2f(rec[h] - Mh[h]), acc);
-        }
-        acc /= Lh[h];
-#pragma unroll 8
-        for (int r = 0; r < nr; ++r)
-            acc = fmaf(WSM ? Wr[r * 8 + h] : __ldcg(W + (int64_t)r * 8 + h),
-                       __half2float(__ushort_as_half(rv[(int64_t)r * D + c])), acc);
-        out[(int64_t)h * D + c] = acc;
+    for (int ch = 0; ch < nch; ++ch) {
+        const float *rec = part + (int64_t)ch * LRD_PARTIAL;
+        acc = fmaf(rec[16 + h * D + c], exp2f(rec[h] - Ms), acc);
     }
+    acc /= Ls;
+    const uint16_t *rv = a.v.ref_values + (int64_t)seq * a.NR * D;
+#pragma unroll 8
+    for (int r = 0; r < nr; ++r)
+        acc = fmaf(WSM ? w_sm[r] : W[(int64_t)r * 8 + h],
+                   __half2float(__ushort_as_half(rv[(int64_t)r * D + c])), acc);
+    out[c] = acc;
 }
 
 size_t lrd_workspace_floats(int B, int Hkv, int T, int s) {
@@ -481,11 +497,14 @@ cudaError_t launch_lr_decode(const LrdView &K, const LrdView &V, int B, int Hkv,
     if (e != cudaSuccess) return e;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t wsm = (size_t)a.NR * 8 * sizeof(float);
+    lrd_weights_kernel<<<dim3((unsigned)a.n_chunks, (unsigned)nseq), LRD_WEIGHT_THREADS, 0, st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t wsm = (size_t)a.NR * sizeof(float);
     if (wsm <= (size_t)LRD_W_SMEM_MAX)
-        lrd_combine_kernel<true><<<(unsigned)nseq, LRD_COMBINE_THREADS, wsm, st>>>(a);
+        lrd_out_kernel<true><<<dim3((unsigned)a.G, (unsigned)nseq), D, wsm, st>>>(a);
     else
-        lrd_combine_kernel<false><<<(unsigned)nseq, LRD_COMBINE_THREADS, 0, st>>>(a);
+        lrd_out_kernel<false><<<dim3((unsigned)a.G, (unsigned)nseq), D, 0, st>>>(a);
     return cudaGetLastError();
 }
 
