@@ -14,7 +14,8 @@
 //  1. refdot: q . k^_r for every stored K reference (1/stride of the tokens);
 //     refmean: every token's reference part of its score (the mean of its
 //     references' dots), written where the split kernel completes the score.
-//  2. split: one warp per 256-token chunk of a sequence.  Each 32-token tile's
+//  2. split: one warp per chunk of a sequence (sized so the grid fills one
+//     wave; at least 128 tokens).  Each 32-token tile's
 //     codes are staged in shared memory as exact fp16 (code - 8); the K side
 //     is an MMA with the tokens as rows (ldmatrix), the scores add the mean of
 //     the reference dots; online softmax; the V side is an MMA with the
@@ -34,7 +35,8 @@
 namespace dkv {
 
 constexpr int LRD_TILE = 32;                // tokens per staged tile
-constexpr int LRD_CHUNK = 256;              // tokens per split warp
+constexpr int LRD_CHUNK_MIN = 128;          // tokens per split warp, at least (the host sizes
+                                            // chunks so the split grid fills one wave)
 constexpr int LRD_WARPS = 4;
 constexpr int LRD_ROW = D + 8;              // staged row stride (halves): 272 B, conflict-free
 constexpr int LRD_PARTIAL = 8 + 8 + 8 * D;  // m[8], l[8], o[8][128]
@@ -49,6 +51,7 @@ struct LrdTensor {
 struct LrdArgs {
     LrdTensor k, v;
     int B, Hkv, T, s, m, Hq, G, NR, n_chunks;
+    int chunk;                   // tokens per split warp (a multiple of LRD_TILE)
     const int32_t *lens;         // [B] device
     const void *Q;
     int q_dtype;
@@ -171,7 +174,7 @@ __global__ void __launch_bounds__(256) lrd_refmean_kernel(LrdArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// 2. split: one warp per (sequence, 256-token chunk).  QHL: fp32 queries as
+// 2. split: one warp per (sequence, chunk of a.chunk tokens).  QHL: fp32 queries as
 //    an fp16 hi + lo pair.
 // ---------------------------------------------------------------------------
 template <bool QHL>
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(LRD_WARPS * 32) lrd_split_kernel(LrdArgs a) {
     const int seq = (int)(item / a.n_chunks), chunk = (int)(item % a.n_chunks);
     const int b = seq / a.Hkv, kvh = seq % a.Hkv;
     const int len = lrd_len(a, b);
-    const int pb = chunk * LRD_CHUNK, pe = min(len, pb + LRD_CHUNK);
+    const int pb = chunk * a.chunk, pe = min(len, pb + a.chunk);
     if (pb >= pe) return;
     __half *Kc = reinterpret_cast<__half *>(lrd_smem) + warp * 2 * LRD_TILE * LRD_ROW;
     __half *Vc = Kc + LRD_TILE * LRD_ROW;
@@ -358,7 +361,7 @@ __global__ void __launch_bounds__(LRD_WARPS * 32) lrd_split_kernel(LrdArgs a) {
 
 // ---------------------------------------------------------------------------
 // 3. combine, in two launches.
-//  weights: one block per (256-token chunk, sequence): the log-sum-exp over
+//  weights: one block per (chunk, sequence): the log-sum-exp over
 //    the sequence's chunks, then the final weight of each of the chunk's
 //    tokens added onto its V references (W_r, zeroed by refmean).
 //  output: one block per (head, sequence), one thread per channel: the merged
@@ -381,9 +384,9 @@ __global__ void __launch_bounds__(LRD_WEIGHT_THREADS) lrd_weights_kernel(LrdArgs
     __shared__ float Mh[8], Lh[8];
     const int chunk = blockIdx.x, seq = blockIdx.y, b = seq / a.Hkv;
     const int len = lrd_len(a, b);
-    const int pb = chunk * LRD_CHUNK, pe = min(len, pb + LRD_CHUNK);
+    const int pb = chunk * a.chunk, pe = min(len, pb + a.chunk);
     if (pb >= pe) return;                                   // uniform over the block
-    const int nch = (len + LRD_CHUNK - 1) / LRD_CHUNK;
+    const int nch = (len + a.chunk - 1) / a.chunk;
     const float *part = a.part + (int64_t)seq * a.n_chunks * LRD_PARTIAL;
     if ((int)threadIdx.x < a.G) lrd_lse(part, nch, threadIdx.x, Mh[threadIdx.x], Lh[threadIdx.x]);
     __syncthreads();
@@ -422,7 +425,7 @@ __global__ void __launch_bounds__(D) lrd_out_kernel(LrdArgs a) {
         out[c] = 0.f;
         return;
     }
-    const int nch = (len + LRD_CHUNK - 1) / LRD_CHUNK;
+    const int nch = (len + a.chunk - 1) / a.chunk;
     const int nr = (len + a.s - 1) / a.s;
     const float *part = a.part + (int64_t)seq * a.n_chunks * LRD_PARTIAL;
     if (c == 0) {
@@ -453,7 +456,7 @@ __global__ void __launch_bounds__(D) lrd_out_kernel(LrdArgs a) {
 
 size_t lrd_workspace_floats(int B, int Hkv, int T, int s) {
     const int64_t nseq = (int64_t)B * Hkv, NR = (T + s - 1) / s;
-    const int64_t nch = (T + LRD_CHUNK - 1) / LRD_CHUNK;
+    const int64_t nch = (T + LRD_CHUNK_MIN - 1) / LRD_CHUNK_MIN;
     return (size_t)(nseq * NR * 8 * 2 + nseq * (int64_t)T * 8 + nseq * nch * LRD_PARTIAL);
 }
 
@@ -465,7 +468,6 @@ cudaError_t launch_lr_decode(const LrdView &K, const LrdView &V, int B, int Hkv,
     a.v = LrdTensor{V.ref, V.ref_values, V.scales, V.codes};
     a.B = B; a.Hkv = Hkv; a.T = T; a.s = s; a.m = m; a.Hq = Hq; a.G = Hq / Hkv;
     a.NR = (T + s - 1) / s;
-    a.n_chunks = (T + LRD_CHUNK - 1) / LRD_CHUNK;
     a.lens = lens; a.Q = Q; a.q_dtype = q_dtype;
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
     const int64_t nseq = (int64_t)B * Hkv;
@@ -482,19 +484,31 @@ cudaError_t launch_lr_decode(const LrdView &K, const LrdView &V, int B, int Hkv,
     lrd_refmean_kernel<<<g2, 256, 0, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    // chunks sized so that the split grid fills one wave of resident warps:
+    // chunks per sequence = resident warps / sequences, whole 32-token tiles,
+    // at least LRD_CHUNK_MIN tokens (the workspace is sized for that)
+    const size_t smem = (size_t)LRD_WARPS * 2 * LRD_TILE * LRD_ROW * sizeof(__half);
+    const void *split_fn = q_dtype == DKV_F32 ? (const void *)lrd_split_kernel<true>
+                                              : (const void *)lrd_split_kernel<false>;
+    e = cudaFuncSetAttribute(split_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0, dev = 0, nsm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_fn, LRD_WARPS * 32, smem);
+    if (e == cudaSuccess) e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int64_t resident = (int64_t)(per_sm < 1 ? 1 : per_sm) * nsm * LRD_WARPS;
+    const int64_t per_seq = resident / nseq > 1 ? resident / nseq : 1;
+    int64_t chunk = (T + per_seq - 1) / per_seq;
+    chunk = (chunk + LRD_TILE - 1) / LRD_TILE * LRD_TILE;
+    a.chunk = (int)(chunk < LRD_CHUNK_MIN ? LRD_CHUNK_MIN : chunk);
+    a.n_chunks = (T + a.chunk - 1) / a.chunk;
     const int64_t warps = nseq * a.n_chunks;
     const unsigned ctas = (unsigned)((warps + LRD_WARPS - 1) / LRD_WARPS);
-    const size_t smem = (size_t)LRD_WARPS * 2 * LRD_TILE * LRD_ROW * sizeof(__half);
-    if (q_dtype == DKV_F32) {
-        e = cudaFuncSetAttribute(lrd_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e == cudaSuccess) lrd_split_kernel<true><<<ctas, LRD_WARPS * 32, smem, st>>>(a);
-    } else {
-        e = cudaFuncSetAttribute(lrd_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e == cudaSuccess) lrd_split_kernel<false><<<ctas, LRD_WARPS * 32, smem, st>>>(a);
-    }
-    if (e != cudaSuccess) return e;
+    if (q_dtype == DKV_F32)
+        lrd_split_kernel<true><<<ctas, LRD_WARPS * 32, smem, st>>>(a);
+    else
+        lrd_split_kernel<false><<<ctas, LRD_WARPS * 32, smem, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     lrd_weights_kernel<<<dim3((unsigned)a.n_chunks, (unsigned)nseq), LRD_WEIGHT_THREADS, 0, st>>>(a);
