@@ -1023,6 +1023,11 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        # N replicas hold N GPUs for the whole run: the untimed extras (other
+        # workloads, comparator formats, quality report) and the host-core
+        # oracle baseline belong to the single-GPU run only
+        args.cpu_baseline = args.comparators = args.configs = False
 
     import synthetic as S
     w = S.WORKLOADS[args.workload]
