@@ -805,18 +805,23 @@ def run_ours(args, w, rank, world, local):
     peak, peak_kind = measured_peak()
 
     # ---- end to end through the public API with host buffers ------------------
-    pin_k = [t.cpu().pin_memory() for t in app_k[O_E2E:]]
-    pin_v = [t.cpu().pin_memory() for t in app_v[O_E2E:]]
-    pin_q = [t.cpu().pin_memory() for t in qs[O_E2E:]]
-    dk = torch.empty_like(app_k[0]); dv = torch.empty_like(app_v[0]); dq = torch.empty_like(qs[0])
+    # each step's inputs (K_new | V_new | q) packed in one pinned host buffer
+    # and moved by one H2D copy into one device buffer that they view
+    parts0 = (app_k[0], app_v[0], qs[0])
+    nbytes = [t.numel() * t.element_size() for t in parts0]
+    offs = [0, nbytes[0], nbytes[0] + nbytes[1]]
+    h2d = sum(nbytes)
+    pins = []
+    for j in range(len(qs) - O_E2E):
+        ts = (app_k[O_E2E + j], app_v[O_E2E + j], qs[O_E2E + j])
+        pins.append(torch.cat([t.contiguous().view(-1).view(torch.uint8) for t in ts]).cpu().pin_memory())
+    dbuf = torch.empty(h2d, dtype=torch.uint8, device=dev)
+    dk, dv, dq = (dbuf[o:o + n].view(t.dtype).view(t.shape) for o, n, t in zip(offs, nbytes, parts0))
     host_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
-    h2d = pin_k[0].numel() * pin_k[0].element_size() * 2 + pin_q[0].numel() * pin_q[0].element_size()
     d2h = host_out.numel() * 4
 
     def e2e_step(j):
-        dk.copy_(pin_k[j], non_blocking=True)
-        dv.copy_(pin_v[j], non_blocking=True)
-        dq.copy_(pin_q[j], non_blocking=True)
+        dbuf.copy_(pins[j], non_blocking=True)
         cache.append(dk, dv)
         cache.decode_attn(dq, scale, out=out)
         host_out.copy_(out, non_blocking=True)
@@ -985,7 +990,9 @@ def run_ours(args, w, rank, world, local):
         "encode": res["encode"],
         "append": res["append"],
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "launch": "per step: one H2D copy of the packed inputs from pinned memory, "
+                          "append, decode, D2H of the output, issued one by one"},
         "gpu_launches": 3 * K,
         "clocks": clocks,
         "clocks_kernel_timing": clk_eager.summary(),

@@ -1101,6 +1101,8 @@ __global__ void __launch_bounds__(WARPS * 32, (QHL ? 2 : KCfg<FMT, MODE>::MINB))
         reinterpret_cast<uint4 *>(mystages)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async();
     __syncwarp();
+    pdl_trigger();
+    pdl_wait();           // every global access below follows the previous kernel
 
     const int64_t NW = (int64_t)gridDim.x * WARPS;
     const int64_t gw = (int64_t)blockIdx.x * WARPS + warp;
@@ -1738,6 +1740,8 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
                                                     int64_t NW, const float *ws, int64_t ws_floats,
                                                     float *out) {
     extern __shared__ uint8_t merge_flags[];        // SEGS: one byte per warp slot
+    pdl_trigger();
+    pdl_wait();                                     // the split kernel's records
     merge_body<FIN, SEGS, BATCH>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out, merge_flags);
     if constexpr (FIN) {
         // fused append: publish batch entry b's new length (no other block of
@@ -1857,9 +1861,8 @@ static cudaError_t launch_inst(const SplitArgs &a, int ctas, cudaStream_t st) {
             }
         }
     }
-    split_kernel<FMT, MODE, ZT, PAGED, MQ, APP, QHL, RC>
-        <<<ctas, WARPS * 32, split_smem<FMT, MODE>(), st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(split_kernel<FMT, MODE, ZT, PAGED, MQ, APP, QHL, RC>, dim3(ctas),
+                      dim3(WARPS * 32), split_smem<FMT, MODE>(), st, a);
 }
 
 // fp32 queries take the hi + lo instance
@@ -1957,19 +1960,19 @@ cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const 
         const size_t fl = (size_t)(NW + 15) / 16 * 16;
         if (fl > 48 * 1024) return cudaErrorInvalidConfiguration;
         if (cv.len_add > 0)
-            merge_kernel<true, true, DKV_MERGE_BATCH><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW,
-                                                                             ws, ws_floats, out);
+            e = launch_pdl(merge_kernel<true, true, DKV_MERGE_BATCH>, grid, dim3(128), fl, st,
+                           cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out);
         else
-            merge_kernel<false, true, DKV_MERGE_BATCH><<<grid, 128, fl, st>>>(cv, Hq, G, NHG, nq, NW,
-                                                                              ws, ws_floats, out);
+            e = launch_pdl(merge_kernel<false, true, DKV_MERGE_BATCH>, grid, dim3(128), fl, st,
+                           cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out);
     } else if (cv.len_add > 0) {
-        merge_kernel<true, false, DKV_MERGE_BATCH><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws,
-                                                                         ws_floats, out);
+        e = launch_pdl(merge_kernel<true, false, DKV_MERGE_BATCH>, grid, dim3(128), 0, st,
+                       cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out);
     } else {
-        merge_kernel<false, false, DKV_MERGE_BATCH><<<grid, 128, 0, st>>>(cv, Hq, G, NHG, nq, NW, ws,
-                                                                          ws_floats, out);
+        e = launch_pdl(merge_kernel<false, false, DKV_MERGE_BATCH>, grid, dim3(128), 0, st,
+                       cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out);
     }
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace dkv

@@ -177,6 +177,34 @@ __device__ inline void fence_proxy_async() {
 __device__ inline void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;\n" ::: "memory");
 }
+
+// Programmatic dependent launch.  The library's step kernels (append, decode
+// split, merge) are launched with programmatic stream serialization, so each
+// may be scheduled while the kernel before it in the stream still runs.
+// pdl_wait() returns once every kernel before it in the stream has completed
+// and its global writes are visible: each of those kernels calls it before its
+// first global access, so the order of the stream holds for memory.  It
+// returns at once in a launch without that attribute.  pdl_trigger() lets the
+// next such kernel be scheduled; it orders nothing.
+__device__ inline void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ inline void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// host side: a launch with programmatic stream serialization allowed
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 __device__ inline void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
                  "r"(bytes)

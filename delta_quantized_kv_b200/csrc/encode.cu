@@ -70,6 +70,8 @@ template <int FMT>
 __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
     __shared__ uint8_t codes[SEG][D];
     __shared__ __half scl[SEG][NB];
+    pdl_trigger();
+    pdl_wait();           // every global access below follows the previous kernel
     const CacheView &cv = a.cv;
     const int b = blockIdx.z, kvh = blockIdx.y >> 1, t = blockIdx.y & 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -677,11 +679,10 @@ cudaError_t launch_encode(const CacheView &cv, const void *K, const void *V, int
     items = items < 1 ? 1 : items;
     dim3 grid(items, cv.Hkv * 2, cv.B);
     switch (cv.fmt) {
-        case DKV_FMT_DELTA: encode_kernel<DKV_FMT_DELTA><<<grid, 128, 0, st>>>(a); break;
-        case DKV_FMT_Q4_0: encode_kernel<DKV_FMT_Q4_0><<<grid, 128, 0, st>>>(a); break;
-        default: encode_kernel<DKV_FMT_FP16><<<grid, 128, 0, st>>>(a); break;
+        case DKV_FMT_DELTA: return launch_pdl(encode_kernel<DKV_FMT_DELTA>, grid, dim3(128), 0, st, a);
+        case DKV_FMT_Q4_0: return launch_pdl(encode_kernel<DKV_FMT_Q4_0>, grid, dim3(128), 0, st, a);
+        default: return launch_pdl(encode_kernel<DKV_FMT_FP16>, grid, dim3(128), 0, st, a);
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_readback(const CacheView &cv, uint8_t *codes, uint16_t *scales,
