@@ -1736,9 +1736,8 @@ __device__ inline void merge_body(const CacheView &cv, int Hq, int G, int NHG, i
 }
 
 template <bool FIN, bool SEGS, int BATCH>
-__global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G, int NHG, int nq,
-                                                    int64_t NW, const float *ws, int64_t ws_floats,
-                                                    float *out) {
+__device__ inline void merge_entry(const CacheView &cv, int Hq, int G, int NHG, int nq, int64_t NW,
+                                   const float *ws, int64_t ws_floats, float *out) {
     extern __shared__ uint8_t merge_flags[];        // SEGS: one byte per warp slot
     pdl_trigger();
     pdl_wait();                                     // the split kernel's records
@@ -1753,6 +1752,25 @@ __global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G,
             if (blockIdx.y == 0) cv.header[2] ^= 1;
         }
     }
+}
+
+template <bool FIN, bool SEGS, int BATCH>
+__global__ void __launch_bounds__(128) merge_kernel(CacheView cv, int Hq, int G, int NHG, int nq,
+                                                    int64_t NW, const float *ws, int64_t ws_floats,
+                                                    float *out) {
+    merge_entry<FIN, SEGS, BATCH>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
+}
+
+// The whole-group merge capped at 72 registers, so that 7 blocks fit an SM
+// instead of 6.  It is taken when the grid is more than one wave of the
+// uncapped kernel (a batch of 16 x 64 query heads: 1024 blocks, 1.15 waves
+// uncapped, 0.99 capped); smaller grids keep the uncapped kernel, which does
+// not spill.
+template <bool FIN, int BATCH>
+__global__ void __launch_bounds__(128, 7) merge_kernel_capped(CacheView cv, int Hq, int G, int NHG,
+                                                              int nq, int64_t NW, const float *ws,
+                                                              int64_t ws_floats, float *out) {
+    merge_entry<FIN, false, BATCH>(cv, Hq, G, NHG, nq, NW, ws, ws_floats, out);
 }
 
 // ---------------------------------------------------------------------------
@@ -1773,6 +1791,28 @@ static cudaError_t current_device(int *dev) {
     cudaError_t e = cudaGetDevice(dev);
     if (e != cudaSuccess) return e;
     return (*dev < 0 || *dev >= kMaxDevices) ? cudaErrorInvalidDevice : cudaSuccess;
+}
+
+// how many blocks of the uncapped whole-group merge the current device holds
+// at once (resident blocks per SM x SMs), cached per device
+static cudaError_t merge_wave(int64_t *blocks) {
+    static std::atomic<int64_t> wave_of[kMaxDevices];  // 0: not queried yet
+    int dev;
+    cudaError_t e = current_device(&dev);
+    if (e != cudaSuccess) return e;
+    int64_t w = wave_of[dev].load(std::memory_order_acquire);
+    if (w == 0) {
+        int per_sm = 0, nsm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &per_sm, merge_kernel<false, false, DKV_MERGE_BATCH>, 128, 0);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        w = (int64_t)(per_sm < 1 ? 1 : per_sm) * nsm;
+        wave_of[dev].store(w, std::memory_order_release);
+    }
+    *blocks = w;
+    return cudaSuccess;
 }
 
 template <int FMT, int MODE, bool ZT>
@@ -1965,12 +2005,21 @@ cudaError_t launch_merge(const CacheView &cv, int Hq, int nq, float *out, const 
         else
             e = launch_pdl(merge_kernel<false, true, DKV_MERGE_BATCH>, grid, dim3(128), fl, st,
                            cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out);
-    } else if (cv.len_add > 0) {
-        e = launch_pdl(merge_kernel<true, false, DKV_MERGE_BATCH>, grid, dim3(128), 0, st,
-                       cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out);
     } else {
-        e = launch_pdl(merge_kernel<false, false, DKV_MERGE_BATCH>, grid, dim3(128), 0, st,
-                       cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out);
+        int64_t wave = 0;
+        e = merge_wave(&wave);
+        if (e != cudaSuccess) return e;
+        const bool cap = (int64_t)grid.x * grid.y > wave;
+        if (cv.len_add > 0)
+            e = cap ? launch_pdl(merge_kernel_capped<true, DKV_MERGE_BATCH>, grid, dim3(128), 0,
+                                 st, cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out)
+                    : launch_pdl(merge_kernel<true, false, DKV_MERGE_BATCH>, grid, dim3(128), 0, st,
+                                 cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out);
+        else
+            e = cap ? launch_pdl(merge_kernel_capped<false, DKV_MERGE_BATCH>, grid, dim3(128), 0,
+                                 st, cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out)
+                    : launch_pdl(merge_kernel<false, false, DKV_MERGE_BATCH>, grid, dim3(128), 0, st,
+                                 cv, Hq, G, NHG, nq, NW, (const float *)ws, ws_floats, out);
     }
     return e;
 }
