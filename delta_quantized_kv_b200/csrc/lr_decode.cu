@@ -27,7 +27,9 @@
 //     per chunk; then out = the merged delta part + sum_r W_r v^_r, one block
 //     per head.
 // Inputs are the canonical layouts dkv_lr_encode writes.
+#include <atomic>
 #include <cstdint>
+#include <mutex>
 
 #include "dkv_common.cuh"
 #include "dkv_internal.h"
@@ -79,6 +81,8 @@ __device__ inline float lrd_q(const LrdArgs &a, int64_t i) {
 //    lanes hold channels 4 lane .. 4 lane + 3, binary32 products in order.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(LRD_WARPS * 32) lrd_refdot_kernel(LrdArgs a) {
+    pdl_trigger();
+    pdl_wait();           // every global access below follows the previous kernel
     const int seq = blockIdx.y, b = seq / a.Hkv, kvh = seq % a.Hkv;
     const int lane = threadIdx.x & 31;
     const int nr = (lrd_len(a, b) + a.s - 1) / a.s;
@@ -161,6 +165,8 @@ __device__ inline float2 lrd_refpart(const LrdArgs &a, int seq, int p, int h0) {
 // 1b. The reference part of every token's score, into S (the split kernel
 //     adds the token's own residual dot): one thread per (token, head pair).
 __global__ void __launch_bounds__(256) lrd_refmean_kernel(LrdArgs a) {
+    pdl_trigger();
+    pdl_wait();           // every global access below follows the previous kernel
     const int seq = blockIdx.y, b = seq / a.Hkv;
     const int len = lrd_len(a, b);
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // token * 4 + head pair
@@ -180,6 +186,8 @@ __global__ void __launch_bounds__(256) lrd_refmean_kernel(LrdArgs a) {
 template <bool QHL>
 __global__ void __launch_bounds__(LRD_WARPS * 32) lrd_split_kernel(LrdArgs a) {
     extern __shared__ __align__(128) uint8_t lrd_smem[];
+    pdl_trigger();
+    pdl_wait();           // every global access below follows the previous kernel
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, tq = lane & 3;
     const int64_t item = (int64_t)blockIdx.x * LRD_WARPS + warp;
@@ -382,6 +390,8 @@ constexpr int LRD_WEIGHT_THREADS = 256;
 
 __global__ void __launch_bounds__(LRD_WEIGHT_THREADS) lrd_weights_kernel(LrdArgs a) {
     __shared__ float Mh[8], Lh[8];
+    pdl_trigger();
+    pdl_wait();           // every global access below follows the previous kernel
     const int chunk = blockIdx.x, seq = blockIdx.y, b = seq / a.Hkv;
     const int len = lrd_len(a, b);
     const int pb = chunk * a.chunk, pe = min(len, pb + a.chunk);
@@ -418,6 +428,8 @@ template <bool WSM>
 __global__ void __launch_bounds__(D) lrd_out_kernel(LrdArgs a) {
     extern __shared__ float w_sm[];                         // WSM: [NR]
     __shared__ float Ms, Ls;
+    pdl_trigger();
+    pdl_wait();           // every global access below follows the previous kernel
     const int h = blockIdx.x, seq = blockIdx.y, b = seq / a.Hkv, kvh = seq % a.Hkv;
     const int len = lrd_len(a, b), c = threadIdx.x;
     float *out = a.out + ((int64_t)b * a.Hq + kvh * a.G + h) * D;
@@ -460,6 +472,43 @@ size_t lrd_workspace_floats(int B, int Hkv, int T, int s) {
     return (size_t)(nseq * NR * 8 * 2 + nseq * (int64_t)T * 8 + nseq * nch * LRD_PARTIAL);
 }
 
+
+// The split kernel's resident warps on the current device (its shared-memory
+// attribute is set on the first call), cached per device and query variant.
+constexpr size_t kLrdSplitSmem = (size_t)LRD_WARPS * 2 * LRD_TILE * LRD_ROW * sizeof(__half);
+constexpr int kLrdMaxDevices = 64;
+static std::mutex g_lrd_mu;
+
+static cudaError_t lrd_split_resident(bool qhl, int64_t *resident) {
+    static std::atomic<int64_t> res_of[2][kLrdMaxDevices];   // 0: not computed yet
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kLrdMaxDevices) return cudaErrorInvalidDevice;
+    int64_t r = res_of[qhl][dev].load(std::memory_order_acquire);
+    if (r == 0) {
+        std::lock_guard<std::mutex> lock(g_lrd_mu);
+        r = res_of[qhl][dev].load(std::memory_order_relaxed);
+        if (r == 0) {
+            const void *fn = qhl ? (const void *)lrd_split_kernel<true>
+                                 : (const void *)lrd_split_kernel<false>;
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kLrdSplitSmem);
+            if (e != cudaSuccess) return e;
+            int per_sm = 0, nsm = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, LRD_WARPS * 32,
+                                                              kLrdSplitSmem);
+            if (e != cudaSuccess) return e;
+            e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            r = (int64_t)(per_sm < 1 ? 1 : per_sm) * nsm * LRD_WARPS;
+            res_of[qhl][dev].store(r, std::memory_order_release);
+        }
+    }
+    *resident = r;
+    return cudaSuccess;
+}
+
 cudaError_t launch_lr_decode(const LrdView &K, const LrdView &V, int B, int Hkv, int T, int s,
                              int m, const int32_t *lens, const void *Q, int q_dtype, int Hq,
                              float softmax_scale, float *out, float *ws, cudaStream_t st) {
@@ -477,27 +526,18 @@ cudaError_t launch_lr_decode(const LrdView &K, const LrdView &V, int B, int Hkv,
     a.part = a.S + nseq * (int64_t)T * 8;
     a.out = out;
     dim3 g1((unsigned)min(1024, (a.NR + LRD_WARPS - 1) / LRD_WARPS), (unsigned)nseq);
-    lrd_refdot_kernel<<<g1, LRD_WARPS * 32, 0, st>>>(a);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(lrd_refdot_kernel, g1, dim3(LRD_WARPS * 32), 0, st, a);
     if (e != cudaSuccess) return e;
     dim3 g2((unsigned)(((int64_t)T * 4 + 255) / 256), (unsigned)nseq);
-    lrd_refmean_kernel<<<g2, 256, 0, st>>>(a);
-    e = cudaGetLastError();
+    e = launch_pdl(lrd_refmean_kernel, g2, dim3(256), 0, st, a);
     if (e != cudaSuccess) return e;
     // chunks sized so that the split grid fills one wave of resident warps:
     // chunks per sequence = resident warps / sequences, whole 32-token tiles,
     // at least LRD_CHUNK_MIN tokens (the workspace is sized for that)
-    const size_t smem = (size_t)LRD_WARPS * 2 * LRD_TILE * LRD_ROW * sizeof(__half);
-    const void *split_fn = q_dtype == DKV_F32 ? (const void *)lrd_split_kernel<true>
-                                              : (const void *)lrd_split_kernel<false>;
-    e = cudaFuncSetAttribute(split_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = kLrdSplitSmem;
+    int64_t resident = 0;
+    e = lrd_split_resident(q_dtype == DKV_F32, &resident);
     if (e != cudaSuccess) return e;
-    int per_sm = 0, dev = 0, nsm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_fn, LRD_WARPS * 32, smem);
-    if (e == cudaSuccess) e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    const int64_t resident = (int64_t)(per_sm < 1 ? 1 : per_sm) * nsm * LRD_WARPS;
     const int64_t per_seq = resident / nseq > 1 ? resident / nseq : 1;
     int64_t chunk = (T + per_seq - 1) / per_seq;
     chunk = (chunk + LRD_TILE - 1) / LRD_TILE * LRD_TILE;
@@ -505,21 +545,19 @@ cudaError_t launch_lr_decode(const LrdView &K, const LrdView &V, int B, int Hkv,
     a.n_chunks = (T + a.chunk - 1) / a.chunk;
     const int64_t warps = nseq * a.n_chunks;
     const unsigned ctas = (unsigned)((warps + LRD_WARPS - 1) / LRD_WARPS);
-    if (q_dtype == DKV_F32)
-        lrd_split_kernel<true><<<ctas, LRD_WARPS * 32, smem, st>>>(a);
-    else
-        lrd_split_kernel<false><<<ctas, LRD_WARPS * 32, smem, st>>>(a);
-    e = cudaGetLastError();
+    e = q_dtype == DKV_F32
+            ? launch_pdl(lrd_split_kernel<true>, dim3(ctas), dim3(LRD_WARPS * 32), smem, st, a)
+            : launch_pdl(lrd_split_kernel<false>, dim3(ctas), dim3(LRD_WARPS * 32), smem, st, a);
     if (e != cudaSuccess) return e;
-    lrd_weights_kernel<<<dim3((unsigned)a.n_chunks, (unsigned)nseq), LRD_WEIGHT_THREADS, 0, st>>>(a);
-    e = cudaGetLastError();
+    e = launch_pdl(lrd_weights_kernel, dim3((unsigned)a.n_chunks, (unsigned)nseq),
+                   dim3(LRD_WEIGHT_THREADS), 0, st, a);
     if (e != cudaSuccess) return e;
     const size_t wsm = (size_t)a.NR * sizeof(float);
-    if (wsm <= (size_t)LRD_W_SMEM_MAX)
-        lrd_out_kernel<true><<<dim3((unsigned)a.G, (unsigned)nseq), D, wsm, st>>>(a);
-    else
-        lrd_out_kernel<false><<<dim3((unsigned)a.G, (unsigned)nseq), D, 0, st>>>(a);
-    return cudaGetLastError();
+    return wsm <= (size_t)LRD_W_SMEM_MAX
+               ? launch_pdl(lrd_out_kernel<true>, dim3((unsigned)a.G, (unsigned)nseq), dim3(D), wsm,
+                            st, a)
+               : launch_pdl(lrd_out_kernel<false>, dim3((unsigned)a.G, (unsigned)nseq), dim3(D), 0,
+                            st, a);
 }
 
 }  // namespace dkv
