@@ -463,11 +463,13 @@ def lr_decode_bench(dev, T=4096, stride=32, n_refs=1, n_iter=10):
         run()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(n_iter):
-        run()
-    e1.record(st)
-    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.synchronize()
+        e0.record(st)
+        for _ in range(n_iter):
+            run()
+        e1.record(st)
+        torch.cuda.synchronize()
     t_lr = e0.elapsed_time(e1) / n_iter
     nr = -(-T // stride)
     lr_bytes = B * Hkv * 2 * (T * (D + 8 + 4 * n_refs) + nr * 2 * D)
@@ -490,7 +492,7 @@ def lr_decode_bench(dev, T=4096, stride=32, n_refs=1, n_iter=10):
             "lr_gbps": lr_bytes / (t_lr * 1e-3) / 1e9,
             "delta_step_us": 1e3 * t_d, "delta_bytes": d_bytes,
             "delta_gbps": d_bytes / (t_d * 1e-3) / 1e9,
-            "max_row_rel_diff_lr_vs_delta": diff}
+            "max_row_rel_diff_lr_vs_delta": diff, "launches": n_iter, "clocks": clk.summary()}
 
 
 # ---------------------------------------------------------------------------
@@ -782,6 +784,10 @@ def run_ours(args, w, rank, world, local):
         with sampler:
             torch.cuda.synchronize()
             barrier(world)
+            # ~1 ms of GPU spin ahead of the timed region, so the host has
+            # queued every replay before the first one runs: a host stall
+            # cannot leave the GPU idle inside the region
+            torch.cuda._sleep(2_000_000)
             e0.record(stream)
             for k in range(K):
                 graphs[W + k].replay()
@@ -843,6 +849,19 @@ def run_ours(args, w, rank, world, local):
 
     # ---- comparators and MSE (rank 0 only, outside the timed region) ----------
     extra = {}
+    def timed_loop(fn, n):
+        """Mean event time of n back-to-back calls (ms), and the SM clocks
+        sampled meanwhile."""
+        with ClockSampler(local) as clk_c:
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(n):
+                fn(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n, clk_c.summary()
+
     if rank == 0 and args.comparators and args.fmt == "delta":
         for fmt in ("fp16", "q4"):
             cc = dkv.Cache(B, Hkv, T0, fmt, kf=w.kf, device=dev)
@@ -850,19 +869,12 @@ def run_ours(args, w, rank, world, local):
             wsc = cc.workspace(Hq)
             for _ in range(3):
                 cc.decode_attn(qs[0], scale, out=out)
-            torch.cuda.synchronize()
-            a, bq = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            n = max(5, K)
-            a.record(stream)
-            for i in range(n):
-                dkv.dkv_decode_attn_split(cc.c, qs[i % len(qs)], qcode, Hq, scale, wsc,
-                                          wsc.numel() * 4, stream)
-            bq.record(stream)
-            torch.cuda.synchronize()
-            t = a.elapsed_time(bq) / n
+            n = max(20, K)
+            t, clk_c = timed_loop(lambda i: dkv.dkv_decode_attn_split(
+                cc.c, qs[i % len(qs)], qcode, Hq, scale, wsc, wsc.numel() * 4, stream), n)
             nb = kv_bytes(fmt, [T0] * B, Hkv, w.kf)
             extra[fmt] = {"split_us": 1e3 * t, "bytes": nb, "gbps": nb / (t * 1e-3) / 1e9,
-                          "speedup_delta_vs": t / split_plain}
+                          "speedup_delta_vs": t / split_plain, "launches": n, "clocks": clk_c}
             del cc
         # the same decode through a paged cache: pages of 16 groups (512 tokens)
         # in a shuffled pool, every record reached through the block table
@@ -872,20 +884,14 @@ def run_ours(args, w, rank, world, local):
             wsp = cp.workspace(Hq)
             for _ in range(3):
                 cp.decode_attn(qs[0], scale, out=out)
-            torch.cuda.synchronize()
-            a, bq = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            n = max(5, K)
-            a.record(stream)
-            for i in range(n):
-                dkv.dkv_decode_attn_split(cp.c, qs[i % len(qs)], qcode, Hq, scale, wsp,
-                                          wsp.numel() * 4, stream)
-            bq.record(stream)
-            torch.cuda.synchronize()
-            t = a.elapsed_time(bq) / n
+            n = max(20, K)
+            t, clk_c = timed_loop(lambda i: dkv.dkv_decode_attn_split(
+                cp.c, qs[i % len(qs)], qcode, Hq, scale, wsp, wsp.numel() * 4, stream), n)
             nb = kv_bytes("delta", [T0] * B, Hkv, w.kf)
             extra["delta_paged_16_groups"] = {"split_us": 1e3 * t, "bytes": nb,
                                               "gbps": nb / (t * 1e-3) / 1e9,
-                                              "status": cp.device_status()}
+                                              "status": cp.device_status(), "launches": n,
+                                              "clocks": clk_c}
             del cp
         # multi-query decode: 2 queries per sequence (speculative decoding), G = 8,
         # so 16 virtual heads per kv head in two groups of 8 (the cache is read
@@ -897,18 +903,12 @@ def run_ours(args, w, rank, world, local):
             out2 = torch.empty((B, nq, Hq, D), dtype=torch.float32, device=dev)
             for _ in range(3):
                 cache.decode_attn_mq(Q2, scale, out=out2)
-            torch.cuda.synchronize()
-            a, bq = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            n = max(5, K)
-            a.record(stream)
-            for i in range(n):
-                cache.decode_attn_mq(Q2, scale, out=out2)
-            bq.record(stream)
-            torch.cuda.synchronize()
-            t = a.elapsed_time(bq) / n
+            n = max(20, K)
+            t, clk_c = timed_loop(lambda i: cache.decode_attn_mq(Q2, scale, out=out2), n)
             nb = kv_bytes("delta", [T0 + n_tok] * B, Hkv, w.kf)
             extra["delta_2_queries"] = {"decode_attn_us": 1e3 * t, "bytes": nb,
-                                        "gbps": nb / (t * 1e-3) / 1e9}
+                                        "gbps": nb / (t * 1e-3) / 1e9, "launches": n,
+                                        "clocks": clk_c}
         # reconstruction MSE on a slice (first 2 batch entries)
         nb_ = min(2, B)
         xs = {"K": Kp[:nb_].float(), "V": Vp[:nb_].float()}
