@@ -25,10 +25,11 @@
  *    the stream it is given).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call is asynchronous on that stream.  The append,
- *    decode-split and merge kernels are launched with programmatic stream
- *    serialization: one may be scheduled while the kernel before it on the
- *    stream is finishing, but it waits for that kernel to complete before its
- *    first global memory access, so stream order holds for all memory.
+ *    decode-split and merge kernels, and the long-range decode's kernels, are
+ *    launched with programmatic stream serialization: one may be scheduled
+ *    while the kernel before it on the stream is finishing, but it waits for
+ *    that kernel to complete before its first global memory access, so stream
+ *    order holds for all memory.
  *  - Host-side validation happens before any launch; a failed check returns
  *    an error and launches nothing.  Device pointers must be 16-byte aligned
  *    (DKV_EALIGN otherwise); the cache base must be 256-byte aligned.
