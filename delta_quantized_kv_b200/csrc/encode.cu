@@ -76,9 +76,25 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
     const int b = blockIdx.z, kvh = blockIdx.y >> 1, t = blockIdx.y & 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = warp * 32 + lane;
+    const void *src = t == 0 ? a.K : a.V;
+    const int64_t in_base = (((int64_t)b * cv.Hkv + kvh) * a.T_in) * D;
+    // An append of a few tokens is latency-bound.  The first input row and
+    // both state slots do not depend on the length or on the slot parity, so
+    // they are loaded together with those (all in bounds by construction: b,
+    // kvh and t index their arrays, and an append has T_in >= 1).
+    constexpr bool PF = FMT == DKV_FMT_DELTA && !DKV_CHECKED;
+    const int64_t slot = (((int64_t)b * cv.Hkv + kvh) * 2 + t) * D + c;
+    const int64_t slot_stride = (int64_t)cv.B * cv.Hkv * 2 * D;
+    float x_first = 0.f, st_pf[2] = {0.f, 0.f};
+    if (PF && a.append) {
+        x_first = load_in(src, a.dtype, in_base + c);
+        st_pf[0] = cv.state[slot];
+        st_pf[1] = cv.state[slot + slot_stride];
+    }
     const int parity = cv.header[2] & 1;
     float *state_old = cv.state + ((((int64_t)parity * cv.B + b) * cv.Hkv + kvh) * 2 + t) * D;
     float *state_new = cv.state + ((((int64_t)(parity ^ 1) * cv.B + b) * cv.Hkv + kvh) * 2 + t) * D;
+    const float st_old = (PF && a.append) ? st_pf[parity] : 0.f;   // state_old[c] when PF
 
     int start, n;
     encode_range(a, b, start, n);
@@ -86,10 +102,8 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
     if (n < 0 && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         set_status(cv.header, n == -2 ? DKV_DEV_CAPACITY : DKV_DEV_BAD_SEQLEN);
     if (n <= 0 && blockIdx.x == 0 && FMT == DKV_FMT_DELTA)
-        state_new[c] = a.append ? state_old[c] : 0.0f;  // carry the state over
+        state_new[c] = a.append ? (PF ? st_old : state_old[c]) : 0.0f;  // carry the state over
 
-    const void *src = t == 0 ? a.K : a.V;
-    const int64_t in_base = (((int64_t)b * cv.Hkv + kvh) * a.T_in) * D;
     uint8_t *sb = seq_base(cv, b, kvh);
     // checked build (block-uniform): this sequence's state rows, its n input
     // rows and, for the comparators, its data
@@ -112,18 +126,21 @@ __global__ void __launch_bounds__(128) encode_kernel(EncodeArgs a) {
             if (p0 < p1 && !rec) {
                 // bad block-table entry (flagged by rec_ptr): nothing written;
                 // the state carries over
-                if (p1 == start + n) state_new[c] = (p0 % kf) ? state_old[c] : 0.0f;
+                if (p1 == start + n)
+                    state_new[c] = (p0 % kf) ? ((PF && a.append) ? st_old : state_old[c]) : 0.0f;
             } else if (p0 < p1) {
                 uint8_t *sc_base = rec + KF_BYTES;
                 uint8_t *nib_base = rec + KF_BYTES + (int64_t)(kf - 1) * SC_BYTES +
                                     (int64_t)t * (kf - 1) * NIB_BYTES;
-                float xh = (p0 % kf) ? state_old[c] : 0.0f;
+                float xh = (p0 % kf) ? ((PF && a.append) ? st_old : state_old[c]) : 0.0f;
                 for (int cb = p0; cb < p1; cb += SEG) {
                     const int ce = min(p1, cb + SEG);
                     // first delta index and count of delta positions in [cb, ce)
                     int first_delta = -1, nd = 0;
                     for (int p = cb; p < ce; ++p) {
-                        float x = load_in(src, a.dtype, in_base + (int64_t)(p - start) * D + c);
+                        const float x = (PF && a.append && p == start)
+                                            ? x_first
+                                            : load_in(src, a.dtype, in_base + (int64_t)(p - start) * D + c);
                         if (p % kf == 0) {
                             __half h = __float2half_rn(x);
                             int idx = t == 0 ? k_half_idx(c) : v_half_idx(c);
