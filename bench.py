@@ -1012,7 +1012,7 @@ def run_ours(args, w, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
-def main(argv=None):
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -1035,7 +1035,11 @@ def main(argv=None):
         # workloads, comparator formats, quality report) and the host-core
         # oracle baseline belong to the single-GPU run only
         args.cpu_baseline = args.comparators = args.configs = False
+    return args
 
+
+def main(argv=None):
+    args = parse_args(argv)
     import synthetic as S
     w = S.WORKLOADS[args.workload]
     if args.kf:

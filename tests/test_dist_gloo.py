@@ -152,3 +152,18 @@ def test_quality_report_arithmetic_against_numpy():
             assert got["D_V"] == pytest.approx(dv, rel=2e-2, abs=1e-12), (name, fmt)
         assert rep[name]["entries"] == 1
         assert rep[name]["delta"]["rel_mse"] < rep[name]["q4"]["rel_mse"]
+
+
+def test_multi_gpu_runs_only_the_timed_step(monkeypatch):
+    """Under torchrun with N > 1 replicas the untimed extras (other workloads,
+    comparator formats, quality report) and the host-core oracle baseline are
+    switched off, so rank 0 does not hold N GPUs alone; at N = 1 they stay on."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    one = bench.parse_args([])
+    assert one.cpu_baseline and one.comparators and one.configs
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    two = bench.parse_args(["--steps", "7", "--warmup", "1"])
+    assert not (two.cpu_baseline or two.comparators or two.configs)
+    assert two.steps == 7 and two.warmup == 3      # at least 3 warm-up steps
